@@ -1,0 +1,132 @@
+"""Python binding over the C ABI (argument marshalling only).
+
+torch provides device memory and the current CUDA stream; every step of the
+computation runs in the library's kernels.  Functions mirror include/fa.h:
+
+* ``fwd(q, k, v, causal, scale)``            -> (o, lse)
+* ``bwd(q, k, v, o, do, lse, causal, scale)`` -> (dq, dk, dv)
+* ``quant_fp8(x, signs=None)``               -> (x8 as uint8, block scales)
+* ``fwd_fp8(q8, k8, v8, sq, sk, sv, causal, scale)`` -> (o, lse)
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import torch
+
+from ._lib import check, lib
+
+__all__ = ["fwd", "bwd", "bwd_workspace_size", "quant_fp8", "fwd_fp8", "get_status",
+           "clear_status", "n_blocks"]
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _check_bhnd(name: str, t: torch.Tensor, dtype, shape=None) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != 4 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous [B, H, N, d] tensor")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def n_blocks(N: int) -> int:
+    """Number of 128-row quantisation blocks of a length-N sequence."""
+    return (N + 127) // 128
+
+
+def fwd(q, k, v, causal: bool = False, scale: Optional[float] = None, out=None, lse=None):
+    """Exact attention forward (bf16).  Returns (o bf16 [B,H,N,d], lse fp32 [B,H,N])."""
+    _check_bhnd("q", q, torch.bfloat16)
+    B, H, N, d = q.shape
+    _check_bhnd("k", k, torch.bfloat16, q.shape)
+    _check_bhnd("v", v, torch.bfloat16, q.shape)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = torch.empty_like(q) if out is None else out
+    lse_t = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    code = lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), B, H, N, d, float(scale),
+                        int(bool(causal)), _stream())
+    check("fa_fwd", code)
+    return o, lse_t
+
+
+def bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(lib().fa_bwd_workspace_size(B, H, N, d))
+
+
+def bwd(q, k, v, o, do, lse, causal: bool = False, scale: Optional[float] = None,
+        workspace: Optional[torch.Tensor] = None, dq=None, dk=None, dv=None):
+    """Attention backward (bf16).  Returns (dq, dk, dv)."""
+    _check_bhnd("q", q, torch.bfloat16)
+    B, H, N, d = q.shape
+    for name, t in (("k", k), ("v", v), ("o", o), ("do", do)):
+        _check_bhnd(name, t, torch.bfloat16, q.shape)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [B, H, N] tensor")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    ws_bytes = bwd_workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    code = lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
+                        _ptr(dk), _ptr(dv), B, H, N, d, float(scale), int(bool(causal)),
+                        _ptr(workspace), workspace.numel(), _stream())
+    check("fa_bwd", code)
+    return dq, dk, dv
+
+
+def quant_fp8(x, signs: Optional[torch.Tensor] = None, out=None, scales=None):
+    """Per-128-row E4M3 quantisation.  Returns (codes uint8 [B,H,N,d], scales fp32 [B,H,nblk])."""
+    _check_bhnd("x", x, torch.bfloat16)
+    B, H, N, d = x.shape
+    if signs is not None:
+        if signs.dtype != torch.float32 or signs.numel() != d or not signs.is_cuda:
+            raise ValueError("signs must be a CUDA fp32 tensor of d elements")
+        signs = signs.contiguous()
+    x8 = torch.empty((B, H, N, d), dtype=torch.uint8, device=x.device) if out is None else out
+    sc = torch.empty((B, H, n_blocks(N)), dtype=torch.float32, device=x.device) if scales is None else scales
+    code = lib().fa_quant_fp8(_ptr(x), _ptr(x8), _ptr(sc), B, H, N, d, _ptr(signs), _stream())
+    check("fa_quant_fp8", code)
+    return x8, sc
+
+
+def fwd_fp8(q8, k8, v8, sq, sk, sv, causal: bool = False, scale: Optional[float] = None,
+            out=None, lse=None):
+    """FP8 attention forward on quantised inputs.  Returns (o bf16, lse fp32)."""
+    _check_bhnd("q8", q8, torch.uint8)
+    B, H, N, d = q8.shape
+    _check_bhnd("k8", k8, torch.uint8, q8.shape)
+    _check_bhnd("v8", v8, torch.uint8, q8.shape)
+    for name, s in (("sq", sq), ("sk", sk), ("sv", sv)):
+        if s.dtype != torch.float32 or tuple(s.shape) != (B, H, n_blocks(N)) or not s.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous fp32 [B, H, ceil(N/128)] tensor")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q8.device) if out is None else out
+    lse_t = torch.empty((B, H, N), dtype=torch.float32, device=q8.device) if lse is None else lse
+    code = lib().fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk), _ptr(sv), _ptr(o),
+                            _ptr(lse_t), B, H, N, d, float(scale), int(bool(causal)), _stream())
+    check("fa_fwd_fp8", code)
+    return o, lse_t
+
+
+def get_status() -> int:
+    return int(lib().fa_get_status())
+
+
+def clear_status() -> None:
+    lib().fa_clear_status()

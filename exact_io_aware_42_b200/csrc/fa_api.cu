@@ -1,0 +1,197 @@
+// C-ABI layer: argument validation, TMA tensor-map encoding, the device
+// status word, and dispatch to the kernels.  See include/fa.h for the
+// contract of each entry point.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_internal.h"
+
+namespace fa {
+
+// First in-kernel failure since the last fa_clear_status (one word per device).
+__device__ unsigned int g_status = 0;
+
+namespace {
+
+constexpr int kMaxN = 1 << 20;
+constexpr int kMaxBH = 1 << 20;
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool probed = false;
+  bool ok = false;
+  unsigned int* status = nullptr;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// Current device checked once: sm_100 present, status-word address, driver
+// entry point for tensor-map encoding.
+fa_status current_device(DeviceInfo** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return FA_ERR_NO_DEVICE;
+  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.probed) {
+    di.probed = true;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_NO_DEVICE;
+    }
+    if (major != 10 || minor != 0) return FA_ERR_UNSUPPORTED;
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_status) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_NO_DEVICE;
+    }
+    di.status = static_cast<unsigned int*>(addr);
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                           &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr) {
+        cudaGetLastError();
+        return FA_ERR_NO_DEVICE;
+      }
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    di.ok = true;
+  }
+  if (!di.ok) return FA_ERR_UNSUPPORTED;
+  *out = &di;
+  return FA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 3-D view [BH, N, d] of a contiguous [B, H, N, d] tensor, 128-byte swizzle,
+// box {box_inner elements, box_rows, 1}; out-of-range elements read as zero
+// and are skipped on store.
+bool encode_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, int d, int N,
+               int BH, int box_inner, int box_rows) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * esize,
+                           static_cast<cuuint64_t>(N) * d * esize};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+fa_status check_shape(int B, int H, int N, int d, float scale) {
+  if (B < 0 || H < 0 || N < 0) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale < 0.f) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (N > kMaxN || static_cast<long long>(B) * H > kMaxBH) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+}  // namespace
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                            int B, int H, int N, int d, float scale, int causal, void* stream) {
+  fa_status st = check_shape(B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  if (static_cast<long long>(B) * H * N == 0) return FA_OK;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return FA_ERR_MISALIGNED;
+  DeviceInfo* di = nullptr;
+  if ((st = current_device(&di)) != FA_OK) return st;
+
+  FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  const int BH = B * H;
+  const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!encode_3d(&p.tm_q, q, bf, 2, d, N, BH, 64, kBlockM) ||
+      !encode_3d(&p.tm_k, k, bf, 2, d, N, BH, 64, kBlockN) ||
+      !encode_3d(&p.tm_v, v, bf, 2, d, N, BH, 64, kBlockN) ||
+      !encode_3d(&p.tm_o, o, bf, 2, d, N, BH, 64, kBlockM))
+    return FA_ERR_INVALID_ARG;
+  p.lse = lse;
+  p.status = di->status;
+  p.N = N;
+  p.BH = BH;
+  p.n_kv = (N + kBlockN - 1) / kBlockN;
+  p.n_pairs = ((N + kBlockM - 1) / kBlockM + 1) / 2;
+  p.scale = scale;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  cudaError_t e = launch_fwd_bf16(p, d, causal != 0, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+  }
+  return FA_OK;
+}
+
+extern "C" size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (B < 0 || H < 0 || N < 0 || (d != 64 && d != 128)) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  return up(rows * d * sizeof(float)) + up(rows * sizeof(float));
+}
+
+extern "C" fa_status fa_bwd(const void*, const void*, const void*, const void*, const void*,
+                            const float*, void*, void*, void*, int, int, int, int, float, int,
+                            void*, size_t, void*) {
+  return FA_ERR_UNSUPPORTED;
+}
+
+extern "C" fa_status fa_quant_fp8(const void*, void*, float*, int, int, int, int, const float*,
+                                  void*) {
+  return FA_ERR_UNSUPPORTED;
+}
+
+extern "C" fa_status fa_fwd_fp8(const void*, const void*, const void*, const float*,
+                                const float*, const float*, void*, float*, int, int, int, int,
+                                float, int, void*) {
+  return FA_ERR_UNSUPPORTED;
+}
+
+extern "C" unsigned int fa_get_status(void) {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, fa::g_status, sizeof(v)) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_NO_DEVICE;
+  }
+  return v;
+}
+
+extern "C" void fa_clear_status(void) {
+  const unsigned int z = 0;
+  if (cudaMemcpyToSymbol(fa::g_status, &z, sizeof(z)) != cudaSuccess) cudaGetLastError();
+}
+
+extern "C" const char* fa_status_string(int s) {
+  switch (s & 0xFF) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    case FA_ERR_LAUNCH: return "FA_ERR_LAUNCH";
+    case FA_ERR_PIPELINE_TIMEOUT: return "FA_ERR_PIPELINE_TIMEOUT";
+    case FA_ERR_NO_DEVICE: return "FA_ERR_NO_DEVICE";
+    default: return "FA_ERR_UNKNOWN";
+  }
+}

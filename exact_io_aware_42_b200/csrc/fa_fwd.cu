@@ -1,0 +1,402 @@
+// Fused exact attention forward for sm_100a (bf16 in, fp32 accumulate).
+//
+// What it computes: O = softmax(scale * Q K^T [causal]) V and the per-row
+// logsumexp L, exactly as the standard definition ("FlashAttention" concept
+// note, "How it works"), reached by the online softmax of "FlashAttention
+// v1/v2/v3/v4: the librarian who never clears the desk" (online softmax
+// section, eq. 2): per K/V tile the running max m and sum l are updated, the
+// running output is rescaled by 2^(m_old - m_new), and the division by l is
+// deferred to the end (lineage page, "FA2 (2023)", refinement 2).
+//
+// Work unit: one CTA owns two 128-row query tiles of one (b, h) and streams
+// every needed 128-key K/V tile once for both (each K/V tile is read from
+// L2/HBM once per 256 query rows).  Roles:
+//   warps 0-3  softmax for query tile 0 (thread r owns row r = TMEM lane r)
+//   warps 4-7  softmax for query tile 1
+//   warp  8    TMA producer: Q tiles, then K_0, V_0, K_1, V_1, ... into a
+//              ring of 128 x d shared-memory tiles (full/empty mbarriers)
+//   warp  9    allocates TMEM; one thread issues every tcgen05.mma
+// TMEM (512 columns x 128 lanes, fp32):
+//   [0,128)    S_0 (tile 0 scores); after softmax the first 64 columns hold
+//              P_0 as packed bf16 pairs, read back as the A operand of P V
+//   [128,256)  S_1 / P_1
+//   [256,256+d)        O_0 accumulator
+//   [256+d,256+2d)     O_1 accumulator
+// MMA order per key tile j:  PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), so each
+// softmax warpgroup works on its tile while the tensor core runs the other
+// tile's two products (the lineage page's "pingpong" idea, "FA3 (2024)",
+// carried by two TMEM-resident tiles instead of two register warpgroups).
+//
+// Conditional rescaling (librarian page, "FA4", idea 2): a row keeps its
+// stale max m until a new tile's max exceeds it by more than kRescaleTau
+// (log2 units).  p = 2^(x - m) is then at most 2^tau, the same stale m is
+// used for p, l, O and L, and the result is unchanged up to rounding.  The
+// O rescale in TMEM runs only for warps where some row moved its max.
+//
+// Causal: key j visible to query i iff j <= i.  Tiles entirely above the
+// diagonal are never loaded or multiplied; only the diagonal tile and the
+// ragged key tail (keys >= N, zero-filled by TMA) are masked to -inf.
+#include "fa_ptx.cuh"
+#include "fa_internal.h"
+
+namespace fa {
+namespace {
+
+template <int D>
+struct FwdCfg {
+  static constexpr int kPanels = D / 64;             // 128-byte swizzle panels per row
+  static constexpr int kPanelBytes = 128 * 128;      // 128 rows x 128 bytes
+  static constexpr int kTileBytes = kBlockM * D * 2; // one 128 x D bf16 tile
+  static constexpr int kStages = (D == 128) ? 5 : 8;
+  static constexpr int kThreads = 320;
+  static constexpr int kOffQ = 0;                    // two query tiles
+  static constexpr int kOffRing = 2 * kTileBytes;
+  static constexpr int kOffBar = kOffRing + kStages * kTileBytes;
+  static constexpr int kNumBars = 2 + 2 * kStages + 7;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // + base alignment slack
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS = 0;       // + 128 * t
+  static constexpr uint32_t kColO = 256;     // + D * t
+};
+
+// barrier slots
+__device__ __forceinline__ int bar_q(int t) { return t; }
+template <int NS> __device__ __forceinline__ int bar_full(int s) { return 2 + s; }
+template <int NS> __device__ __forceinline__ int bar_empty(int s) { return 2 + NS + s; }
+template <int NS> __device__ __forceinline__ int bar_s(int t) { return 2 + 2 * NS + t; }
+template <int NS> __device__ __forceinline__ int bar_p(int t) { return 4 + 2 * NS + t; }
+template <int NS> __device__ __forceinline__ int bar_pv(int t) { return 6 + 2 * NS + t; }
+template <int NS> __device__ __forceinline__ int bar_drain() { return 8 + 2 * NS; }
+
+// wait-site codes reported in bits 8..15 of the status word
+enum : unsigned int { kSiteProdEmpty = 1, kSiteMmaQ, kSiteMmaFull, kSiteMmaP, kSiteSmS, kSiteSmPv,
+                      kSiteEpiPv, kSiteDrain };
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ float max4(float a, float b, float c, float d) {
+  return fmaxf(fmaxf(a, b), fmaxf(c, d));
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(320, 1) fwd_bf16_kernel(const __grid_constant__ FwdParams p) {
+  using C = FwdCfg<D>;
+  constexpr int NS = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sbase + C::kOffBar + 8 * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.x % p.BH;
+  const int pair = p.n_pairs - 1 - blockIdx.x / p.BH;   // heaviest causal pairs first
+  const int qt0 = 2 * pair;
+  int n_t[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) n_t[t] = CAUSAL ? min(qt0 + t + 1, p.n_kv) : p.n_kv;
+  const int n_iter = n_t[1];
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(bar_q(0)), 1);
+    mbar_init(bar(bar_q(1)), 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar(bar_full<NS>(s)), 1);
+      mbar_init(bar(bar_empty<NS>(s)), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(bar_s<NS>(t)), 1);
+      mbar_init(bar(bar_p<NS>(t)), 128);
+      mbar_init(bar(bar_pv<NS>(t)), 1);
+    }
+    mbar_init(bar(bar_drain<NS>()), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Abort ab{abort_flag, p.status};
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_q);
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
+      for (int t = 0; t < 2; ++t) {
+        mbar_arrive_expect_tx(bar(bar_q(t)), C::kTileBytes);
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_3d(sbase + C::kOffQ + t * C::kTileBytes + pn * C::kPanelBytes, &p.tm_q,
+                      bar(bar_q(t)), pn * 64, (qt0 + t) * kBlockM, bh);
+      }
+      int seq = 0;
+      bool ok = true;
+      for (int j = 0; j < n_iter && ok; ++j) {
+        for (int w = 0; w < 2 && ok; ++w) {
+          const int s = seq % NS;
+          const uint32_t ph = (seq / NS) & 1;
+          if (!mbar_wait(bar(bar_empty<NS>(s)), ph ^ 1, ab, kSiteProdEmpty)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(bar_full<NS>(s)), C::kTileBytes);
+          const CUtensorMap* m = (w == 0) ? &p.tm_k : &p.tm_v;
+          for (int pn = 0; pn < C::kPanels; ++pn)
+            tma_load_3d(sbase + C::kOffRing + s * C::kTileBytes + pn * C::kPanelBytes, m,
+                        bar(bar_full<NS>(s)), pn * 64, j * kBlockN, bh);
+          ++seq;
+        }
+      }
+      if (*abort_flag) {
+        // Another role gave up: let every copy this thread started land before
+        // the CTA exits (bounded, ignoring the abort flag).
+        volatile int never = 0;
+        const Abort drain{&never, p.status};
+        for (int t = 0; t < 2; ++t) mbar_wait(bar(bar_q(t)), 0, drain, kSiteDrain);
+        const int first = seq > NS ? seq - NS : 0;
+        for (int q = first; q < seq; ++q)
+          mbar_wait(bar(bar_full<NS>(q % NS)), (q / NS) & 1, drain, kSiteDrain);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t kIdescO = idesc_bf16_f32(128, D, false, true);
+      const uint32_t q_addr[2] = {sbase + C::kOffQ, sbase + C::kOffQ + C::kTileBytes};
+      auto ring = [&](int s) -> uint32_t { return sbase + C::kOffRing + s * C::kTileBytes; };
+      auto issue_s = [&](int t, uint32_t k_addr) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * C::kPanelBytes + (kk % 4) * 32;
+          const uint64_t a = smem_desc_sw128(q_addr[t] + off, 16, 1024);
+          const uint64_t b = smem_desc_sw128(k_addr + off, 16, 1024);
+          mma_f16_ss(tmem + C::kColS + 128 * t, a, b, kIdescS, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(bar_s<NS>(t)));
+      };
+      auto issue_pv = [&](int t, uint32_t v_addr, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < kBlockN / 16; ++kk) {
+          const uint64_t b = smem_desc_sw128(v_addr + kk * 16 * 128, C::kPanelBytes, 1024);
+          mma_f16_ts(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + kk * 8, b, kIdescO,
+                     (acc || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(bar(bar_pv<NS>(t)));
+      };
+      bool ok = mbar_wait(bar(bar_q(0)), 0, ab, kSiteMmaQ) && mbar_wait(bar(bar_q(1)), 0, ab, kSiteMmaQ);
+      int seq = 0;
+      int ks = 0;
+      if (ok) ok = mbar_wait(bar(bar_full<NS>(0)), 0, ab, kSiteMmaFull);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, ring(0));
+        issue_s(1, ring(0));
+        tc_commit(bar(bar_empty<NS>(0)));
+        seq = 1;
+      }
+      for (int j = 0; j < n_iter && ok; ++j) {
+        const int vs = seq % NS;
+        if (!(ok = mbar_wait(bar(bar_full<NS>(vs)), (seq / NS) & 1, ab, kSiteMmaFull))) break;
+        ++seq;
+        const bool has_next = j + 1 < n_iter;
+        if (has_next) {
+          ks = seq % NS;
+          if (!(ok = mbar_wait(bar(bar_full<NS>(ks)), (seq / NS) & 1, ab, kSiteMmaFull))) break;
+          ++seq;
+        }
+        tc_fence_after();
+        if (j < n_t[0]) {
+          if (!(ok = mbar_wait(bar(bar_p<NS>(0)), j & 1, ab, kSiteMmaP))) break;
+          tc_fence_after();
+          issue_pv(0, ring(vs), j > 0);
+          if (j + 1 < n_t[0]) issue_s(0, ring(ks));
+        }
+        if (!(ok = mbar_wait(bar(bar_p<NS>(1)), j & 1, ab, kSiteMmaP))) break;
+        tc_fence_after();
+        issue_pv(1, ring(vs), j > 0);
+        tc_commit(bar(bar_empty<NS>(vs)));
+        if (has_next) {
+          issue_s(1, ring(ks));
+          tc_commit(bar(bar_empty<NS>(ks)));
+        }
+      }
+      // Every MMA issued above must be finished before TMEM is released,
+      // also when a role gave up part-way.
+      tc_commit(bar(bar_drain<NS>()));
+      volatile int never = 0;
+      const Abort drain{&never, p.status};
+      mbar_wait(bar(bar_drain<NS>()), 0, drain, kSiteDrain);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int t = warp >> 2;                 // query tile of this warpgroup
+    const int r = threadIdx.x - 128 * t;     // row within the tile == TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + C::kColS + 128 * t + lane_off;
+    const uint32_t tO = tmem + C::kColO + D * t + lane_off;
+    const int qi = qt0 + t;
+    const int row = qi * kBlockM + r;
+    const int n = n_t[t];
+    const float c = p.scale_log2;
+    float m_use = -INFINITY;
+    float l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      if (!(ok = mbar_wait_warp(bar(bar_s<NS>(t)), j & 1, ab, kSiteSmS))) break;
+      tc_fence_after();
+      float s[128];
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t u[32];
+        tmem_ld32(tS + ch * 32, u);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[ch * 32 + i] = __uint_as_float(u[i]);
+      }
+      const bool masked = (CAUSAL && j == qi) || ((j + 1) * kBlockN > p.N);
+      float mt;
+      if (masked) {
+        const int key0 = j * kBlockN;
+#pragma unroll
+        for (int i = 0; i < 128; ++i) {
+          const int key = key0 + i;
+          const bool vis = key < p.N && (!CAUSAL || key <= row);
+          s[i] = vis ? s[i] * c : -INFINITY;
+        }
+      }
+      {
+        float m8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = s[i];
+#pragma unroll
+        for (int i = 8; i < 128; i += 8) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) m8[k] = fmaxf(m8[k], s[i + k]);
+        }
+        mt = fmaxf(max4(m8[0], m8[1], m8[2], m8[3]), max4(m8[4], m8[5], m8[6], m8[7]));
+        if (!masked) mt *= c;
+      }
+      const float m_new = fmaxf(m_use, mt);
+      const bool need = m_new > m_use + kRescaleTau;
+      float alpha = 1.f;
+      if (need) {
+        alpha = ex2_sfu(m_use - m_new);
+        m_use = m_new;
+      }
+      const float neg_m = -m_use;
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float x0 = s[64 * h + 2 * i];
+          const float x1 = s[64 * h + 2 * i + 1];
+          const float p0 = masked ? ex2_sfu(x0 + neg_m) : ex2_sfu(fmaf(x0, c, neg_m));
+          const float p1 = masked ? ex2_sfu(x1 + neg_m) : ex2_sfu(fmaf(x1, c, neg_m));
+          sum4[(2 * i) & 3] += p0;
+          sum4[(2 * i + 1) & 3] += p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tS + 32 * h, pk);
+      }
+      tmem_st_wait();
+      l = l * alpha + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
+      if (j > 0) {
+        // PV(j-1) must be done before O is touched or PV(j) is released;
+        // waiting every tile also keeps this waiter within one phase.
+        if (!(ok = mbar_wait_warp(bar(bar_pv<NS>(t)), (j - 1) & 1, ab, kSiteSmPv))) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t u[32];
+            tmem_ld32(tO + ch * 32, u);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+            tmem_st32(tO + ch * 32, u);
+          }
+          tmem_st_wait();
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(bar_p<NS>(t)));
+    }
+    if (ok) ok = mbar_wait_warp(bar(bar_pv<NS>(t)), (n - 1) & 1, ab, kSiteEpiPv);
+    // All 128 threads of the warpgroup reach this barrier (every wait above is
+    // bounded) and take the epilogue together or not at all.
+    ok = named_bar_and(1 + t, 128, ok);
+    if (ok) {
+      tc_fence_after();
+      // ---------------------------------------------------------- epilogue
+      const float inv_l = 1.f / l;
+      const uint32_t o_stage = sbase + C::kOffQ + t * C::kTileBytes;   // Q_t no longer read
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t u[32];
+        tmem_ld32(tO + ch * 32, u);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack_bf16x2(__uint_as_float(u[2 * i]) * inv_l, __uint_as_float(u[2 * i + 1]) * inv_l);
+        const int col0 = ch * 32;
+        const uint32_t panel = o_stage + (col0 / 64) * C::kPanelBytes + r * 128;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t chunk = ((col0 % 64) / 8 + q) ^ (r & 7);
+          st_shared_v4(panel + (chunk << 4), pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1 + t, 128);
+      if (r == 0 && qi * kBlockM < p.N) {   // a tile wholly past N is padding
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_store_3d(&p.tm_o, o_stage + pn * C::kPanelBytes, pn * 64, qi * kBlockM, bh);
+        tma_store_commit();
+        tma_store_wait_all();
+      }
+      if (row < p.N) p.lse[static_cast<size_t>(bh) * p.N + row] = (m_use + log2f(l)) * 0.69314718055994531f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int D, bool CAUSAL>
+cudaError_t launch_impl(const FwdParams& p, cudaStream_t stream) {
+  using C = FwdCfg<D>;
+  auto kern = fwd_bf16_kernel<D, CAUSAL>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(p.n_pairs) * static_cast<unsigned>(p.BH);
+  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_bf16(const FwdParams& p, int d, bool causal, cudaStream_t stream) {
+  if (d == 64) return causal ? launch_impl<64, true>(p, stream) : launch_impl<64, false>(p, stream);
+  return causal ? launch_impl<128, true>(p, stream) : launch_impl<128, false>(p, stream);
+}
+
+}  // namespace fa

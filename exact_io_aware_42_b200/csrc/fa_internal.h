@@ -1,0 +1,35 @@
+// Internal launch interface between the C-ABI layer (fa_api.cu) and the
+// kernels.  Not installed; not part of the public header.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fa {
+
+constexpr int kBlockM = 128;      // query rows per tile (one TMEM lane per row)
+constexpr int kBlockN = 128;      // keys per K/V tile
+constexpr float kRescaleTau = 8.0f;   // log2 units; see the forward kernel
+
+struct FwdParams {
+  CUtensorMap tm_q;     // [BH, N, d] bf16 or e4m3, box {64 or 128 elems, 128, 1}
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  CUtensorMap tm_o;     // bf16 output, box {64, 128, 1}
+  float* lse;           // [BH, N]
+  unsigned int* status;
+  const float* sq;      // fp8 only: block scales [BH, n_qblk]
+  const float* sk;
+  const float* sv;
+  int N;
+  int BH;
+  int n_pairs;          // ceil(ceil(N/128) / 2): CTAs per (b, h)
+  int n_kv;             // ceil(N / 128)
+  float scale_log2;     // scale * log2(e)
+  float scale;
+};
+
+cudaError_t launch_fwd_bf16(const FwdParams& p, int d, bool causal, cudaStream_t stream);
+
+}  // namespace fa

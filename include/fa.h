@@ -1,0 +1,140 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact-attention library (libfa_b200.so).
+ *
+ * What the library computes is standard scaled-dot-product attention,
+ *   S = scale * Q K^T  (+ causal mask),  P = softmax(S),  O = P V,
+ *   L = m + ln(l)      (per-row logsumexp of the scaled, masked scores),
+ * as defined on the "FlashAttention" concept note ("Definition", "How it
+ * works") and in the online-softmax section of "FlashAttention v1/v2/v3/v4:
+ * the librarian who never clears the desk" (eq. 1 and eq. 2).  The forward
+ * never writes the N x N score matrix to memory; the backward rebuilds P
+ * from L ("How it works", recomputation).
+ *
+ * Conventions shared by every entry point
+ *  - Tensors are [B, H, N, d] row-major and contiguous (d fastest), one
+ *    device allocation each, base address 16-byte aligned.  bf16 means
+ *    __nv_bfloat16; e4m3 means the OCP e4m3fn byte (max 448, no infinity).
+ *  - LSE tensors are [B, H, N] fp32, natural log, of scale * Q K^T.
+ *  - All pointers are DEVICE pointers owned by the caller.  Nothing is
+ *    allocated, freed or retained by the library.
+ *  - ``stream`` is a cudaStream_t (NULL = the legacy default stream).  All
+ *    calls are asynchronous on that stream.
+ *  - Argument errors are returned synchronously, before any launch, and
+ *    leave the outputs untouched.  Supported: d in {64, 128}; 0 <= N <=
+ *    2^20; 0 <= B * H <= 2^20; scale finite and >= 0.  B * H * N == 0 is a
+ *    valid empty problem: FA_OK, nothing launched.
+ *  - Causal reading: with equal query and key lengths, key j is visible to
+ *    query i iff j <= i.
+ *  - A pipeline wait inside a kernel that exceeds ~2 s gives up: the kernel
+ *    ends early and records FA_ERR_PIPELINE_TIMEOUT in a device status word
+ *    that fa_get_status() reads after the caller has synchronised.
+ *  - The library keeps no state besides that status word and per-process
+ *    caches of kernel attributes; calls on different streams may overlap.
+ */
+#ifndef FA_B200_H_
+#define FA_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fa_status {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,      /* null pointer, negative size, bad scale     */
+  FA_ERR_UNSUPPORTED = 2,      /* d not in {64,128}, size limit, not sm_100  */
+  FA_ERR_MISALIGNED = 3,       /* a tensor base not 16-byte aligned          */
+  FA_ERR_WORKSPACE = 4,        /* workspace null or smaller than required    */
+  FA_ERR_LAUNCH = 5,           /* CUDA reported an error at launch           */
+  FA_ERR_PIPELINE_TIMEOUT = 6, /* a bounded in-kernel wait ran out           */
+  FA_ERR_NO_DEVICE = 7         /* no CUDA device / driver entry point        */
+} fa_status;
+
+/*
+ * Forward: O = softmax(scale * Q K^T [causal]) V and L = logsumexp per row.
+ *  q, k, v : bf16 [B, H, N, d] inputs.
+ *  o       : bf16 [B, H, N, d] output (O rounded to nearest even).
+ *  lse     : fp32 [B, H, N] output, natural log.
+ * One fused kernel: for each 128-row query tile it streams 128-row K/V tiles
+ * through shared memory, keeps the score tile and the running (m, l, o) on
+ * chip and divides by l once at the end ("How it works"; the lineage page,
+ * "FA2 (2023)", deferred normalisation).  Causal runs skip fully masked
+ * tiles.
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int N, int d, float scale, int causal, void* stream);
+
+/*
+ * Bytes of scratch fa_bwd needs for this shape (fp32 dQ accumulator
+ * [B, H, N, d] plus fp32 D [B, H, N], rounded up to 256 bytes each).
+ * Returns 0 for an unsupported d or a negative size.
+ */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward of the forward above for the loss sum(O * dO).
+ *  q, k, v, o, dout : bf16 [B, H, N, d]; o and lse from fa_fwd on the same
+ *                     inputs.
+ *  lse              : fp32 [B, H, N].
+ *  dq, dk, dv       : bf16 [B, H, N, d] outputs.
+ *  workspace        : device scratch of at least fa_bwd_workspace_size()
+ *                     bytes, 256-byte aligned; its contents on entry do not
+ *                     matter.
+ * P is recomputed as exp(S - L) tile by tile, never stored ("How it works",
+ * recomputation; lineage page "FA1 (2022)", idea 3).  The gradient itself is
+ * the textbook one: dV = P^T dO, dP = dO V^T, D = rowsum(dO o O),
+ * dS = P o (dP - D), dQ = scale dS K, dK = scale dS^T Q.
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                 float scale, int causal, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * FP8 block quantisation of one tensor ("the librarian" page, "FA3 -- the
+ * Hopper moment", pillar 3; lineage page, "FA3 (2024)", idea 3).
+ *  x      : bf16 [B, H, N, d] input.
+ *  x8     : e4m3 [B, H, N, d] output codes.
+ *  scales : fp32 [B, H, ceil(N / 128)] output, one per 128-row block:
+ *           scale = amax / 448 (1 for an all-zero block).
+ *  signs  : NULL for no rotation, else d fp32 values in {+1, -1}: each row
+ *           is first multiplied by diag(signs) H_d / sqrt(d) (H_d the
+ *           Sylvester Hadamard matrix), which leaves Q K^T unchanged when
+ *           applied to both Q and K with the same signs.  V is quantised
+ *           with signs = NULL.
+ * code = round_to_nearest_even_satfinite(fp32(x) / scale).
+ */
+fa_status fa_quant_fp8(const void* x, void* x8, float* scales, int B, int H, int N, int d,
+                       const float* signs, void* stream);
+
+/*
+ * FP8 forward: attention on block-quantised inputs.
+ *  q8, k8, v8 : e4m3 [B, H, N, d] from fa_quant_fp8.
+ *  sq, sk, sv : their fp32 block scales [B, H, ceil(N / 128)].
+ *  o, lse     : as in fa_fwd (bf16 O, fp32 natural-log L).
+ * Both products run on the E4M3 tensor cores; the scores are dequantised
+ * with sq * sk per tile pair, P is rounded to E4M3 (scaled by a power of
+ * two) and V's scale is applied to the accumulator per key tile.
+ */
+fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* sq,
+                     const float* sk, const float* sv, void* o, float* lse, int B, int H, int N,
+                     int d, float scale, int causal, void* stream);
+
+/*
+ * Device status word of the current device: FA_OK, or the first in-kernel
+ * failure (FA_ERR_PIPELINE_TIMEOUT, with the failing wait's site in bits
+ * 8..15) since the last fa_clear_status().  Synchronises with the device
+ * (cudaMemcpyFromSymbol); call it after synchronising your stream.
+ */
+unsigned int fa_get_status(void);
+void fa_clear_status(void);
+
+/* Static, human-readable name of a status code. */
+const char* fa_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H_ */

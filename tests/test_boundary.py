@@ -1,0 +1,90 @@
+"""Host-side checks of the C ABI that need no GPU: the library builds and
+loads, exports every entry point include/fa.h declares, and rejects bad
+arguments with the documented status codes before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from exact_io_aware_42_b200 import build
+    from exact_io_aware_42_b200._lib import lib
+    build.build()
+    return lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_documented_calls():
+    names = declared_functions()
+    for n in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_quant_fp8", "fa_fwd_fp8",
+              "fa_get_status", "fa_clear_status", "fa_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    from exact_io_aware_42_b200._lib import SIGNATURES
+    for name in declared_functions():
+        assert hasattr(L, name), name
+        assert name in SIGNATURES, f"{name} has no ctypes signature"
+
+
+def test_status_strings(L):
+    assert L.fa_status_string(0) == b"FA_OK"
+    assert L.fa_status_string(6) == b"FA_ERR_PIPELINE_TIMEOUT"
+    assert L.fa_status_string(6 | (3 << 8)) == b"FA_ERR_PIPELINE_TIMEOUT"
+    assert L.fa_status_string(99) == b"FA_ERR_UNKNOWN"
+
+
+A = 4096  # a 16-byte aligned fake device address; never dereferenced on these paths
+
+
+@pytest.mark.parametrize("args,code", [
+    ((A, A, A, A, A, 1, 1, 128, 96, 0.1, 0), 2),         # d unsupported
+    ((A, A, A, A, A, 1, 1, 128, 256, 0.1, 0), 2),
+    ((A, A, A, A, A, -1, 1, 128, 64, 0.1, 0), 1),        # negative size
+    ((A, A, A, A, A, 1, 1, -5, 64, 0.1, 0), 1),
+    ((A, A, A, A, A, 1, 1, 128, 64, -0.5, 0), 1),        # negative scale
+    ((A, A, A, A, A, 1, 1, 128, 64, float("nan"), 0), 1),
+    ((A, A, A, A, A, 1, 1, (1 << 20) + 1, 64, 0.1, 0), 2),  # N above the limit
+    ((None, A, A, A, A, 1, 1, 128, 64, 0.1, 0), 1),      # null pointer
+    ((A + 8, A, A, A, A, 1, 1, 128, 64, 0.1, 0), 3),     # misaligned
+    ((A, A, A, A, A + 2, 1, 1, 128, 64, 0.1, 0), 3),     # lse not 4-byte aligned
+    ((None, None, None, None, None, 1, 1, 0, 64, 0.1, 0), 0),   # empty problem
+    ((None, None, None, None, None, 0, 8, 128, 128, 0.1, 1), 0),
+])
+def test_fwd_argument_errors(L, args, code):
+    assert L.fa_fwd(*args, None) == code
+
+
+def test_workspace_size(L):
+    assert L.fa_bwd_workspace_size(1, 1, 128, 96) == 0
+    assert L.fa_bwd_workspace_size(-1, 1, 128, 64) == 0
+    got = L.fa_bwd_workspace_size(4, 16, 4096, 128)
+    rows = 4 * 16 * 4096
+    assert got == rows * 128 * 4 + rows * 4
+    assert L.fa_bwd_workspace_size(1, 1, 1, 64) == 256 + 256
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_call_without_device_reports_no_device(L):
+    assert L.fa_fwd(A, A, A, A, A, 1, 1, 128, 64, 0.1, 0, None) == 7
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    import exact_io_aware_42_b200._lib as lb
+    monkeypatch.setattr(lb, "_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(lb, "_LIB", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        lb.lib()

@@ -1,0 +1,135 @@
+"""GPU parity of the bf16 forward (fa_fwd through the C ABI) against the fp64 oracle.
+
+Sizes span several 128-row tiles and ragged tails; the full-size workload is
+checked on sampled heads against the oracle and on every head against closed
+forms that hold at any size.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_io_aware_42_b200 import inputs
+from tests.helpers import assert_fwd_close, f64, LSE_MAX_ABS, O_MAX_ABS
+
+pytestmark = pytest.mark.gpu
+
+
+def _fa():
+    import exact_io_aware_42_b200 as fa
+    return fa
+
+
+def run_fwd(q, k, v, causal, scale=None):
+    fa = _fa()
+    o, lse = fa.fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.get_status() == 0
+    return o.cpu(), lse.cpu()
+
+
+def test_fwd_tiny_workload():
+    w = inputs.TINY
+    q, k, v = inputs.make_workload(w)
+    o, lse = run_fwd(q, k, v, False)
+    o_ref, l_ref = oracle.attn_fwd_ref(q, k, v, 1 / math.sqrt(w.d), False)
+    assert_fwd_close(o, lse, o_ref, l_ref, w.name)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fwd_small_workload(causal):
+    w = inputs.SMALL
+    q, k, v = inputs.make_workload(w)
+    o, lse = run_fwd(q, k, v, causal)
+    o_ref, l_ref = oracle.attn_fwd_ref(q, k, v, 1 / math.sqrt(w.d), causal)
+    assert_fwd_close(o, lse, o_ref, l_ref, f"{w.name} causal={causal}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 7, 127, 128, 129, 200, 255, 256, 257, 383, 513])
+def test_fwd_ragged(N, d, causal):
+    q, k, v = inputs.make_qkv(1, 2, N, d, seed=100 + N + d)
+    o, lse = run_fwd(q, k, v, causal)
+    o_ref, l_ref = oracle.attn_fwd_ref(q, k, v, 1 / math.sqrt(d), causal)
+    assert_fwd_close(o, lse, o_ref, l_ref, f"N={N} d={d} causal={causal}")
+
+
+def test_fwd_long_workload_sampled_heads():
+    w = inputs.LONG
+    q, k, v, _ = inputs.make_workload(w)
+    o, lse = run_fwd(q, k, v, True)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    for b, h in ((0, 0), (1, 7), (3, 15)):
+        o_ref, l_ref = oracle.attn_fwd_ref(q[b:b + 1, h:h + 1], k[b:b + 1, h:h + 1],
+                                           v[b:b + 1, h:h + 1], 1 / math.sqrt(w.d), True)
+        assert_fwd_close(o[b:b + 1, h:h + 1], lse[b:b + 1, h:h + 1], o_ref, l_ref, f"b={b} h={h}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fwd_scale_zero_closed_form_full_size(causal):
+    """scale = 0: every visible score is 0, so O is the (prefix) mean of V and
+    L = ln(number of visible keys), at the full 4096-token size."""
+    w = inputs.LONG
+    q, k, v, _ = inputs.make_workload(w)
+    o, lse = run_fwd(q, k, v, causal, scale=0.0)
+    vv = f64(v)
+    n = w.N
+    if causal:
+        cnt = np.arange(1, n + 1, dtype=np.float64)
+        o_ref = np.cumsum(vv, axis=2) / cnt[None, None, :, None]
+        l_ref = np.broadcast_to(np.log(cnt), lse.shape)
+    else:
+        o_ref = np.broadcast_to(vv.mean(axis=2, keepdims=True), vv.shape)
+        l_ref = np.full(lse.shape, math.log(n))
+    assert np.max(np.abs(f64(lse) - l_ref)) <= LSE_MAX_ABS
+    assert np.max(np.abs(f64(o) - o_ref)) <= O_MAX_ABS
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fwd_one_hot_values_recover_p(causal):
+    """V = identity: O equals the probability matrix P itself."""
+    N, d = 128, 128
+    q, k, _ = inputs.make_qkv(1, 1, N, d, seed=7)
+    v = torch.eye(N, d, dtype=torch.bfloat16)[None, None].contiguous()
+    o, lse = run_fwd(q, k, v, causal)
+    o_ref, l_ref = oracle.attn_fwd_ref(q, k, v, 1 / math.sqrt(d), causal)
+    assert_fwd_close(o, lse, o_ref, l_ref, "one-hot V")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fwd_large_magnitude_exercises_rescale(causal):
+    """Q x 8 with a growing ramp: the running max moves by more than the
+    rescale threshold across tiles, so the O correction path runs."""
+    N, d = 1024, 64
+    q, k, v = inputs.make_qkv(1, 2, N, d, seed=9)
+    ramp = torch.linspace(0.2, 3.0, N)[None, None, :, None]
+    q = (q.float() * 8.0).to(torch.bfloat16)
+    k = (k.float() * ramp).to(torch.bfloat16)
+    o, lse = run_fwd(q, k, v, causal)
+    o_ref, l_ref = oracle.attn_fwd_ref(q, k, v, 1 / math.sqrt(d), causal)
+    assert_fwd_close(o, lse, o_ref, l_ref, "large magnitude")
+
+
+def test_fwd_identical_keys_give_mean():
+    N, d = 300, 128
+    q, k, v = inputs.make_qkv(2, 1, N, d, seed=11)
+    k = k[:, :, :1].expand(-1, -1, N, -1).contiguous()
+    o, lse = run_fwd(q, k, v, False)
+    o_ref = np.broadcast_to(f64(v).mean(axis=2, keepdims=True), o.shape)
+    assert np.max(np.abs(f64(o) - o_ref)) <= O_MAX_ABS
+
+
+def test_fwd_empty_and_errors():
+    fa = _fa()
+    z = torch.empty((1, 1, 0, 64), dtype=torch.bfloat16, device="cuda")
+    o, lse = fa.fwd(z, z, z)
+    assert o.shape == (1, 1, 0, 64) and lse.shape == (1, 1, 0)
+    x = torch.zeros((1, 1, 16, 96), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(fa.FaError) as e:
+        fa.fwd(x, x, x)
+    assert e.value.code == 2
+    torch.cuda.synchronize()
+    assert fa.get_status() == 0
