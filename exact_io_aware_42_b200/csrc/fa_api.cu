@@ -5,6 +5,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -75,6 +76,19 @@ fa_status current_device(DeviceInfo** out) {
   return FA_OK;
 }
 
+// Share of the exp2 work on the FMA pipe (pairs of 8); FA_POLY_PAIRS in the
+// environment overrides the per-d default for measurement (0, 2 or 4).
+int poly_pairs(int d) {
+  static int env = [] {
+    const char* e = std::getenv("FA_POLY_PAIRS");
+    if (!e) return -1;
+    const int x = std::atoi(e);
+    return (x == 0 || x == 2 || x == 4) ? x : -1;
+  }();
+  if (env >= 0) return env;
+  return d == 64 ? kDefaultPolyPairsD64 : kDefaultPolyPairsD128;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // 3-D view [BH, N, d] of a contiguous [B, H, N, d] tensor, 128-byte swizzle,
@@ -136,6 +150,7 @@ extern "C" fa_status fa_fwd(const void* q, const void* k, const void* v, void* o
   p.n_pairs = ((N + kBlockM - 1) / kBlockM + 1) / 2;
   p.scale = scale;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.poly_pairs = poly_pairs(d);
   cudaError_t e = launch_fwd_bf16(p, d, causal != 0, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     cudaGetLastError();

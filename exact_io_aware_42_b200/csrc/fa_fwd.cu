@@ -36,8 +36,9 @@
 // Causal: key j visible to query i iff j <= i.  Tiles entirely above the
 // diagonal are never loaded or multiplied; only the diagonal tile and the
 // ragged key tail (keys >= N, zero-filled by TMA) are masked to -inf.
-#include "fa_ptx.cuh"
+#include "fa_exp2.cuh"
 #include "fa_internal.h"
+#include "fa_ptx.cuh"
 
 namespace fa {
 namespace {
@@ -80,11 +81,9 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
-__device__ __forceinline__ float max4(float a, float b, float c, float d) {
-  return fmaxf(fmaxf(a, b), fmaxf(c, d));
-}
-
-template <int D, bool CAUSAL>
+// NPOLY of every 8 column pairs take the polynomial exp2 (degree DEG), the
+// rest the SFU.
+template <int D, bool CAUSAL, int NPOLY, int DEG>
 __global__ void __launch_bounds__(320, 1) fwd_bf16_kernel(const __grid_constant__ FwdParams p) {
   using C = FwdCfg<D>;
   constexpr int NS = C::kStages;
@@ -242,7 +241,7 @@ __global__ void __launch_bounds__(320, 1) fwd_bf16_kernel(const __grid_constant_
       mbar_wait(bar(bar_drain<NS>()), 0, drain, kSiteDrain);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ softmax
     const int t = warp >> 2;                 // query tile of this warpgroup
     const int r = threadIdx.x - 128 * t;     // row within the tile == TMEM lane
@@ -259,35 +258,31 @@ __global__ void __launch_bounds__(320, 1) fwd_bf16_kernel(const __grid_constant_
     for (int j = 0; j < n; ++j) {
       if (!(ok = mbar_wait_warp(bar(bar_s<NS>(t)), j & 1, ab, kSiteSmS))) break;
       tc_fence_after();
-      float s[128];
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t u[32];
-        tmem_ld32(tS + ch * 32, u);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[ch * 32 + i] = __uint_as_float(u[i]);
-      }
+      uint32_t u[128];
+      tmem_ld128(tS, u);
       const bool masked = (CAUSAL && j == qi) || ((j + 1) * kBlockN > p.N);
-      float mt;
       if (masked) {
+        // scaled scores with -inf where the key is hidden or past N
         const int key0 = j * kBlockN;
 #pragma unroll
         for (int i = 0; i < 128; ++i) {
           const int key = key0 + i;
           const bool vis = key < p.N && (!CAUSAL || key <= row);
-          s[i] = vis ? s[i] * c : -INFINITY;
+          u[i] = __float_as_uint(vis ? __uint_as_float(u[i]) * c : -INFINITY);
         }
       }
+      float mt;
       {
-        float m8[8];
+        float a[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) m8[i] = s[i];
+        for (int k = 0; k < 8; ++k) a[k] = fmaxf(__uint_as_float(u[k]), __uint_as_float(u[8 + k]));
 #pragma unroll
-        for (int i = 8; i < 128; i += 8) {
+        for (int i = 16; i < 128; i += 16) {
 #pragma unroll
-          for (int k = 0; k < 8; ++k) m8[k] = fmaxf(m8[k], s[i + k]);
+          for (int k = 0; k < 8; ++k)
+            a[k] = max3f(a[k], __uint_as_float(u[i + k]), __uint_as_float(u[i + 8 + k]));
         }
-        mt = fmaxf(max4(m8[0], m8[1], m8[2], m8[3]), max4(m8[4], m8[5], m8[6], m8[7]));
+        mt = max3f(max3f(a[0], a[1], a[2]), max3f(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
         if (!masked) mt *= c;
       }
       const float m_new = fmaxf(m_use, mt);
@@ -298,23 +293,38 @@ __global__ void __launch_bounds__(320, 1) fwd_bf16_kernel(const __grid_constant_
         m_use = m_new;
       }
       const float neg_m = -m_use;
-      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+      if (masked) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float x0 = s[64 * h + 2 * i];
-          const float x1 = s[64 * h + 2 * i + 1];
-          const float p0 = masked ? ex2_sfu(x0 + neg_m) : ex2_sfu(fmaf(x0, c, neg_m));
-          const float p1 = masked ? ex2_sfu(x1 + neg_m) : ex2_sfu(fmaf(x1, c, neg_m));
-          sum4[(2 * i) & 3] += p0;
-          sum4[(2 * i + 1) & 3] += p1;
-          pk[i] = pack_bf16x2(p0, p1);
+        for (int i = 0; i < 64; ++i) {
+          const float p0 = ex2_sfu(__uint_as_float(u[2 * i]) + neg_m);
+          const float p1 = ex2_sfu(__uint_as_float(u[2 * i + 1]) + neg_m);
+          acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
+          u[i] = pack_bf16x2(p0, p1);       // P overwrites the consumed scores
         }
-        tmem_st32(tS + 32 * h, pk);
+      } else {
+        const uint64_t c2 = f2_pack(c, c);
+        const uint64_t nm2 = f2_pack(neg_m, neg_m);
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const uint64_t x2 =
+              f2_fma(f2_pack(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1])), c2, nm2);
+          const uint64_t p2 = ((i & 7) < NPOLY) ? exp2_poly_f2<DEG>(x2) : exp2_sfu_f2(x2);
+          acc[i & 3] = f2_add(acc[i & 3], p2);
+          float p0, p1;
+          f2_unpack(p2, p0, p1);
+          u[i] = pack_bf16x2(p0, p1);
+        }
       }
+      tmem_st64(tS, *reinterpret_cast<uint32_t(*)[64]>(&u[0]));
       tmem_st_wait();
+      float sum4[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float lo, hi;
+        f2_unpack(acc[k], lo, hi);
+        sum4[k] = lo + hi;
+      }
       l = l * alpha + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
       if (j > 0) {
         // PV(j-1) must be done before O is touched or PV(j) is released;
@@ -381,10 +391,10 @@ __global__ void __launch_bounds__(320, 1) fwd_bf16_kernel(const __grid_constant_
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, int NPOLY>
 cudaError_t launch_impl(const FwdParams& p, cudaStream_t stream) {
   using C = FwdCfg<D>;
-  auto kern = fwd_bf16_kernel<D, CAUSAL>;
+  auto kern = fwd_bf16_kernel<D, CAUSAL, NPOLY, 3>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(p.n_pairs) * static_cast<unsigned>(p.BH);
@@ -394,9 +404,18 @@ cudaError_t launch_impl(const FwdParams& p, cudaStream_t stream) {
 
 }  // namespace
 
+template <int D, bool CAUSAL>
+cudaError_t launch_np(const FwdParams& p, cudaStream_t stream) {
+  switch (p.poly_pairs) {
+    case 0: return launch_impl<D, CAUSAL, 0>(p, stream);
+    case 4: return launch_impl<D, CAUSAL, 4>(p, stream);
+    default: return launch_impl<D, CAUSAL, 2>(p, stream);
+  }
+}
+
 cudaError_t launch_fwd_bf16(const FwdParams& p, int d, bool causal, cudaStream_t stream) {
-  if (d == 64) return causal ? launch_impl<64, true>(p, stream) : launch_impl<64, false>(p, stream);
-  return causal ? launch_impl<128, true>(p, stream) : launch_impl<128, false>(p, stream);
+  if (d == 64) return causal ? launch_np<64, true>(p, stream) : launch_np<64, false>(p, stream);
+  return causal ? launch_np<128, true>(p, stream) : launch_np<128, false>(p, stream);
 }
 
 }  // namespace fa

@@ -28,7 +28,16 @@ struct FwdParams {
   int n_kv;             // ceil(N / 128)
   float scale_log2;     // scale * log2(e)
   float scale;
+  int poly_pairs;       // of every 8 column pairs, how many use the FMA-pipe exp2
 };
+
+// Default share of the softmax exp2 taken by the polynomial (of 8 column
+// pairs), chosen by measurement on B200: at d = 128 the SFU-only softmax was
+// fastest (the polynomial's extra FMA-pipe instructions cost more than the
+// SFU time they free); at d = 64, where the softmax is the bound, half the
+// pairs on the polynomial was fastest.
+constexpr int kDefaultPolyPairsD128 = 0;
+constexpr int kDefaultPolyPairsD64 = 4;
 
 cudaError_t launch_fwd_bf16(const FwdParams& p, int d, bool causal, cudaStream_t stream);
 
