@@ -1,0 +1,383 @@
+"""Benchmark of the exact-attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the whole path over the workload "B4 H16 N4096 d128
+causal" (4 x 16 heads, 4096 tokens, head dim 128, bf16, synthetic N(0, 1)
+inputs from exact_io_aware_42_b200.inputs):
+
+  bf16 forward (O, LSE) -> bf16 backward (dQ, dK, dV) -> FP8 block
+  quantisation of Q, K (rotated) and V -> FP8 forward.
+
+``value`` is the whole job's attention TFLOPS: algorithmic FLOPs of every
+stage (forward 4 B H N^2 d, halved when causal; backward 2.5 x forward; the
+FP8 forward counted like a forward) over the device time of the K timed steps,
+max over ranks.  Inputs (4 x 64 MiB) exceed the 126 MB L2, so no flush is
+needed between steps.  ``e2e`` is the same metric through the public API with
+the inputs copied from pinned host memory and every output copied back inside
+the timed region.  Under torchrun every rank runs its own copy of the
+workload on its own GPU (independent heads, no collective on the data path):
+weak scaling.
+
+``--impl reference`` times the fp64 CPU oracle (the only other code this
+script may run) on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = dict(name="attn_B4_H16_N4096_d128_causal", B=4, H=16, N=4096, d=128, causal=True,
+                seed=2)
+
+
+def fwd_flops(B, H, N, d, causal):
+    f = 4.0 * B * H * N * N * d
+    return f / 2 if causal else f
+
+
+def fwd_bytes(B, H, N, d):
+    """Algorithmic bytes of the forward: Q, K, V read once, O written, LSE written."""
+    return 3 * B * H * N * d * 2 + B * H * N * d * 2 + B * H * N * 4
+
+
+def bwd_bytes(B, H, N, d):
+    return 5 * B * H * N * d * 2 + 2 * B * H * N * 4 + 3 * B * H * N * d * 2
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in ("fa_fwd.cu", "fa_ptx.cuh", "fa_exp2.cuh", "fa_exp2_poly.h", "fa_internal.h"):
+        with open(os.path.join(ROOT, "exact_io_aware_42_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per forward launch from the committed ncu summary, if it was
+    taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "fwd_bf16_B4_H16_N4096_d128_causal.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)\s+source_sha:\s*([0-9a-f]+)", text)
+    if not m or m.group(2) != kernel_source_hash():
+        return None
+    return float(m.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs):
+    """The hot path as a list of (stage name, callable, FLOPs, kernel launches)."""
+    state = {}
+
+    def s_fwd():
+        state["o"], state["lse"] = fa.fwd(q, k, v, causal=causal)
+
+    stages = [("fwd_bf16", s_fwd, fwd_flops(B, H, N, d, causal), 1)]
+    return stages, state
+
+
+def time_stages(torch, stages, steps, stream):
+    """Device time of ``steps`` passes over the stages, plus per-stage event times."""
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in stages] for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        for j, (_, fn, _, _) in enumerate(stages):
+            ev[i][j][0].record(stream)
+            fn()
+            ev[i][j][1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    total_ms = start.elapsed_time(end)
+    per_stage = [sum(ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(steps)) / steps
+                 for j in range(len(stages))]
+    return total_ms, per_stage
+
+
+_ORACLE_INPUTS = {}
+
+
+def oracle_sample(budget_s: float, B, H, N, d, causal, with_bwd: bool):
+    """Time the fp64 oracle head by head on the host cores until ``budget_s``."""
+    import numpy as np
+    import oracle
+    from exact_io_aware_42_b200 import inputs
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
+    except Exception:  # noqa: BLE001
+        cores = os.cpu_count()
+    key = (B, H, N, d)
+    if key not in _ORACLE_INPUTS:
+        _ORACLE_INPUTS[key] = inputs.make_qkv(B, H, N, d, WORKLOAD["seed"], with_do=True)
+    q, k, v, do = _ORACLE_INPUTS[key]
+    sc = 1.0 / math.sqrt(d)
+    flops, heads, t0 = 0.0, 0, time.perf_counter()
+    for idx in range(B * H):
+        b, h = divmod(idx, H)
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        oracle.attn_fwd_ref(q[sl], k[sl], v[sl], sc, causal)
+        flops += fwd_flops(1, 1, N, d, causal)
+        if with_bwd:
+            oracle.attn_bwd_ref(q[sl], k[sl], v[sl], do[sl], sc, causal)
+            flops += 2.5 * fwd_flops(1, 1, N, d, causal)
+        heads += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": "TFLOPS", "cores": int(cores), "kind": "oracle",
+            "sample": f"{heads} of {B * H} heads of {WORKLOAD['name']}, fwd"
+                      + ("+bwd" if with_bwd else "") + f", fp64 numpy, {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = WORKLOAD
+    with_bwd = STAGES_WITH_BWD
+    for _ in range(args.warmup):
+        oracle_sample(0.0, 1, 1, 256, w["d"], w["causal"], with_bwd)
+    vals = []
+    t_all = time.perf_counter()
+    for _ in range(args.steps):
+        vals.append(oracle_sample(args.ref_seconds, w["B"], w["H"], w["N"], w["d"], w["causal"], with_bwd))
+    dt = time.perf_counter() - t_all
+    v = sum(x["value"] for x in vals) / len(vals)
+    cpu = dict(vals[-1])
+    cpu["value"] = v
+    line = {"metric": METRIC, "value": v, "unit": "TFLOPS", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference", "config": config_block(), "cpu_baseline": cpu,
+            "e2e": {"value": v, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+METRIC = "attention fwd/bwd TFLOPS (BF16 causal+non-causal) and % of B200 tensor peak"
+STAGES_WITH_BWD = False
+
+
+def config_block():
+    w = WORKLOAD
+    return {"workload": w["name"], "B": w["B"], "H": w["H"], "N": w["N"], "d": w["d"],
+            "causal": w["causal"], "global_batch": w["B"], "seq_len": w["N"],
+            "parallelism": "independent replicas per GPU (heads), no collective",
+            "l2": "inputs 4 x 64 MiB > 126 MB L2, no flush",
+            "step": "fwd_bf16" + (" + bwd_bf16" if STAGES_WITH_BWD else "")}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import exact_io_aware_42_b200 as fa
+    from exact_io_aware_42_b200 import inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    w = WORKLOAD
+    B, H, N, d, causal = w["B"], w["H"], w["N"], w["d"], w["causal"]
+    hq, hk, hv, hdo = inputs.make_qkv(B, H, N, d, w["seed"] + rank, with_do=True)
+    signs = inputs.signs(d).to(dev)
+    q, k, v, do = (t.to(dev) for t in (hq, hk, hv, hdo))
+    stages, state = build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs)
+    step_flops = sum(s[2] for s in stages)
+    launches_per_step = sum(s[3] for s in stages)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        for s in stages:
+            s[1]()
+    barrier()
+    with ClockSampler(local) as clk:
+        total_ms, per_stage = time_stages(torch, stages, args.steps, stream)
+    barrier()
+    fa_status = fa.get_status()
+    total_ms = max_over_ranks(total_ms)
+    per_stage = [max_over_ranks(x) for x in per_stage]
+    ms_step = total_ms / args.steps
+    value = world * step_flops / (ms_step * 1e-3) / 1e12
+
+    # end to end through the public API, host buffers in and out
+    pin = {n: t.pin_memory() for n, t in (("q", hq), ("k", hk), ("v", hv), ("do", hdo))}
+    dev_in = {"q": q, "k": k, "v": v, "do": do}
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    outs_host = {}
+
+    def e2e_step():
+        for n, t in pin.items():
+            dev_in[n].copy_(t, non_blocking=True)
+        for s in stages:
+            s[1]()
+        for n, t in state.items():
+            if n not in outs_host:
+                outs_host[n] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+            outs_host[n].copy_(t, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    d2h = sum(t.numel() * t.element_size() for t in outs_host.values())
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+    barrier()
+
+    peaks, peak_src = measured_peaks()
+    fwd_idx = [i for i, s in enumerate(stages) if s[0] == "fwd_bf16"][0]
+    fwd_ms = per_stage[fwd_idx]
+    achieved = stages[fwd_idx][2] / (fwd_ms * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops_sustained"])
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_block(),
+        "pct_of_peak": {"measured_bf16_burst": value / world / float(peaks["bf16_tflops"]),
+                        "nominal_2250": value / world / 2250.0},
+        "stages": {s[0]: {"ms": per_stage[i], "tflops": s[2] / (per_stage[i] * 1e-3) / 1e12}
+                   for i, s in enumerate(stages)},
+        "roofline": {"kernel": "fwd_bf16_kernel<128, causal>", "bound": "tensor",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside the step loop)",
+                     "traffic": profiled_traffic(),
+                     "algorithmic_bytes": fwd_bytes(B, H, N, d)},
+        "e2e": {"value": world * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+        "device_status": fa_status,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_sample(args.ref_seconds, B, H, N, d, causal, STAGES_WITH_BWD)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0 if fa_status == 0 else 1
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--ref-seconds", type=float, default=12.0,
+                    help="host-core seconds of oracle work per reference step / cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

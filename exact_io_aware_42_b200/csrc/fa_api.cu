@@ -166,10 +166,56 @@ extern "C" size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   return up(rows * d * sizeof(float)) + up(rows * sizeof(float));
 }
 
-extern "C" fa_status fa_bwd(const void*, const void*, const void*, const void*, const void*,
-                            const float*, void*, void*, void*, int, int, int, int, float, int,
-                            void*, size_t, void*) {
-  return FA_ERR_UNSUPPORTED;
+extern "C" fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o,
+                            const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                            int B, int H, int N, int d, float scale, int causal, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  fa_status st = check_shape(B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  if (static_cast<long long>(B) * H * N == 0) return FA_OK;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return FA_ERR_MISALIGNED;
+  const size_t need = fa_bwd_workspace_size(B, H, N, d);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return FA_ERR_WORKSPACE;
+  DeviceInfo* di = nullptr;
+  if ((st = current_device(&di)) != FA_OK) return st;
+
+  const int BH = B * H;
+  const long long rows = static_cast<long long>(BH) * N;
+  float* dq_acc = static_cast<float*>(workspace);
+  float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                          ((static_cast<size_t>(rows) * d * 4 + 255) & ~static_cast<size_t>(255)));
+  BwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!encode_3d(&p.tm_q, q, bf, 2, d, N, BH, 64, 128) || !encode_3d(&p.tm_k, k, bf, 2, d, N, BH, 64, 128) ||
+      !encode_3d(&p.tm_v, v, bf, 2, d, N, BH, 64, 128) || !encode_3d(&p.tm_do, dout, bf, 2, d, N, BH, 64, 128))
+    return FA_ERR_INVALID_ARG;
+  p.lse = lse;
+  p.delta = delta;
+  p.dq_acc = dq_acc;
+  p.dk = static_cast<uint16_t*>(dk);
+  p.dv = static_cast<uint16_t*>(dv);
+  p.status = di->status;
+  p.N = N;
+  p.BH = BH;
+  p.n_kv = (N + 127) / 128;
+  p.n_q = (N + 127) / 128;
+  p.scale = scale;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_bwd_preprocess(static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout),
+                                        delta, dq_acc, rows, d, s);
+  if (e == cudaSuccess) e = launch_bwd_main(p, d, causal != 0, s);
+  if (e == cudaSuccess) e = launch_bwd_postprocess(dq_acc, static_cast<uint16_t*>(dq), rows * d, scale, s);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+  }
+  return FA_OK;
 }
 
 extern "C" fa_status fa_quant_fp8(const void*, void*, float*, int, int, int, int, const float*,

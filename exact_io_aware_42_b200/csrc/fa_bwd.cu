@@ -1,0 +1,484 @@
+// Attention backward for sm_100a: dQ, dK, dV of the loss sum(O * dO).
+//
+// The probabilities are never stored: every tile of P is rebuilt from the
+// saved logsumexp, P = exp(S - L) ("FlashAttention" concept note, "How it
+// works", recomputation; lineage page, "FA1 (2022)", idea 3).  The gradient
+// is the textbook one of softmax(scale Q K^T) V:
+//   dV = P^T dO,  dP = dO V^T,  D = rowsum(dO o O),  dS = P o (dP - D),
+//   dQ = scale dS K,  dK = scale dS^T Q.
+//
+// Three kernels:
+//   preprocess  D per row and a zeroed fp32 dQ accumulator (memory-bound)
+//   main        one CTA per (b, h, 128-key block j): K_j, V_j stay in shared
+//               memory while the 128-query blocks i stream past
+//   postprocess dQ = bf16(scale * dQ accumulator) (memory-bound)
+//
+// Main kernel, per query block i (TMEM lanes are the CTA's 128 keys):
+//   S^T  = K_j Q_i^T            tcgen05 SS   -> TMEM [0,128)
+//   dP^T = V_j dO_i^T           tcgen05 SS   -> TMEM [128,256)
+//   P^T  = 2^(S^T c - L log2 e) softmax warps, bf16 back into TMEM [0,64)
+//   dV  += P^T dO_i             tcgen05 TS   (A = P^T from TMEM)
+//   dS^T = P^T o (dP^T - D)     softmax warps, bf16 into TMEM [128,192) and
+//                               into shared memory (MN-major, 128-B swizzle)
+//   dK  += dS^T Q_i             tcgen05 TS
+//   dQ_i = dS K_j               tcgen05 SS (A = dS, MN-major) -> TMEM [0,d)
+//   dQ accumulator += dQ_i      dQ warps: TMEM -> red.global.add.v4.f32
+// dV and dK accumulate in TMEM [256,256+d) and [256+d,256+2d) over all i and
+// are written once at the end.  dQ accumulation: every key block adds its
+// share of a query block's dQ into one fp32 buffer with vector reductions in
+// L2 (the summation order across key blocks is not fixed, so dQ may differ in
+// the last bits from run to run; dK and dV are deterministic).
+//
+// Roles: warps 0-3 softmax / dS and the dK, dV epilogue (thread = key row);
+// warps 4-7 dQ reduction (thread = query row); warp 8 TMA producer (also
+// stages L and D of each query block in shared memory); warp 9 TMEM owner and
+// the single MMA-issuing thread.  Every wait is bounded (fa_ptx.cuh).
+#include "fa_internal.h"
+#include "fa_ptx.cuh"
+
+namespace fa {
+namespace {
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kPanels = D / 64;
+  static constexpr int kPanelBytes = 128 * 128;
+  static constexpr int kTileBytes = 128 * D * 2;       // one 128 x D bf16 tile
+  static constexpr int kStages = (D == 128) ? 2 : 3;   // (Q_i, dO_i) ring depth
+  static constexpr int kThreads = 320;
+  // All swizzled tiles are 1024-byte aligned offsets from the (1024-aligned)
+  // dynamic shared memory base.
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kTileBytes;
+  static constexpr int kOffQ = 2 * kTileBytes;          // + s * 2 * kTileBytes
+  static constexpr int kOffDS = kOffQ + kStages * 2 * kTileBytes;   // dS^T, 128 x 128 bf16
+  static constexpr int kOffLD = kOffDS + 128 * 128 * 2;             // + s * 1024: L2[128], D[128]
+  static constexpr int kOffBar = kOffLD + kStages * 1024;
+  static constexpr int kNumBars = 1 + 2 * kStages + 9;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS = 0;      // S^T, then P^T (bf16), then dQ_i
+  static constexpr uint32_t kColDP = 128;   // dP^T, then dS^T (bf16)
+  static constexpr uint32_t kColDV = 256;
+  static constexpr uint32_t kColDK = 256 + D;
+};
+static_assert(BwdCfg<128>::kSmemBytes <= 232448, "backward d=128 shared memory");
+
+enum : unsigned int { kSiteBProd = 16, kSiteBMmaKV, kSiteBMmaQ, kSiteBMmaFree, kSiteBMmaP, kSiteBMmaDS,
+                      kSiteBSmS, kSiteBSmDP, kSiteBSmDQ, kSiteBDq, kSiteBEpi, kSiteBDrain, kSiteBAlign };
+
+// ------------------------------------------------------------------ preprocess
+// One group of d/8 threads per row: 16-byte loads of O and dO, fp32 dot
+// product reduced by shuffles; the same threads zero that row of dQ_acc.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const uint4* __restrict__ o,
+                                                             const uint4* __restrict__ dout,
+                                                             float* __restrict__ delta,
+                                                             float4* __restrict__ dq_acc,
+                                                             long long rows) {
+  constexpr int kTpr = D / 8;                       // threads per row (8 or 16)
+  constexpr int kRowsPerWarp = 32 / kTpr;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane % kTpr;
+  const long long warp_id = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) / 32;
+  const long long nwarps = static_cast<long long>(gridDim.x) * blockDim.x / 32;
+  // The loop bound is uniform across the warp so every shuffle sees all lanes.
+  for (long long wrow = warp_id * kRowsPerWarp; wrow < rows; wrow += nwarps * kRowsPerWarp) {
+    const long long row = wrow + lane / kTpr;
+    const bool valid = row < rows;
+    uint4 a = make_uint4(0, 0, 0, 0), b = a;
+    if (valid) {
+      a = o[row * kTpr + sub];
+      b = dout[row * kTpr + sub];
+    }
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+    const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+    float acc = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      acc = fmaf(__uint_as_float(aw[w] << 16), __uint_as_float(bw[w] << 16), acc);
+      acc = fmaf(__uint_as_float(aw[w] & 0xFFFF0000u), __uint_as_float(bw[w] & 0xFFFF0000u), acc);
+    }
+#pragma unroll
+    for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (valid) {
+      if (sub == 0) delta[row] = acc;
+      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      dq_acc[row * (D / 4) + 2 * sub] = z;
+      dq_acc[row * (D / 4) + 2 * sub + 1] = z;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ postprocess
+__global__ void __launch_bounds__(256) bwd_postprocess_kernel(const float4* __restrict__ acc,
+                                                              uint2* __restrict__ dq, long long n4,
+                                                              float scale) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4; i += stride) {
+    const float4 a = acc[i];
+    dq[i] = make_uint2(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale));
+  }
+}
+
+// ------------------------------------------------------------------ main
+__device__ __forceinline__ void st_shared_v4b(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                              uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c, float d) {
+  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a),
+               "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ void st_global_v4(void* dst, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(320, 1) bwd_main_kernel(const __grid_constant__ BwdParams p) {
+  using C = BwdCfg<D>;
+  constexpr int NS = C::kStages;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {   // the swizzled layouts below need a 1024-byte aligned base
+    if (threadIdx.x == 0) atomicCAS(p.status, 0u, FA_ERR_LAUNCH | (kSiteBAlign << 8));
+    return;
+  }
+  auto bar = [&](int i) -> uint32_t { return sbase + C::kOffBar + 8 * i; };
+  const int B_KV = 0;
+  auto B_QF = [](int s) { return 1 + s; };
+  auto B_QE = [](int s) { return 1 + NS + s; };
+  const int B_S = 1 + 2 * NS, B_DP = B_S + 1, B_P = B_S + 2, B_DS = B_S + 3, B_DQ = B_S + 4,
+            B_DQFREE = B_S + 5, B_FINAL = B_S + 6, B_DRAIN = B_S + 7;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.x % p.BH;
+  const int j = blockIdx.x / p.BH;                 // key block; small j (most work) first
+  const int i0 = CAUSAL ? j : 0;
+  const int n_i = p.n_q - i0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_KV), 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar(B_QF(s)), 1);
+      mbar_init(bar(B_QE(s)), 1);
+    }
+    mbar_init(bar(B_S), 1);
+    mbar_init(bar(B_DP), 1);
+    mbar_init(bar(B_P), 128);
+    mbar_init(bar(B_DS), 128);
+    mbar_init(bar(B_DQ), 1);
+    mbar_init(bar(B_DQFREE), 128);
+    mbar_init(bar(B_FINAL), 1);
+    mbar_init(bar(B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Abort ab{abort_flag, p.status};
+  const uint32_t kAddr = sbase + C::kOffK, vAddr = sbase + C::kOffV, dsAddr = sbase + C::kOffDS;
+  auto qAddr = [&](int s) -> uint32_t { return sbase + C::kOffQ + s * 2 * C::kTileBytes; };
+  auto doAddr = [&](int s) -> uint32_t { return qAddr(s) + C::kTileBytes; };
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    int issued = 0;
+    bool ok = true;
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_q);
+      tma_prefetch_desc(&p.tm_do);
+      mbar_arrive_expect_tx(bar(B_KV), 2 * C::kTileBytes);
+      for (int pn = 0; pn < C::kPanels; ++pn) {
+        tma_load_3d(kAddr + pn * C::kPanelBytes, &p.tm_k, bar(B_KV), pn * 64, j * 128, bh);
+        tma_load_3d(vAddr + pn * C::kPanelBytes, &p.tm_v, bar(B_KV), pn * 64, j * 128, bh);
+      }
+    }
+    for (int idx = 0; idx < n_i && ok; ++idx) {
+      const int i = i0 + idx;
+      const int s = idx % NS;
+      const uint32_t ph = (idx / NS) & 1;
+      bool w = true;
+      if (lane == 0) w = mbar_wait(bar(B_QE(s)), ph ^ 1, ab, kSiteBProd);
+      ok = __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      // L (in log2 units) and D of the 128 query rows, +inf / 0 past N
+      float* ld = reinterpret_cast<float*>(smem + C::kOffLD + s * 1024);
+      float lv[4], dv4[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int q = i * 128 + lane * 4 + t;
+        const bool in = q < p.N;
+        const size_t g = static_cast<size_t>(bh) * p.N + q;
+        lv[t] = in ? p.lse[g] * 1.4426950408889634f : INFINITY;
+        dv4[t] = in ? p.delta[g] : 0.f;
+      }
+      reinterpret_cast<float4*>(ld)[lane] = make_float4(lv[0], lv[1], lv[2], lv[3]);
+      reinterpret_cast<float4*>(ld + 128)[lane] = make_float4(dv4[0], dv4[1], dv4[2], dv4[3]);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar(B_QF(s)), 2 * C::kTileBytes);
+        for (int pn = 0; pn < C::kPanels; ++pn) {
+          tma_load_3d(qAddr(s) + pn * C::kPanelBytes, &p.tm_q, bar(B_QF(s)), pn * 64, i * 128, bh);
+          tma_load_3d(doAddr(s) + pn * C::kPanelBytes, &p.tm_do, bar(B_QF(s)), pn * 64, i * 128, bh);
+        }
+      }
+      ++issued;
+    }
+    if (lane == 0 && *abort_flag) {
+      volatile int never = 0;
+      const Abort drain{&never, p.status};
+      mbar_wait(bar(B_KV), 0, drain, kSiteBDrain);
+      const int first = issued > NS ? issued - NS : 0;
+      for (int q = first; q < issued; ++q) mbar_wait(bar(B_QF(q % NS)), (q / NS) & 1, drain, kSiteBDrain);
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdescKK = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
+      constexpr uint32_t kIdescTS = idesc_bf16_f32(128, D, false, true);      // dV, dK
+      constexpr uint32_t kIdescQ = idesc_bf16_f32(128, D, true, true);        // dQ
+      auto gemm_kk = [&](uint32_t dcol, uint32_t a_addr, uint32_t b_addr) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * C::kPanelBytes + (kk % 4) * 32;
+          mma_f16_ss(tmem + dcol, smem_desc_sw128(a_addr + off, 16, 1024),
+                     smem_desc_sw128(b_addr + off, 16, 1024), kIdescKK, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto gemm_ts = [&](uint32_t dcol, uint32_t a_col, uint32_t b_addr, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_f16_ts(tmem + dcol, tmem + a_col + kk * 8,
+                     smem_desc_sw128(b_addr + kk * 2048, C::kPanelBytes, 1024), kIdescTS,
+                     (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(bar(B_KV), 0, ab, kSiteBMmaKV);
+      for (int idx = 0; idx < n_i && ok; ++idx) {
+        const int s = idx % NS;
+        if (!(ok = mbar_wait(bar(B_QF(s)), (idx / NS) & 1, ab, kSiteBMmaQ))) break;
+        tc_fence_after();
+        gemm_kk(C::kColDP, vAddr, doAddr(s));                    // dP^T = V dO^T
+        tc_commit(bar(B_DP));
+        if (idx > 0) {
+          if (!(ok = mbar_wait(bar(B_DQFREE), (idx - 1) & 1, ab, kSiteBMmaFree))) break;
+          tc_fence_after();
+        }
+        gemm_kk(C::kColS, kAddr, qAddr(s));                      // S^T = K Q^T
+        tc_commit(bar(B_S));
+        if (!(ok = mbar_wait(bar(B_P), idx & 1, ab, kSiteBMmaP))) break;
+        tc_fence_after();
+        gemm_ts(C::kColDV, C::kColS, doAddr(s), idx > 0);        // dV += P^T dO
+        if (!(ok = mbar_wait(bar(B_DS), idx & 1, ab, kSiteBMmaDS))) break;
+        tc_fence_after();
+        gemm_ts(C::kColDK, C::kColDP, qAddr(s), idx > 0);        // dK += dS^T Q
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)                           // dQ_i = dS K
+          mma_f16_ss(tmem + C::kColS, smem_desc_sw128(dsAddr + kk * 2048, C::kPanelBytes, 1024),
+                     smem_desc_sw128(kAddr + kk * 2048, C::kPanelBytes, 1024), kIdescQ,
+                     kk > 0 ? 1u : 0u);
+        tc_commit(bar(B_DQ));
+        tc_commit(bar(B_QE(s)));
+      }
+      tc_commit(bar(B_FINAL));
+      tc_commit(bar(B_DRAIN));
+      volatile int never = 0;
+      const Abort drain{&never, p.status};
+      mbar_wait(bar(B_DRAIN), 0, drain, kSiteBDrain);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ P, dS (thread = key row)
+    const int r = threadIdx.x;
+    const int key = j * 128 + r;
+    const bool key_ok = key < p.N;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tS = tmem + C::kColS + lane_off;
+    const uint32_t tDP = tmem + C::kColDP + lane_off;
+    const float cs = p.scale_log2;
+    bool ok = true;
+    for (int idx = 0; idx < n_i && ok; ++idx) {
+      const int i = i0 + idx;
+      const int s = idx % NS;
+      const float* L2s = reinterpret_cast<const float*>(smem + C::kOffLD + s * 1024);
+      const float* Ds = L2s + 128;
+      const bool diag = CAUSAL && i == j;
+      if (!(ok = mbar_wait_warp(bar(B_S), idx & 1, ab, kSiteBSmS))) break;
+      tc_fence_after();
+      {
+        uint32_t u[128];
+        tmem_ld128(tS, u);
+#pragma unroll
+        for (int c4 = 0; c4 < 32; ++c4) {
+          const float4 l4 = reinterpret_cast<const float4*>(L2s)[c4];
+          const float lq[4] = {l4.x, l4.y, l4.z, l4.w};
+          float pv[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int c = 4 * c4 + t;
+            float x = fmaf(__uint_as_float(u[c]), cs, -lq[t]);
+            if (diag && r > c) x = -INFINITY;     // key after query
+            pv[t] = ex2_sfu(x);
+          }
+          if (!key_ok) pv[0] = pv[1] = pv[2] = pv[3] = 0.f;
+          u[2 * c4] = pack_bf16x2(pv[0], pv[1]);
+          u[2 * c4 + 1] = pack_bf16x2(pv[2], pv[3]);
+        }
+        tmem_st64(tS, *reinterpret_cast<uint32_t(*)[64]>(&u[0]));
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(B_P));
+      if (!(ok = mbar_wait_warp(bar(B_DP), idx & 1, ab, kSiteBSmDP))) break;
+      if (idx > 0 && !(ok = mbar_wait_warp(bar(B_DQ), (idx - 1) & 1, ab, kSiteBSmDQ))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {                 // queries 64h .. 64h+63
+        uint32_t dp[64], pp[32], ds[32];
+        tmem_ld32(tDP + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+        tmem_ld32(tDP + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+        tmem_ld32(tS + 32 * h, pp);
+#pragma unroll
+        for (int c2 = 0; c2 < 32; ++c2) {
+          const int c = 64 * h + 2 * c2;
+          const float p0 = __uint_as_float(pp[c2] << 16), p1 = __uint_as_float(pp[c2] & 0xFFFF0000u);
+          const float d0 = p0 * (__uint_as_float(dp[2 * c2]) - Ds[c]);
+          const float d1 = p1 * (__uint_as_float(dp[2 * c2 + 1]) - Ds[c + 1]);
+          ds[c2] = pack_bf16x2(d0, d1);
+        }
+        tmem_st32(tDP + 32 * h, ds);
+        const uint32_t row = dsAddr + h * C::kPanelBytes + r * 128;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          st_shared_v4b(row + ((q ^ (r & 7)) << 4), ds[4 * q], ds[4 * q + 1], ds[4 * q + 2], ds[4 * q + 3]);
+      }
+      tmem_st_wait();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(B_DS));
+    }
+    if (ok) ok = mbar_wait_warp(bar(B_FINAL), 0, ab, kSiteBEpi);
+    ok = named_bar_and(1, 128, ok);
+    if (ok) {
+      // Every lane takes part in the warp-collective TMEM loads; only the
+      // global stores depend on the key being inside the sequence.
+      tc_fence_after();
+      const size_t g = (static_cast<size_t>(bh) * p.N + (key_ok ? key : 0)) * D;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {      // 0: dV, 1: dK (times scale)
+        const uint32_t src = tmem + (which ? C::kColDK : C::kColDV) + lane_off;
+        uint16_t* dst = (which ? p.dk : p.dv) + g;
+        const float mul = which ? p.scale : 1.f;
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t u[32];
+          tmem_ld32(src + 32 * ch, u);
+          uint32_t pk[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t)
+            pk[t] = pack_bf16x2(__uint_as_float(u[2 * t]) * mul, __uint_as_float(u[2 * t + 1]) * mul);
+          if (key_ok) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              st_global_v4(dst + 32 * ch + 8 * q, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ dQ reduction (thread = query row)
+    const int r = threadIdx.x - 128;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    bool ok = true;
+    for (int idx = 0; idx < n_i && ok; ++idx) {
+      const int row = (i0 + idx) * 128 + r;
+      if (!(ok = mbar_wait_warp(bar(B_DQ), idx & 1, ab, kSiteBDq))) break;
+      tc_fence_after();
+      float* dst = p.dq_acc + (static_cast<size_t>(bh) * p.N + row) * D;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t u[32];
+        tmem_ld32(tmem + C::kColS + lane_off + 32 * ch, u);
+        if (row < p.N) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            red_add_v4(dst + 32 * ch + 4 * q, __uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1]),
+                       __uint_as_float(u[4 * q + 2]), __uint_as_float(u[4 * q + 3]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(B_DQFREE));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int D, bool CAUSAL>
+cudaError_t launch_main_impl(const BwdParams& p, cudaStream_t stream) {
+  using C = BwdCfg<D>;
+  auto kern = bwd_main_kernel<D, CAUSAL>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(p.n_kv) * static_cast<unsigned>(p.BH);
+  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(p);
+  return cudaGetLastError();
+}
+
+unsigned elementwise_grid(long long items) {
+  const long long blocks = (items + 255) / 256;
+  return static_cast<unsigned>(blocks < 148LL * 16 ? (blocks > 0 ? blocks : 1) : 148LL * 16);
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_preprocess(const uint16_t* o, const uint16_t* dout, float* delta,
+                                  float* dq_acc, long long rows, int d, cudaStream_t stream) {
+  const unsigned grid = elementwise_grid(rows * (d / 8));
+  if (d == 64)
+    bwd_preprocess_kernel<64><<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(o),
+                                                        reinterpret_cast<const uint4*>(dout), delta,
+                                                        reinterpret_cast<float4*>(dq_acc), rows);
+  else
+    bwd_preprocess_kernel<128><<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(o),
+                                                         reinterpret_cast<const uint4*>(dout), delta,
+                                                         reinterpret_cast<float4*>(dq_acc), rows);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_main(const BwdParams& p, int d, bool causal, cudaStream_t stream) {
+  if (d == 64) return causal ? launch_main_impl<64, true>(p, stream) : launch_main_impl<64, false>(p, stream);
+  return causal ? launch_main_impl<128, true>(p, stream) : launch_main_impl<128, false>(p, stream);
+}
+
+cudaError_t launch_bwd_postprocess(const float* dq_acc, uint16_t* dq, long long n, float scale,
+                                   cudaStream_t stream) {
+  const long long n4 = n / 4;
+  bwd_postprocess_kernel<<<elementwise_grid(n4), 256, 0, stream>>>(
+      reinterpret_cast<const float4*>(dq_acc), reinterpret_cast<uint2*>(dq), n4, scale);
+  return cudaGetLastError();
+}
+
+}  // namespace fa

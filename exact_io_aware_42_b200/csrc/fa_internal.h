@@ -41,4 +41,31 @@ constexpr int kDefaultPolyPairsD64 = 4;
 
 cudaError_t launch_fwd_bf16(const FwdParams& p, int d, bool causal, cudaStream_t stream);
 
+struct BwdParams {
+  CUtensorMap tm_q;     // bf16 [BH, N, d], box {64, 128, 1}
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  CUtensorMap tm_do;
+  const float* lse;     // [BH, N], natural log
+  const float* delta;   // [BH, N], D = rowsum(dO o O)
+  float* dq_acc;        // [BH, N, d] fp32, zeroed by the preprocess kernel
+  uint16_t* dk;         // bf16 [BH, N, d]
+  uint16_t* dv;
+  unsigned int* status;
+  int N;
+  int BH;
+  int n_kv;             // ceil(N / 128): key blocks = CTAs per (b, h)
+  int n_q;              // ceil(N / 128): query blocks
+  float scale_log2;     // scale * log2(e)
+  float scale;
+};
+
+// D = rowsum(dO o O) per row, and dq_acc <- 0.
+cudaError_t launch_bwd_preprocess(const uint16_t* o, const uint16_t* dout, float* delta,
+                                  float* dq_acc, long long rows, int d, cudaStream_t stream);
+cudaError_t launch_bwd_main(const BwdParams& p, int d, bool causal, cudaStream_t stream);
+// dq <- bf16(scale * dq_acc)
+cudaError_t launch_bwd_postprocess(const float* dq_acc, uint16_t* dq, long long n, float scale,
+                                   cudaStream_t stream);
+
 }  // namespace fa

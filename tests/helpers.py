@@ -5,7 +5,10 @@ Tolerances (fixed by the target of this library, stated once here):
   LSE            max |err| <= 1e-4
   dQ, dK, dV     relative RMS <= 1e-2
   FP8 forward O  relative RMS <= 5e-2 (vs the fp64 oracle on unquantised inputs)
-relative RMS = sqrt(mean((x - ref)^2)) / sqrt(mean(ref^2)).
+relative RMS = sqrt(mean((x - ref)^2)) / sqrt(mean(ref^2)); for gradients the
+denominator is floored at 1e-3 (absolute), because some exact gradients are
+identically zero (N = 1: P = 1, so dS = 0 and dQ = dK = 0) and a relative
+error against zero is undefined.
 """
 import numpy as np
 import torch
@@ -23,10 +26,13 @@ def f64(t) -> np.ndarray:
     return np.asarray(t, dtype=np.float64)
 
 
-def rel_rms(x, ref) -> float:
+def rel_rms(x, ref, floor: float = 1e-300) -> float:
     x, ref = f64(x), f64(ref)
     den = np.sqrt(np.mean(ref ** 2))
-    return float(np.sqrt(np.mean((x - ref) ** 2)) / max(den, 1e-300))
+    return float(np.sqrt(np.mean((x - ref) ** 2)) / max(den, floor))
+
+
+GRAD_RMS_FLOOR = 1e-3
 
 
 def max_abs(x, ref) -> float:
