@@ -148,10 +148,20 @@ def build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs):
     """The hot path as a list of (stage name, callable, FLOPs, kernel launches)."""
     state = {}
 
-    def s_fwd():
-        state["o"], state["lse"] = fa.fwd(q, k, v, causal=causal)
+    ws = torch.empty(fa.bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=q.device)
+    bufs = {n: torch.empty_like(q) for n in ("o", "dq", "dk", "dv")}
+    bufs["lse"] = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
 
-    stages = [("fwd_bf16", s_fwd, fwd_flops(B, H, N, d, causal), 1)]
+    def s_fwd():
+        state["o"], state["lse"] = fa.fwd(q, k, v, causal=causal, out=bufs["o"], lse=bufs["lse"])
+
+    def s_bwd():
+        state["dq"], state["dk"], state["dv"] = fa.bwd(
+            q, k, v, bufs["o"], do, bufs["lse"], causal=causal, workspace=ws,
+            dq=bufs["dq"], dk=bufs["dk"], dv=bufs["dv"])
+
+    f = fwd_flops(B, H, N, d, causal)
+    stages = [("fwd_bf16", s_fwd, f, 1), ("bwd_bf16", s_bwd, 2.5 * f, 3)]
     return stages, state
 
 
@@ -236,7 +246,7 @@ def run_reference(args):
 
 
 METRIC = "attention fwd/bwd TFLOPS (BF16 causal+non-causal) and % of B200 tensor peak"
-STAGES_WITH_BWD = False
+STAGES_WITH_BWD = True
 
 
 def config_block():
