@@ -23,6 +23,8 @@ SIGNATURES = {
     "fa_bwd_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int]),
     "fa_bwd": (c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, c_int, c_int, c_int, c_int, c_float,
                        c_int, _P, c_size_t, _P]),
+    "fa_bwd_noalloc": (c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, c_int, c_int, c_int, c_int,
+                               c_float, c_int, _P]),
     "fa_quant_fp8": (c_int, [_P, _P, _P, c_int, c_int, c_int, c_int, _P, _P]),
     "fa_fwd_fp8": (c_int, [_P, _P, _P, _P, _P, _P, _P, _P, c_int, c_int, c_int, c_int, c_float,
                            c_int, _P]),
@@ -33,7 +35,7 @@ SIGNATURES = {
 
 STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_MISALIGNED",
           4: "FA_ERR_WORKSPACE", 5: "FA_ERR_LAUNCH", 6: "FA_ERR_PIPELINE_TIMEOUT",
-          7: "FA_ERR_NO_DEVICE"}
+          7: "FA_ERR_NO_DEVICE", 8: "FA_ERR_SCRATCH_LIMIT"}
 
 
 class FaError(RuntimeError):

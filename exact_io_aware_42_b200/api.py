@@ -130,3 +130,21 @@ def get_status() -> int:
 
 def clear_status() -> None:
     lib().fa_clear_status()
+
+
+def bwd_noalloc(q, k, v, o, do, lse, causal: bool = False, scale: Optional[float] = None,
+                dq=None, dk=None, dv=None):
+    """Backward with the library's built-in scratch instead of a workspace
+    (for callers that cannot allocate device memory; see fa_bwd_noalloc)."""
+    _check_bhnd("q", q, torch.bfloat16)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    code = lib().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
+                                _ptr(dk), _ptr(dv), B, H, N, d, float(scale), int(bool(causal)),
+                                _stream())
+    check("fa_bwd_noalloc", code)
+    return dq, dk, dv

@@ -253,6 +253,7 @@ extern "C" const char* fa_status_string(int s) {
     case FA_ERR_LAUNCH: return "FA_ERR_LAUNCH";
     case FA_ERR_PIPELINE_TIMEOUT: return "FA_ERR_PIPELINE_TIMEOUT";
     case FA_ERR_NO_DEVICE: return "FA_ERR_NO_DEVICE";
+    case FA_ERR_SCRATCH_LIMIT: return "FA_ERR_SCRATCH_LIMIT";
     default: return "FA_ERR_UNKNOWN";
   }
 }

@@ -28,8 +28,9 @@
  *  - A pipeline wait inside a kernel that exceeds ~2 s gives up: the kernel
  *    ends early and records FA_ERR_PIPELINE_TIMEOUT in a device status word
  *    that fa_get_status() reads after the caller has synchronised.
- *  - The library keeps no state besides that status word and per-process
- *    caches of kernel attributes; calls on different streams may overlap.
+ *  - The library keeps no state besides that status word, the scratch array
+ *    of fa_bwd_noalloc and per-process caches of kernel attributes; calls on
+ *    different streams may overlap (except fa_bwd_noalloc calls, see there).
  */
 #ifndef FA_B200_H_
 #define FA_B200_H_
@@ -49,7 +50,8 @@ typedef enum fa_status {
   FA_ERR_WORKSPACE = 4,        /* workspace null or smaller than required    */
   FA_ERR_LAUNCH = 5,           /* CUDA reported an error at launch           */
   FA_ERR_PIPELINE_TIMEOUT = 6, /* a bounded in-kernel wait ran out           */
-  FA_ERR_NO_DEVICE = 7         /* no CUDA device / driver entry point        */
+  FA_ERR_NO_DEVICE = 7,        /* no CUDA device / driver entry point        */
+  FA_ERR_SCRATCH_LIMIT = 8     /* fa_bwd_noalloc: problem exceeds its scratch */
 } fa_status;
 
 /*
@@ -90,6 +92,30 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                  const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                  float scale, int causal, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Allocation-free backward.  No counterpart in the papers: it exists for
+ * callers that cannot allocate device memory themselves (code inside a host
+ * framework that owns all device memory through its own pool, or a
+ * latency-critical path where cudaMalloc's device synchronisation is not
+ * acceptable).  Same arguments and results as fa_bwd, without the
+ * workspace: the scratch is a device array built into the library, of
+ * FA_BWD_NOALLOC_SCRATCH_BYTES (32 MiB), held on every GPU that loads the
+ * library until the process exits.  Nothing is allocated or freed.
+ *  - Problems whose fa_bwd_workspace_size() exceeds that size are rejected
+ *    with FA_ERR_SCRATCH_LIMIT before any launch (at d = 128 that is
+ *    B * H * N above 65,027 rows; at d = 64, above 129,055).
+ *  - The first call on a device looks up the array's device address on that
+ *    device (cudaGetSymbolAddress); make that first call before any stream
+ *    capture.
+ *  - All calls share the one array, which keeps the previous call's
+ *    contents (the part that must start at zero is cleared on every call).
+ *    Calls that can overlap on the GPU race on it: serialise them.
+ */
+#define FA_BWD_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                         int H, int N, int d, float scale, int causal, void* stream);
 
 /*
  * FP8 block quantisation of one tensor ("the librarian" page, "FA3 -- the
