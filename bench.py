@@ -64,23 +64,26 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def kernel_source_hash():
+def kernel_source_hash(which: str):
     h = hashlib.sha256()
-    for name in ("fa_fwd.cu", "fa_ptx.cuh", "fa_exp2.cuh", "fa_exp2_poly.h", "fa_internal.h"):
+    main = "fa_fwd.cu" if which == "fwd" else "fa_bwd.cu"
+    for name in (main, "fa_ptx.cuh", "fa_exp2.cuh", "fa_exp2_poly.h", "fa_internal.h"):
         with open(os.path.join(ROOT, "exact_io_aware_42_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
-    """DRAM bytes per forward launch from the committed ncu summary, if it was
-    taken on the current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", "fwd_bf16_B4_H16_N4096_d128_causal.md")
+def profiled_traffic(which: str):
+    """DRAM bytes per launch of the forward ("fwd") or backward main ("bwd")
+    kernel from the committed ncu summary, if that capture was taken on the
+    current kernel source (else None)."""
+    name = "fwd_bf16" if which == "fwd" else "bwd_main_bf16"
+    path = os.path.join(ROOT, "profiles", f"{name}_B4_H16_N4096_d128_causal.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)\s+source_sha:\s*([0-9a-f]+)", text)
-    if not m or m.group(2) != kernel_source_hash():
+    if not m or m.group(2) != kernel_source_hash(which):
         return None
     return float(m.group(1))
 
@@ -101,7 +104,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -160,8 +163,24 @@ def build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs):
             q, k, v, bufs["o"], do, bufs["lse"], causal=causal, workspace=ws,
             dq=bufs["dq"], dk=bufs["dk"], dv=bufs["dv"])
 
+    q8 = {n: torch.empty(q.shape, dtype=torch.uint8, device=q.device) for n in ("q", "k", "v")}
+    sc8 = {n: torch.empty((B, H, fa.n_blocks(N)), dtype=torch.float32, device=q.device)
+           for n in ("q", "k", "v")}
+    o8 = torch.empty_like(q)
+    lse8 = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+
+    def s_quant():
+        fa.quant_fp8(q, signs, out=q8["q"], scales=sc8["q"])
+        fa.quant_fp8(k, signs, out=q8["k"], scales=sc8["k"])
+        fa.quant_fp8(v, None, out=q8["v"], scales=sc8["v"])
+
+    def s_fwd8():
+        state["o_fp8"], state["lse_fp8"] = fa.fwd_fp8(q8["q"], q8["k"], q8["v"], sc8["q"], sc8["k"],
+                                                      sc8["v"], causal=causal, out=o8, lse=lse8)
+
     f = fwd_flops(B, H, N, d, causal)
-    stages = [("fwd_bf16", s_fwd, f, 1), ("bwd_bf16", s_bwd, 2.5 * f, 3)]
+    stages = [("fwd_bf16", s_fwd, f, 1), ("bwd_bf16", s_bwd, 2.5 * f, 3),
+              ("quant_fp8", s_quant, 0.0, 3), ("fwd_fp8", s_fwd8, f, 1)]
     return stages, state
 
 
@@ -211,13 +230,20 @@ def oracle_sample(budget_s: float, B, H, N, d, causal, with_bwd: bool):
         if with_bwd:
             oracle.attn_bwd_ref(q[sl], k[sl], v[sl], do[sl], sc, causal)
             flops += 2.5 * fwd_flops(1, 1, N, d, causal)
+            # FP8 rows: block quantisation (Q, K rotated; V) and attention on the
+            # dequantised values
+            sg = inputs.signs(d).numpy()
+            deq = [oracle.dequant_fp8_ref(*oracle.quant_fp8_ref(x[sl].double().numpy(), rot, sg))
+                   for x, rot in ((q, True), (k, True), (v, False))]
+            oracle.attn_fwd_ref(deq[0], deq[1], deq[2], sc, causal)
+            flops += fwd_flops(1, 1, N, d, causal)
         heads += 1
         if time.perf_counter() - t0 >= budget_s:
             break
     dt = time.perf_counter() - t0
     return {"value": flops / dt / 1e12, "unit": "TFLOPS", "cores": int(cores), "kind": "oracle",
             "sample": f"{heads} of {B * H} heads of {WORKLOAD['name']}, fwd"
-                      + ("+bwd" if with_bwd else "") + f", fp64 numpy, {dt:.1f} s"}
+                      + ("+bwd+fp8 quant/fwd" if with_bwd else "") + f", fp64 numpy, {dt:.1f} s"}
 
 
 def run_reference(args):
@@ -255,7 +281,8 @@ def config_block():
             "causal": w["causal"], "global_batch": w["B"], "seq_len": w["N"],
             "parallelism": "independent replicas per GPU (heads), no collective",
             "l2": "inputs 4 x 64 MiB > 126 MB L2, no flush",
-            "step": "fwd_bf16" + (" + bwd_bf16" if STAGES_WITH_BWD else "")}
+            "step": "fwd_bf16 + bwd_bf16 + quant_fp8 (Q, K rotated; V) + fwd_fp8",
+            "fp8": "quantisation and forward in E4M3 (kind::f8f6f4), counted at forward FLOPs"}
 
 
 def run_ours(args):
@@ -339,10 +366,16 @@ def run_ours(args):
     barrier()
 
     peaks, peak_src = measured_peaks()
-    fwd_idx = [i for i, s in enumerate(stages) if s[0] == "fwd_bf16"][0]
-    fwd_ms = per_stage[fwd_idx]
-    achieved = stages[fwd_idx][2] / (fwd_ms * 1e-3) / 1e12
+    idx = {st[0]: i for i, st in enumerate(stages)}
     peak = float(peaks["bf16_tflops_sustained"])
+
+    def roof(name, kernel, nbytes):
+        ms = per_stage[idx[name]]
+        ach = stages[idx[name]][2] / (ms * 1e-3) / 1e12
+        return {"kernel": kernel, "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                "frac": ach / peak,
+                "peak_source": f"{peak_src} bf16_tflops_sustained (timed inside the step loop)",
+                "algorithmic_bytes": nbytes}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -351,11 +384,10 @@ def run_ours(args):
                         "nominal_2250": value / world / 2250.0},
         "stages": {s[0]: {"ms": per_stage[i], "tflops": s[2] / (per_stage[i] * 1e-3) / 1e12}
                    for i, s in enumerate(stages)},
-        "roofline": {"kernel": "fwd_bf16_kernel<128, causal>", "bound": "tensor",
-                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside the step loop)",
-                     "traffic": profiled_traffic(),
-                     "algorithmic_bytes": fwd_bytes(B, H, N, d)},
+        "roofline": dict(roof("bwd_bf16", "bwd_main_kernel<128, causal> (+ pre/post kernels in the timed call)",
+                              bwd_bytes(B, H, N, d)), traffic=profiled_traffic("bwd")),
+        "roofline_fwd": dict(roof("fwd_bf16", "fwd_kernel<128, causal, bf16>", fwd_bytes(B, H, N, d)),
+                             traffic=profiled_traffic("fwd")),
         "e2e": {"value": world * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
@@ -375,7 +407,7 @@ def run_ours(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--ref-seconds", type=float, default=12.0,

@@ -218,15 +218,68 @@ extern "C" fa_status fa_bwd(const void* q, const void* k, const void* v, const v
   return FA_OK;
 }
 
-extern "C" fa_status fa_quant_fp8(const void*, void*, float*, int, int, int, int, const float*,
-                                  void*) {
-  return FA_ERR_UNSUPPORTED;
+extern "C" fa_status fa_quant_fp8(const void* x, void* x8, float* scales, int B, int H, int N,
+                                  int d, const float* signs, void* stream) {
+  if (B < 0 || H < 0 || N < 0) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (N > kMaxN || static_cast<long long>(B) * H > kMaxBH) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H * N == 0) return FA_OK;
+  if (!x || !x8 || !scales) return FA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x8) || (reinterpret_cast<uintptr_t>(scales) & 3u) ||
+      (reinterpret_cast<uintptr_t>(signs) & 3u))
+    return FA_ERR_MISALIGNED;
+  DeviceInfo* di = nullptr;
+  fa_status st = current_device(&di);
+  if (st != FA_OK) return st;
+  cudaError_t e = launch_quant_fp8(static_cast<const uint16_t*>(x), static_cast<uint8_t*>(x8), scales,
+                                   signs, B * H, N, d, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+  }
+  return FA_OK;
 }
 
-extern "C" fa_status fa_fwd_fp8(const void*, const void*, const void*, const float*,
-                                const float*, const float*, void*, float*, int, int, int, int,
-                                float, int, void*) {
-  return FA_ERR_UNSUPPORTED;
+extern "C" fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* sq,
+                                const float* sk, const float* sv, void* o, float* lse, int B, int H,
+                                int N, int d, float scale, int causal, void* stream) {
+  fa_status st = check_shape(B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H * N == 0) return FA_OK;
+  if (!q8 || !k8 || !v8 || !sq || !sk || !sv || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o) ||
+      ((reinterpret_cast<uintptr_t>(lse) | reinterpret_cast<uintptr_t>(sq) |
+        reinterpret_cast<uintptr_t>(sk) | reinterpret_cast<uintptr_t>(sv)) & 3u))
+    return FA_ERR_MISALIGNED;
+  DeviceInfo* di = nullptr;
+  if ((st = current_device(&di)) != FA_OK) return st;
+  FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  const int BH = B * H;
+  const CUtensorMapDataType u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  if (!encode_3d(&p.tm_q, q8, u8, 1, d, N, BH, 128, kBlockM) ||
+      !encode_3d(&p.tm_k, k8, u8, 1, d, N, BH, 128, kBlockN) ||
+      !encode_3d(&p.tm_v, v8, u8, 1, d, N, BH, 128, kBlockN) ||
+      !encode_3d(&p.tm_o, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, BH, 64, kBlockM))
+    return FA_ERR_INVALID_ARG;
+  p.lse = lse;
+  p.status = di->status;
+  p.sq = sq;
+  p.sk = sk;
+  p.sv = sv;
+  p.N = N;
+  p.BH = BH;
+  p.n_kv = (N + kBlockN - 1) / kBlockN;
+  p.n_pairs = ((N + kBlockM - 1) / kBlockM + 1) / 2;
+  p.scale = scale;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  cudaError_t e = launch_fwd_fp8(p, causal != 0, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+  }
+  return FA_OK;
 }
 
 extern "C" unsigned int fa_get_status(void) {

@@ -43,15 +43,21 @@
 namespace fa {
 namespace {
 
-template <int D>
+template <int D, bool FP8 = false>
 struct FwdCfg {
-  static constexpr int kPanels = D / 64;             // 128-byte swizzle panels per row
-  static constexpr int kPanelBytes = 128 * 128;      // 128 rows x 128 bytes
-  static constexpr int kTileBytes = kBlockM * D * 2; // one 128 x D bf16 tile
-  static constexpr int kStages = (D == 128) ? 5 : 8;
+  static constexpr int kElem = FP8 ? 1 : 2;            // bytes per Q/K/V element
+  static constexpr int kPanels = D * kElem / 128;      // 128-byte swizzle panels per row
+  static constexpr int kPanelElems = 128 / kElem;      // elements per panel row
+  static constexpr int kPanelBytes = 128 * 128;        // 128 rows x 128 bytes
+  static constexpr int kTileBytes = kBlockM * D * kElem;   // one 128 x D tile
+  static constexpr int kStages = FP8 ? 8 : ((D == 128) ? 5 : 8);
   static constexpr int kThreads = 320;
-  static constexpr int kOffQ = 0;                    // two query tiles
-  static constexpr int kOffRing = 2 * kTileBytes;
+  static constexpr int kOffQ = 0;                      // two query tiles
+  // bf16 O is staged in the Q tile it replaces; FP8 tiles are half as large,
+  // so FP8 stages O in a buffer of its own (2 x 128 x D bf16).
+  static constexpr int kOffO = FP8 ? 2 * kTileBytes : 0;
+  static constexpr int kOBytes = kBlockM * D * 2;
+  static constexpr int kOffRing = FP8 ? kOffO + 2 * kOBytes : 2 * kTileBytes;
   static constexpr int kOffBar = kOffRing + kStages * kTileBytes;
   static constexpr int kNumBars = 2 + 2 * kStages + 7;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
@@ -60,6 +66,8 @@ struct FwdCfg {
   static constexpr uint32_t kColS = 0;       // + 128 * t
   static constexpr uint32_t kColO = 256;     // + D * t
 };
+static_assert(FwdCfg<128, true>::kSmemBytes <= 232448, "fp8 forward shared memory");
+static_assert(FwdCfg<128, false>::kSmemBytes <= 232448, "bf16 forward shared memory");
 
 // barrier slots
 __device__ __forceinline__ int bar_q(int t) { return t; }
@@ -81,11 +89,20 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
+// E4M3 byte pair <- (lo, hi), round to nearest even, saturating at +-448.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  unsigned short lo, hi;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
 // NPOLY of every 8 column pairs take the polynomial exp2 (degree DEG), the
-// rest the SFU.
-template <int D, bool CAUSAL, int NPOLY, int DEG>
-__global__ void __launch_bounds__(320, 1) fwd_bf16_kernel(const __grid_constant__ FwdParams p) {
-  using C = FwdCfg<D>;
+// rest the SFU.  FP8: Q, K, V are E4M3 with per-128-row block scales and both
+// products run as kind::f8f6f4 (see the FP8 notes at the softmax).
+template <int D, bool CAUSAL, int NPOLY, int DEG, bool FP8>
+__global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ FwdParams p) {
+  using C = FwdCfg<D, FP8>;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -141,7 +158,7 @@ __global__ void __launch_bounds__(320, 1) fwd_bf16_kernel(const __grid_constant_
         mbar_arrive_expect_tx(bar(bar_q(t)), C::kTileBytes);
         for (int pn = 0; pn < C::kPanels; ++pn)
           tma_load_3d(sbase + C::kOffQ + t * C::kTileBytes + pn * C::kPanelBytes, &p.tm_q,
-                      bar(bar_q(t)), pn * 64, (qt0 + t) * kBlockM, bh);
+                      bar(bar_q(t)), pn * C::kPanelElems, (qt0 + t) * kBlockM, bh);
       }
       int seq = 0;
       bool ok = true;
@@ -154,7 +171,7 @@ __global__ void __launch_bounds__(320, 1) fwd_bf16_kernel(const __grid_constant_
           const CUtensorMap* m = (w == 0) ? &p.tm_k : &p.tm_v;
           for (int pn = 0; pn < C::kPanels; ++pn)
             tma_load_3d(sbase + C::kOffRing + s * C::kTileBytes + pn * C::kPanelBytes, m,
-                        bar(bar_full<NS>(s)), pn * 64, j * kBlockN, bh);
+                        bar(bar_full<NS>(s)), pn * C::kPanelElems, j * kBlockN, bh);
           ++seq;
         }
       }
@@ -173,26 +190,38 @@ __global__ void __launch_bounds__(320, 1) fwd_bf16_kernel(const __grid_constant_
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t kIdescO = idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t kIdescS =
+          FP8 ? idesc_e4m3_f32(128, 128, false, false) : idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t kIdescO =
+          FP8 ? idesc_e4m3_f32(128, D, false, true) : idesc_bf16_f32(128, D, false, true);
+      constexpr int kK = FP8 ? 32 : 16;            // K elements per MMA (32 bytes)
       const uint32_t q_addr[2] = {sbase + C::kOffQ, sbase + C::kOffQ + C::kTileBytes};
       auto ring = [&](int s) -> uint32_t { return sbase + C::kOffRing + s * C::kTileBytes; };
       auto issue_s = [&](int t, uint32_t k_addr) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < D / kK; ++kk) {
           const uint32_t off = (kk / 4) * C::kPanelBytes + (kk % 4) * 32;
           const uint64_t a = smem_desc_sw128(q_addr[t] + off, 16, 1024);
           const uint64_t b = smem_desc_sw128(k_addr + off, 16, 1024);
-          mma_f16_ss(tmem + C::kColS + 128 * t, a, b, kIdescS, kk > 0 ? 1u : 0u);
+          if constexpr (FP8)
+            mma_f8_ss(tmem + C::kColS + 128 * t, a, b, kIdescS, kk > 0 ? 1u : 0u);
+          else
+            mma_f16_ss(tmem + C::kColS + 128 * t, a, b, kIdescS, kk > 0 ? 1u : 0u);
         }
         tc_commit(bar(bar_s<NS>(t)));
       };
       auto issue_pv = [&](int t, uint32_t v_addr, bool acc) {
 #pragma unroll
-        for (int kk = 0; kk < kBlockN / 16; ++kk) {
-          const uint64_t b = smem_desc_sw128(v_addr + kk * 16 * 128, C::kPanelBytes, 1024);
-          mma_f16_ts(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + kk * 8, b, kIdescO,
-                     (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kBlockN / kK; ++kk) {
+          // V is MN-major (d contiguous); one K step is kK key rows of 128 bytes.
+          // P in TMEM packs 32 bits per column: 2 bf16 or 4 E4M3 keys.
+          const uint64_t b = smem_desc_sw128(v_addr + kk * kK * 128, C::kPanelBytes, 1024);
+          if constexpr (FP8)
+            mma_f8_ts(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + kk * 8, b, kIdescO,
+                      (acc || kk > 0) ? 1u : 0u);
+          else
+            mma_f16_ts(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + kk * 8, b, kIdescO,
+                       (acc || kk > 0) ? 1u : 0u);
         }
         tc_commit(bar(bar_pv<NS>(t)));
       };
@@ -251,7 +280,19 @@ __global__ void __launch_bounds__(320, 1) fwd_bf16_kernel(const __grid_constant_
     const int qi = qt0 + t;
     const int row = qi * kBlockM + r;
     const int n = n_t[t];
-    const float c = p.scale_log2;
+    // FP8: scores are dequantised per tile pair with s_q(i) * s_k(j); P is
+    // stored as E4M3 times 256 * s_v(j) / max_j s_v(j), which folds V's block
+    // scale into P (p <= 1 because FP8 rescales on every max increase), and O
+    // is multiplied back by max s_v / 256 at the end.
+    const size_t sc_base = static_cast<size_t>(bh) * p.n_kv;
+    float c_q = p.scale_log2;
+    float v_max = 1.f;
+    if constexpr (FP8) {
+      c_q *= (qi < p.n_kv) ? p.sq[sc_base + qi] : 1.f;
+      v_max = 0.f;
+      for (int jj = 0; jj < p.n_kv; ++jj) v_max = fmaxf(v_max, p.sv[sc_base + jj]);
+    }
+    constexpr float kTau = FP8 ? 0.f : kRescaleTau;
     float m_use = -INFINITY;
     float l = 0.f;
     bool ok = true;
@@ -260,6 +301,7 @@ __global__ void __launch_bounds__(320, 1) fwd_bf16_kernel(const __grid_constant_
       tc_fence_after();
       uint32_t u[128];
       tmem_ld128(tS, u);
+      const float c = FP8 ? c_q * p.sk[sc_base + j] : c_q;
       const bool masked = (CAUSAL && j == qi) || ((j + 1) * kBlockN > p.N);
       if (masked) {
         // scaled scores with -inf where the key is hidden or past N
@@ -286,7 +328,7 @@ __global__ void __launch_bounds__(320, 1) fwd_bf16_kernel(const __grid_constant_
         if (!masked) mt *= c;
       }
       const float m_new = fmaxf(m_use, mt);
-      const bool need = m_new > m_use + kRescaleTau;
+      const bool need = m_new > m_use + kTau;
       float alpha = 1.f;
       if (need) {
         alpha = ex2_sfu(m_use - m_new);
@@ -294,29 +336,50 @@ __global__ void __launch_bounds__(320, 1) fwd_bf16_kernel(const __grid_constant_
       }
       const float neg_m = -m_use;
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-      if (masked) {
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float p0 = ex2_sfu(__uint_as_float(u[2 * i]) + neg_m);
-          const float p1 = ex2_sfu(__uint_as_float(u[2 * i + 1]) + neg_m);
-          acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
-          u[i] = pack_bf16x2(p0, p1);       // P overwrites the consumed scores
-        }
-      } else {
+      if constexpr (FP8) {
+        const float f8 = 256.f * p.sv[sc_base + j] / v_max;
         const uint64_t c2 = f2_pack(c, c);
         const uint64_t nm2 = f2_pack(neg_m, neg_m);
+        float keep0 = 0.f, keep1 = 0.f;
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
-          const uint64_t x2 =
-              f2_fma(f2_pack(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1])), c2, nm2);
-          const uint64_t p2 = ((i & 7) < NPOLY) ? exp2_poly_f2<DEG>(x2) : exp2_sfu_f2(x2);
+          const uint64_t s2 = f2_pack(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]));
+          const uint64_t x2 = masked ? f2_add(s2, nm2) : f2_fma(s2, c2, nm2);
+          const uint64_t p2 = exp2_sfu_f2(x2);
           acc[i & 3] = f2_add(acc[i & 3], p2);
           float p0, p1;
           f2_unpack(p2, p0, p1);
-          u[i] = pack_bf16x2(p0, p1);
+          if (i & 1)
+            u[i / 2] = pack_e4m3x4(keep0 * f8, keep1 * f8, p0 * f8, p1 * f8);
+          keep0 = p0;
+          keep1 = p1;
         }
+        tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+      } else {
+        if (masked) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const float p0 = ex2_sfu(__uint_as_float(u[2 * i]) + neg_m);
+            const float p1 = ex2_sfu(__uint_as_float(u[2 * i + 1]) + neg_m);
+            acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
+            u[i] = pack_bf16x2(p0, p1);       // P overwrites the consumed scores
+          }
+        } else {
+          const uint64_t c2 = f2_pack(c, c);
+          const uint64_t nm2 = f2_pack(neg_m, neg_m);
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const uint64_t x2 =
+                f2_fma(f2_pack(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1])), c2, nm2);
+            const uint64_t p2 = ((i & 7) < NPOLY) ? exp2_poly_f2<DEG>(x2) : exp2_sfu_f2(x2);
+            acc[i & 3] = f2_add(acc[i & 3], p2);
+            float p0, p1;
+            f2_unpack(p2, p0, p1);
+            u[i] = pack_bf16x2(p0, p1);
+          }
+        }
+        tmem_st64(tS, *reinterpret_cast<uint32_t(*)[64]>(&u[0]));
       }
-      tmem_st64(tS, *reinterpret_cast<uint32_t(*)[64]>(&u[0]));
       tmem_st_wait();
       float sum4[4];
 #pragma unroll
@@ -353,8 +416,9 @@ __global__ void __launch_bounds__(320, 1) fwd_bf16_kernel(const __grid_constant_
     if (ok) {
       tc_fence_after();
       // ---------------------------------------------------------- epilogue
-      const float inv_l = 1.f / l;
-      const uint32_t o_stage = sbase + C::kOffQ + t * C::kTileBytes;   // Q_t no longer read
+      const float inv_l = (FP8 ? v_max * (1.f / 256.f) : 1.f) / l;
+      // bf16: stage O in Q_t, no longer read; FP8: in its own buffer
+      const uint32_t o_stage = FP8 ? sbase + C::kOffO + t * C::kOBytes : sbase + C::kOffQ + t * C::kTileBytes;
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t u[32];
@@ -374,8 +438,8 @@ __global__ void __launch_bounds__(320, 1) fwd_bf16_kernel(const __grid_constant_
       fence_proxy_async_smem();
       named_bar_sync(1 + t, 128);
       if (r == 0 && qi * kBlockM < p.N) {   // a tile wholly past N is padding
-        for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_store_3d(&p.tm_o, o_stage + pn * C::kPanelBytes, pn * 64, qi * kBlockM, bh);
+        for (int pn = 0; pn < D / 64; ++pn)
+          tma_store_3d(&p.tm_o, o_stage + pn * C::kPanelBytes, pn * 64, qi * kBlockM, bh);   // bf16 O
         tma_store_commit();
         tma_store_wait_all();
       }
@@ -391,10 +455,10 @@ __global__ void __launch_bounds__(320, 1) fwd_bf16_kernel(const __grid_constant_
   }
 }
 
-template <int D, bool CAUSAL, int NPOLY>
+template <int D, bool CAUSAL, int NPOLY, bool FP8>
 cudaError_t launch_impl(const FwdParams& p, cudaStream_t stream) {
-  using C = FwdCfg<D>;
-  auto kern = fwd_bf16_kernel<D, CAUSAL, NPOLY, 3>;
+  using C = FwdCfg<D, FP8>;
+  auto kern = fwd_kernel<D, CAUSAL, NPOLY, 3, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(p.n_pairs) * static_cast<unsigned>(p.BH);
@@ -402,20 +466,24 @@ cudaError_t launch_impl(const FwdParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-}  // namespace
-
 template <int D, bool CAUSAL>
 cudaError_t launch_np(const FwdParams& p, cudaStream_t stream) {
   switch (p.poly_pairs) {
-    case 0: return launch_impl<D, CAUSAL, 0>(p, stream);
-    case 4: return launch_impl<D, CAUSAL, 4>(p, stream);
-    default: return launch_impl<D, CAUSAL, 2>(p, stream);
+    case 0: return launch_impl<D, CAUSAL, 0, false>(p, stream);
+    case 4: return launch_impl<D, CAUSAL, 4, false>(p, stream);
+    default: return launch_impl<D, CAUSAL, 2, false>(p, stream);
   }
 }
+
+}  // namespace
 
 cudaError_t launch_fwd_bf16(const FwdParams& p, int d, bool causal, cudaStream_t stream) {
   if (d == 64) return causal ? launch_np<64, true>(p, stream) : launch_np<64, false>(p, stream);
   return causal ? launch_np<128, true>(p, stream) : launch_np<128, false>(p, stream);
+}
+
+cudaError_t launch_fwd_fp8(const FwdParams& p, bool causal, cudaStream_t stream) {
+  return causal ? launch_impl<128, true, 0, true>(p, stream) : launch_impl<128, false, 0, true>(p, stream);
 }
 
 }  // namespace fa

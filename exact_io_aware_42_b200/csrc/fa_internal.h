@@ -40,6 +40,11 @@ constexpr int kDefaultPolyPairsD128 = 0;
 constexpr int kDefaultPolyPairsD64 = 4;
 
 cudaError_t launch_fwd_bf16(const FwdParams& p, int d, bool causal, cudaStream_t stream);
+// E4M3 forward (d = 128): tm_q/tm_k/tm_v are uint8 maps, sq/sk/sv block scales.
+cudaError_t launch_fwd_fp8(const FwdParams& p, bool causal, cudaStream_t stream);
+// Block quantisation of one bf16 tensor to E4M3 (signs == nullptr: no rotation).
+cudaError_t launch_quant_fp8(const uint16_t* x, uint8_t* x8, float* scales, const float* signs,
+                             int BH, int N, int d, cudaStream_t stream);
 
 struct BwdParams {
   CUtensorMap tm_q;     // bf16 [BH, N, d], box {64, 128, 1}
