@@ -16,9 +16,9 @@
 // Main kernel, per query block i (TMEM lanes are the CTA's 128 keys):
 //   S^T  = K_j Q_i^T            tcgen05 SS   -> TMEM [0,128)
 //   dP^T = V_j dO_i^T           tcgen05 SS   -> TMEM [128,256)
-//   P^T  = 2^(S^T c - L log2 e) softmax warps, bf16 back into TMEM [0,64)
+//   P^T  = 2^(S^T c - L log2 e) softmax warps, bf16 back into TMEM
 //   dV  += P^T dO_i             tcgen05 TS   (A = P^T from TMEM)
-//   dS^T = P^T o (dP^T - D)     softmax warps, bf16 into TMEM [128,192) and
+//   dS^T = P^T o (dP^T - D)     softmax warps, bf16 into TMEM and
 //                               into shared memory (MN-major, 128-B swizzle)
 //   dK  += dS^T Q_i             tcgen05 TS
 //   dQ_i = dS K_j               tcgen05 SS (A = dS, MN-major) -> TMEM [0,d)
@@ -29,10 +29,11 @@
 // L2 (the summation order across key blocks is not fixed, so dQ may differ in
 // the last bits from run to run; dK and dV are deterministic).
 //
-// Roles: warps 0-3 softmax / dS and the dK, dV epilogue (thread = key row);
-// warps 4-7 dQ reduction (thread = query row); warp 8 TMA producer (also
-// stages L and D of each query block in shared memory); warp 9 TMEM owner and
-// the single MMA-issuing thread.  Every wait is bounded (fa_ptx.cuh).
+// Roles: warps 0-7 P / dS and the dK, dV epilogue (thread = key row; warps
+// 0-3 take queries 0..63 of each block, warps 4-7 queries 64..127); warps 8-11
+// dQ reduction (thread = query row); warp 12 TMA producer (also stages L and
+// D of each query block in shared memory); warp 13 TMEM owner and the single
+// MMA-issuing thread.  Every wait is bounded (fa_ptx.cuh).
 #include "fa_internal.h"
 #include "fa_ptx.cuh"
 
@@ -45,7 +46,7 @@ struct BwdCfg {
   static constexpr int kPanelBytes = 128 * 128;
   static constexpr int kTileBytes = 128 * D * 2;       // one 128 x D bf16 tile
   static constexpr int kStages = (D == 128) ? 2 : 3;   // (Q_i, dO_i) ring depth
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 448;
   // All swizzled tiles are 1024-byte aligned offsets from the (1024-aligned)
   // dynamic shared memory base.
   static constexpr int kOffK = 0;
@@ -58,8 +59,12 @@ struct BwdCfg {
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kColS = 0;      // S^T, then P^T (bf16), then dQ_i
-  static constexpr uint32_t kColDP = 128;   // dP^T, then dS^T (bf16)
+  // Two 128-column regions alternate roles per query block idx: region
+  // X = 128 * (idx & 1) holds S^T, then P^T (bf16), then dQ_i; region
+  // Y = 128 - X holds dP^T, then dS^T (bf16).  S^T of the next block goes into
+  // the previous Y, so it never waits for the dQ reduction of the last block.
+  static constexpr uint32_t kColS = 0;
+  static constexpr uint32_t kColDP = 128;
   static constexpr uint32_t kColDV = 256;
   static constexpr uint32_t kColDK = 256 + D;
 };
@@ -142,7 +147,7 @@ __device__ __forceinline__ void st_global_v4(void* dst, uint32_t a, uint32_t b, 
 }
 
 template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(320, 1) bwd_main_kernel(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant__ BwdParams p) {
   using C = BwdCfg<D>;
   constexpr int NS = C::kStages;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -162,8 +167,11 @@ __global__ void __launch_bounds__(320, 1) bwd_main_kernel(const __grid_constant_
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x % p.BH;
-  const int j = blockIdx.x / p.BH;                 // key block; small j (most work) first
+  // Head-major order: the CTAs resident at any time cover a few heads, so
+  // their dQ accumulators (and K, V, Q, dO) stay in L2.  Within a head the
+  // key blocks with the most query blocks (small j, causal) go first.
+  const int bh = blockIdx.x / p.n_kv;
+  const int j = blockIdx.x % p.n_kv;
   const int i0 = CAUSAL ? j : 0;
   const int n_i = p.n_q - i0;
 
@@ -175,8 +183,8 @@ __global__ void __launch_bounds__(320, 1) bwd_main_kernel(const __grid_constant_
     }
     mbar_init(bar(B_S), 1);
     mbar_init(bar(B_DP), 1);
-    mbar_init(bar(B_P), 128);
-    mbar_init(bar(B_DS), 128);
+    mbar_init(bar(B_P), 256);
+    mbar_init(bar(B_DS), 256);
     mbar_init(bar(B_DQ), 1);
     mbar_init(bar(B_DQFREE), 128);
     mbar_init(bar(B_FINAL), 1);
@@ -184,7 +192,7 @@ __global__ void __launch_bounds__(320, 1) bwd_main_kernel(const __grid_constant_
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
     tmem_relinquish();
   }
@@ -197,7 +205,7 @@ __global__ void __launch_bounds__(320, 1) bwd_main_kernel(const __grid_constant_
   auto qAddr = [&](int s) -> uint32_t { return sbase + C::kOffQ + s * 2 * C::kTileBytes; };
   auto doAddr = [&](int s) -> uint32_t { return qAddr(s) + C::kTileBytes; };
 
-  if (warp == 8) {
+  if (warp == 12) {
     // ------------------------------------------------------------ producer
     int issued = 0;
     bool ok = true;
@@ -249,7 +257,7 @@ __global__ void __launch_bounds__(320, 1) bwd_main_kernel(const __grid_constant_
       for (int q = first; q < issued; ++q) mbar_wait(bar(B_QF(q % NS)), (q / NS) & 1, drain, kSiteBDrain);
     }
     __syncwarp();
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdescKK = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
@@ -265,8 +273,8 @@ __global__ void __launch_bounds__(320, 1) bwd_main_kernel(const __grid_constant_
       };
       auto gemm_ts = [&](uint32_t dcol, uint32_t a_col, uint32_t b_addr, bool acc) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_f16_ts(tmem + dcol, tmem + a_col + kk * 8,
+        for (int kk = 0; kk < 8; ++kk)   // packed queries 0..63 at a_col, 64..127 at a_col + 64
+          mma_f16_ts(tmem + dcol, tmem + a_col + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8),
                      smem_desc_sw128(b_addr + kk * 2048, C::kPanelBytes, 1024), kIdescTS,
                      (acc || kk > 0) ? 1u : 0u);
       };
@@ -275,23 +283,24 @@ __global__ void __launch_bounds__(320, 1) bwd_main_kernel(const __grid_constant_
         const int s = idx % NS;
         if (!(ok = mbar_wait(bar(B_QF(s)), (idx / NS) & 1, ab, kSiteBMmaQ))) break;
         tc_fence_after();
-        gemm_kk(C::kColDP, vAddr, doAddr(s));                    // dP^T = V dO^T
-        tc_commit(bar(B_DP));
-        if (idx > 0) {
+        const uint32_t X = 128u * (idx & 1), Y = 128u - X;
+        gemm_kk(X, kAddr, qAddr(s));                             // S^T = K Q^T
+        tc_commit(bar(B_S));
+        if (idx > 0) {   // the dQ reduction of block idx-1 has drained region Y
           if (!(ok = mbar_wait(bar(B_DQFREE), (idx - 1) & 1, ab, kSiteBMmaFree))) break;
           tc_fence_after();
         }
-        gemm_kk(C::kColS, kAddr, qAddr(s));                      // S^T = K Q^T
-        tc_commit(bar(B_S));
+        gemm_kk(Y, vAddr, doAddr(s));                            // dP^T = V dO^T
+        tc_commit(bar(B_DP));
         if (!(ok = mbar_wait(bar(B_P), idx & 1, ab, kSiteBMmaP))) break;
         tc_fence_after();
-        gemm_ts(C::kColDV, C::kColS, doAddr(s), idx > 0);        // dV += P^T dO
+        gemm_ts(C::kColDV, X, doAddr(s), idx > 0);               // dV += P^T dO
         if (!(ok = mbar_wait(bar(B_DS), idx & 1, ab, kSiteBMmaDS))) break;
         tc_fence_after();
-        gemm_ts(C::kColDK, C::kColDP, qAddr(s), idx > 0);        // dK += dS^T Q
+        gemm_ts(C::kColDK, Y, qAddr(s), idx > 0);                // dK += dS^T Q
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)                           // dQ_i = dS K
-          mma_f16_ss(tmem + C::kColS, smem_desc_sw128(dsAddr + kk * 2048, C::kPanelBytes, 1024),
+        for (int kk = 0; kk < 8; ++kk)                           // dQ_i = dS K  -> X
+          mma_f16_ss(tmem + X, smem_desc_sw128(dsAddr + kk * 2048, C::kPanelBytes, 1024),
                      smem_desc_sw128(kAddr + kk * 2048, C::kPanelBytes, 1024), kIdescQ,
                      kk > 0 ? 1u : 0u);
         tc_commit(bar(B_DQ));
@@ -304,44 +313,50 @@ __global__ void __launch_bounds__(320, 1) bwd_main_kernel(const __grid_constant_
       mbar_wait(bar(B_DRAIN), 0, drain, kSiteBDrain);
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ P, dS (thread = key row)
-    const int r = threadIdx.x;
+    // Two warpgroups split the 128 query columns: wg 0 takes queries 0..63,
+    // wg 1 queries 64..127.  Each writes its packed P and dS over the first
+    // half of its own fp32 columns (cols 64 wg .. 64 wg + 31), so neither
+    // touches a column the other still reads.
+    const int wg = warp >> 2;
+    const int r = threadIdx.x & 127;
     const int key = j * 128 + r;
     const bool key_ok = key < p.N;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tmem + C::kColS + lane_off;
-    const uint32_t tDP = tmem + C::kColDP + lane_off;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t col_half = 64u * wg;
     const float cs = p.scale_log2;
     bool ok = true;
     for (int idx = 0; idx < n_i && ok; ++idx) {
       const int i = i0 + idx;
       const int s = idx % NS;
-      const float* L2s = reinterpret_cast<const float*>(smem + C::kOffLD + s * 1024);
-      const float* Ds = L2s + 128;
+      const float4* L4 = reinterpret_cast<const float4*>(smem + C::kOffLD + s * 1024) + 16 * wg;
+      const float4* D4 = L4 + 32;
       const bool diag = CAUSAL && i == j;
+      const uint32_t tS = tmem + 128u * (idx & 1) + lane_off + col_half;           // region X
+      const uint32_t tDP = tmem + 128u - 128u * (idx & 1) + lane_off + col_half;   // region Y
       if (!(ok = mbar_wait_warp(bar(B_S), idx & 1, ab, kSiteBSmS))) break;
       tc_fence_after();
       {
-        uint32_t u[128];
-        tmem_ld128(tS, u);
+        uint32_t u[64];
+        tmem_ld64(tS, u);
 #pragma unroll
-        for (int c4 = 0; c4 < 32; ++c4) {
-          const float4 l4 = reinterpret_cast<const float4*>(L2s)[c4];
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 l4 = L4[c4];
           const float lq[4] = {l4.x, l4.y, l4.z, l4.w};
           float pv[4];
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
-            const int c = 4 * c4 + t;
+            const int c = 4 * c4 + t;                    // query 64 wg + c
             float x = fmaf(__uint_as_float(u[c]), cs, -lq[t]);
-            if (diag && r > c) x = -INFINITY;     // key after query
+            if (diag && r > static_cast<int>(col_half) + c) x = -INFINITY;   // key after query
             pv[t] = ex2_sfu(x);
           }
           if (!key_ok) pv[0] = pv[1] = pv[2] = pv[3] = 0.f;
           u[2 * c4] = pack_bf16x2(pv[0], pv[1]);
           u[2 * c4 + 1] = pack_bf16x2(pv[2], pv[3]);
         }
-        tmem_st64(tS, *reinterpret_cast<uint32_t(*)[64]>(&u[0]));
+        tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
       }
       tmem_st_wait();
       tc_fence_before();
@@ -349,22 +364,25 @@ __global__ void __launch_bounds__(320, 1) bwd_main_kernel(const __grid_constant_
       if (!(ok = mbar_wait_warp(bar(B_DP), idx & 1, ab, kSiteBSmDP))) break;
       if (idx > 0 && !(ok = mbar_wait_warp(bar(B_DQ), (idx - 1) & 1, ab, kSiteBSmDQ))) break;
       tc_fence_after();
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {                 // queries 64h .. 64h+63
+      {
         uint32_t dp[64], pp[32], ds[32];
-        tmem_ld32(tDP + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-        tmem_ld32(tDP + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
-        tmem_ld32(tS + 32 * h, pp);
+        tmem_ld64(tDP, dp);
+        tmem_ld32(tS, pp);
 #pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2) {
-          const int c = 64 * h + 2 * c2;
-          const float p0 = __uint_as_float(pp[c2] << 16), p1 = __uint_as_float(pp[c2] & 0xFFFF0000u);
-          const float d0 = p0 * (__uint_as_float(dp[2 * c2]) - Ds[c]);
-          const float d1 = p1 * (__uint_as_float(dp[2 * c2 + 1]) - Ds[c + 1]);
-          ds[c2] = pack_bf16x2(d0, d1);
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 d4 = D4[c4];
+          const float dq[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+          for (int t2 = 0; t2 < 2; ++t2) {
+            const int c2 = 2 * c4 + t2;                  // packed pair index
+            const float p0 = __uint_as_float(pp[c2] << 16), p1 = __uint_as_float(pp[c2] & 0xFFFF0000u);
+            const float d0 = p0 * (__uint_as_float(dp[2 * c2]) - dq[2 * t2]);
+            const float d1 = p1 * (__uint_as_float(dp[2 * c2 + 1]) - dq[2 * t2 + 1]);
+            ds[c2] = pack_bf16x2(d0, d1);
+          }
         }
-        tmem_st32(tDP + 32 * h, ds);
-        const uint32_t row = dsAddr + h * C::kPanelBytes + r * 128;
+        tmem_st32(tDP, ds);
+        const uint32_t row = dsAddr + wg * C::kPanelBytes + r * 128;
 #pragma unroll
         for (int q = 0; q < 8; ++q)
           st_shared_v4b(row + ((q ^ (r & 7)) << 4), ds[4 * q], ds[4 * q + 1], ds[4 * q + 2], ds[4 * q + 3]);
@@ -375,10 +393,11 @@ __global__ void __launch_bounds__(320, 1) bwd_main_kernel(const __grid_constant_
       mbar_arrive(bar(B_DS));
     }
     if (ok) ok = mbar_wait_warp(bar(B_FINAL), 0, ab, kSiteBEpi);
-    ok = named_bar_and(1, 128, ok);
+    ok = named_bar_and(1, 256, ok);
     if (ok) {
       // Every lane takes part in the warp-collective TMEM loads; only the
-      // global stores depend on the key being inside the sequence.
+      // global stores depend on the key being inside the sequence.  wg 0
+      // writes head-dim columns [0, d/2), wg 1 [d/2, d).
       tc_fence_after();
       const size_t g = (static_cast<size_t>(bh) * p.N + (key_ok ? key : 0)) * D;
 #pragma unroll
@@ -387,7 +406,8 @@ __global__ void __launch_bounds__(320, 1) bwd_main_kernel(const __grid_constant_
         uint16_t* dst = (which ? p.dk : p.dv) + g;
         const float mul = which ? p.scale : 1.f;
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
+        for (int cc = 0; cc < D / 64; ++cc) {
+          const int ch = wg * (D / 64) + cc;
           uint32_t u[32];
           tmem_ld32(src + 32 * ch, u);
           uint32_t pk[16];
@@ -402,9 +422,9 @@ __global__ void __launch_bounds__(320, 1) bwd_main_kernel(const __grid_constant_
         }
       }
     }
-  } else {
+  } else if (warp < 12) {
     // ------------------------------------------------------------ dQ reduction (thread = query row)
-    const int r = threadIdx.x - 128;
+    const int r = threadIdx.x - 256;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     bool ok = true;
     for (int idx = 0; idx < n_i && ok; ++idx) {
@@ -415,7 +435,7 @@ __global__ void __launch_bounds__(320, 1) bwd_main_kernel(const __grid_constant_
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t u[32];
-        tmem_ld32(tmem + C::kColS + lane_off + 32 * ch, u);
+        tmem_ld32(tmem + 128u * (idx & 1) + lane_off + 32 * ch, u);
         if (row < p.N) {
 #pragma unroll
           for (int q = 0; q < 8; ++q)
@@ -430,7 +450,7 @@ __global__ void __launch_bounds__(320, 1) bwd_main_kernel(const __grid_constant_
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }

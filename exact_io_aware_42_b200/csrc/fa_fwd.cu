@@ -114,8 +114,11 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x % p.BH;
-  const int pair = p.n_pairs - 1 - blockIdx.x / p.BH;   // heaviest causal pairs first
+  // Causal: the heaviest pairs of every head first (longest-first balances
+  // the uneven work).  Non-causal: head-major, so the resident CTAs cover a
+  // few heads whose K and V stay in L2.  Both orders measured on B200.
+  const int bh = CAUSAL ? blockIdx.x % p.BH : blockIdx.x / p.n_pairs;
+  const int pair = CAUSAL ? p.n_pairs - 1 - blockIdx.x / p.BH : blockIdx.x % p.n_pairs;
   const int qt0 = 2 * pair;
   int n_t[2];
 #pragma unroll
