@@ -89,6 +89,17 @@ int poly_pairs(int d) {
   return d == 64 ? kDefaultPolyPairsD64 : kDefaultPolyPairsD128;
 }
 
+// Backward P-phase exp2 share on the FMA pipe (groups of 4); FA_BWD_POLY
+// overrides the default for measurement (0, 1 or 2).
+int bwd_poly_groups() {
+  static int v = [] {
+    const char* e = std::getenv("FA_BWD_POLY");
+    const int x = e ? std::atoi(e) : -1;
+    return (x == 0 || x == 1 || x == 2) ? x : kDefaultBwdPolyGroups;
+  }();
+  return v;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // 3-D view [BH, N, d] of a contiguous [B, H, N, d] tensor, 128-byte swizzle,
@@ -192,7 +203,8 @@ extern "C" fa_status fa_bwd(const void* q, const void* k, const void* v, const v
   std::memset(&p, 0, sizeof(p));
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   if (!encode_3d(&p.tm_q, q, bf, 2, d, N, BH, 64, 128) || !encode_3d(&p.tm_k, k, bf, 2, d, N, BH, 64, 128) ||
-      !encode_3d(&p.tm_v, v, bf, 2, d, N, BH, 64, 128) || !encode_3d(&p.tm_do, dout, bf, 2, d, N, BH, 64, 128))
+      !encode_3d(&p.tm_v, v, bf, 2, d, N, BH, 64, 128) || !encode_3d(&p.tm_do, dout, bf, 2, d, N, BH, 64, 128) ||
+      !encode_3d(&p.tm_dqacc, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, N, BH, 32, 128))
     return FA_ERR_INVALID_ARG;
   p.lse = lse;
   p.delta = delta;
@@ -206,6 +218,7 @@ extern "C" fa_status fa_bwd(const void* q, const void* k, const void* v, const v
   p.n_q = (N + 127) / 128;
   p.scale = scale;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.poly_groups = bwd_poly_groups();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = launch_bwd_preprocess(static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout),
                                         delta, dq_acc, rows, d, s);
@@ -231,8 +244,23 @@ extern "C" fa_status fa_quant_fp8(const void* x, void* x8, float* scales, int B,
   DeviceInfo* di = nullptr;
   fa_status st = current_device(&di);
   if (st != FA_OK) return st;
-  cudaError_t e = launch_quant_fp8(static_cast<const uint16_t*>(x), static_cast<uint8_t*>(x8), scales,
-                                   signs, B * H, N, d, static_cast<cudaStream_t>(stream));
+  cudaError_t e;
+  if (d == 128) {
+    QuantParams qp;
+    std::memset(&qp, 0, sizeof(qp));
+    if (!encode_3d(&qp.tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, B * H, 64, 128) ||
+        !encode_3d(&qp.tm_x8, x8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, B * H, 128, 128))
+      return FA_ERR_INVALID_ARG;
+    qp.scales = scales;
+    qp.signs = signs;
+    qp.status = di->status;
+    qp.N = N;
+    qp.nblk = (N + 127) / 128;
+    e = launch_quant_fp8_tma(qp, B * H, static_cast<cudaStream_t>(stream));
+  } else {
+    e = launch_quant_fp8(static_cast<const uint16_t*>(x), static_cast<uint8_t*>(x8), scales, signs,
+                         B * H, N, d, static_cast<cudaStream_t>(stream));
+  }
   if (e != cudaSuccess) {
     cudaGetLastError();
     return FA_ERR_LAUNCH;

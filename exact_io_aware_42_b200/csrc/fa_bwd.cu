@@ -22,18 +22,19 @@
 //                               into shared memory (MN-major, 128-B swizzle)
 //   dK  += dS^T Q_i             tcgen05 TS
 //   dQ_i = dS K_j               tcgen05 SS (A = dS, MN-major) -> TMEM [0,d)
-//   dQ accumulator += dQ_i      dQ warps: TMEM -> red.global.add.v4.f32
+//   dQ accumulator += dQ_i      dQ warps: TMEM -> shared -> TMA bulk reduce-add
 // dV and dK accumulate in TMEM [256,256+d) and [256+d,256+2d) over all i and
 // are written once at the end.  dQ accumulation: every key block adds its
-// share of a query block's dQ into one fp32 buffer with vector reductions in
-// L2 (the summation order across key blocks is not fixed, so dQ may differ in
-// the last bits from run to run; dK and dV are deterministic).
+// share of a query block's dQ into one fp32 buffer with TMA bulk reductions
+// in L2 (the summation order across key blocks is not fixed, so dQ may differ
+// in the last bits from run to run; dK and dV are deterministic).
 //
 // Roles: warps 0-7 P / dS and the dK, dV epilogue (thread = key row; warps
 // 0-3 take queries 0..63 of each block, warps 4-7 queries 64..127); warps 8-11
 // dQ reduction (thread = query row); warp 12 TMA producer (also stages L and
 // D of each query block in shared memory); warp 13 TMEM owner and the single
 // MMA-issuing thread.  Every wait is bounded (fa_ptx.cuh).
+#include "fa_exp2.cuh"
 #include "fa_internal.h"
 #include "fa_ptx.cuh"
 
@@ -135,18 +136,14 @@ __device__ __forceinline__ void st_shared_v4b(uint32_t addr, uint32_t a, uint32_
                : "memory");
 }
 
-__device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c, float d) {
-  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a),
-               "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
-
 __device__ __forceinline__ void st_global_v4(void* dst, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
 }
 
-template <int D, bool CAUSAL>
+// NPOLY of every 4 groups of 4 query columns take the FMA-pipe exp2
+// (fa_exp2.cuh) in the P phase, the rest the SFU.
+template <int D, bool CAUSAL, int NPOLY>
 __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant__ BwdParams p) {
   using C = BwdCfg<D>;
   constexpr int NS = C::kStages;
@@ -345,14 +342,20 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
           const float4 l4 = L4[c4];
           const float lq[4] = {l4.x, l4.y, l4.z, l4.w};
           float pv[4];
+          const uint64_t x01 = f2_fma(f2_pack(__uint_as_float(u[4 * c4]), __uint_as_float(u[4 * c4 + 1])),
+                                      f2_pack(cs, cs), f2_pack(-lq[0], -lq[1]));
+          const uint64_t x23 = f2_fma(f2_pack(__uint_as_float(u[4 * c4 + 2]), __uint_as_float(u[4 * c4 + 3])),
+                                      f2_pack(cs, cs), f2_pack(-lq[2], -lq[3]));
+          const bool poly = (c4 & 3) < NPOLY;
+          const uint64_t p01 = poly ? exp2_poly_f2<3>(x01) : exp2_sfu_f2(x01);
+          const uint64_t p23 = poly ? exp2_poly_f2<3>(x23) : exp2_sfu_f2(x23);
+          f2_unpack(p01, pv[0], pv[1]);
+          f2_unpack(p23, pv[2], pv[3]);
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const int c = 4 * c4 + t;                    // query 64 wg + c
-            float x = fmaf(__uint_as_float(u[c]), cs, -lq[t]);
-            if (diag && r > static_cast<int>(col_half) + c) x = -INFINITY;   // key after query
-            pv[t] = ex2_sfu(x);
+          for (int t = 0; t < 4; ++t) {                  // query 64 wg + 4 c4 + t
+            const bool hidden = !key_ok || (diag && r > static_cast<int>(col_half) + 4 * c4 + t);
+            pv[t] = hidden ? 0.f : pv[t];                // key past N, or key after query
           }
-          if (!key_ok) pv[0] = pv[1] = pv[2] = pv[3] = 0.f;
           u[2 * c4] = pack_bf16x2(pv[0], pv[1]);
           u[2 * c4 + 1] = pack_bf16x2(pv[2], pv[3]);
         }
@@ -362,7 +365,9 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
       tc_fence_before();
       mbar_arrive(bar(B_P));
       if (!(ok = mbar_wait_warp(bar(B_DP), idx & 1, ab, kSiteBSmDP))) break;
-      if (idx > 0 && !(ok = mbar_wait_warp(bar(B_DQ), (idx - 1) & 1, ab, kSiteBSmDQ))) break;
+      // the dS buffer doubles as the dQ staging area: wait until the dQ
+      // reduction of the previous block has left it
+      if (idx > 0 && !(ok = mbar_wait_warp(bar(B_DQFREE), (idx - 1) & 1, ab, kSiteBSmDQ))) break;
       tc_fence_after();
       {
         uint32_t dp[64], pp[32], ds[32];
@@ -424,28 +429,46 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
     }
   } else if (warp < 12) {
     // ------------------------------------------------------------ dQ reduction (thread = query row)
+    // dQ_i leaves TMEM through the dS buffer (free once the dQ MMA has read
+    // it): two passes of 64 head-dim columns, each written as two 128-byte
+    // swizzled boxes of 32 fp32 columns and added into the fp32 accumulator
+    // by TMA bulk reductions (bulk L2 traffic instead of one reduction per
+    // 16 bytes from every thread).
     const int r = threadIdx.x - 256;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     bool ok = true;
     for (int idx = 0; idx < n_i && ok; ++idx) {
-      const int row = (i0 + idx) * 128 + r;
-      if (!(ok = mbar_wait_warp(bar(B_DQ), idx & 1, ab, kSiteBDq))) break;
+      const int i = i0 + idx;
+      ok = mbar_wait_warp(bar(B_DQ), idx & 1, ab, kSiteBDq);
+      // all four warps agree before any of them enters the named barriers below
+      if (!(ok = named_bar_and(2, 128, ok))) break;
       tc_fence_after();
-      float* dst = p.dq_acc + (static_cast<size_t>(bh) * p.N + row) * D;
 #pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t u[32];
-        tmem_ld32(tmem + 128u * (idx & 1) + lane_off + 32 * ch, u);
-        if (row < p.N) {
+      for (int h = 0; h < D / 64; ++h) {
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          uint32_t u[32];
+          tmem_ld32(tmem + 128u * (idx & 1) + lane_off + 64 * h + 32 * b, u);
+          const uint32_t row = dsAddr + b * 16384 + r * 128;
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            red_add_v4(dst + 32 * ch + 4 * q, __uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1]),
-                       __uint_as_float(u[4 * q + 2]), __uint_as_float(u[4 * q + 3]));
+            st_shared_v4b(row + ((q ^ (r & 7)) << 4), u[4 * q], u[4 * q + 1], u[4 * q + 2], u[4 * q + 3]);
         }
+        fence_proxy_async_smem();
+        named_bar_sync(2, 128);
+        if (r == 0) {
+#pragma unroll
+          for (int b = 0; b < 2; ++b)
+            tma_reduce_add_3d(&p.tm_dqacc, dsAddr + b * 16384, 64 * h + 32 * b, i * 128, bh);
+          tma_store_commit();
+          tma_store_wait_read_all();       // staging buffer may be rewritten
+        }
+        named_bar_sync(2, 128);
       }
       tc_fence_before();
       mbar_arrive(bar(B_DQFREE));
     }
+    if (r == 0) tma_store_wait_all();      // every reduction has landed
   }
 
   tc_fence_before();
@@ -456,10 +479,10 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, int NPOLY>
 cudaError_t launch_main_impl(const BwdParams& p, cudaStream_t stream) {
   using C = BwdCfg<D>;
-  auto kern = bwd_main_kernel<D, CAUSAL>;
+  auto kern = bwd_main_kernel<D, CAUSAL, NPOLY>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(p.n_kv) * static_cast<unsigned>(p.BH);
@@ -488,9 +511,18 @@ cudaError_t launch_bwd_preprocess(const uint16_t* o, const uint16_t* dout, float
   return cudaGetLastError();
 }
 
+template <int D, bool CAUSAL>
+cudaError_t launch_main_np(const BwdParams& p, cudaStream_t stream) {
+  switch (p.poly_groups) {
+    case 1: return launch_main_impl<D, CAUSAL, 1>(p, stream);
+    case 2: return launch_main_impl<D, CAUSAL, 2>(p, stream);
+    default: return launch_main_impl<D, CAUSAL, 0>(p, stream);
+  }
+}
+
 cudaError_t launch_bwd_main(const BwdParams& p, int d, bool causal, cudaStream_t stream) {
-  if (d == 64) return causal ? launch_main_impl<64, true>(p, stream) : launch_main_impl<64, false>(p, stream);
-  return causal ? launch_main_impl<128, true>(p, stream) : launch_main_impl<128, false>(p, stream);
+  if (d == 64) return causal ? launch_main_np<64, true>(p, stream) : launch_main_np<64, false>(p, stream);
+  return causal ? launch_main_np<128, true>(p, stream) : launch_main_np<128, false>(p, stream);
 }
 
 cudaError_t launch_bwd_postprocess(const float* dq_acc, uint16_t* dq, long long n, float scale,

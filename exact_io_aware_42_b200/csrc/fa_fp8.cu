@@ -8,7 +8,8 @@
 //   x <- x diag(s) H_d / sqrt(d)       (optional; H_d Sylvester, s given)
 //   scale = amax(|x| over the block) / 448   (1 if the block is all zero)
 //   code  = e4m3_rn_satfinite(fp32(x) / scale)
-// One CTA of 128 threads per block, thread = row.  The rotation is the fast
+// One CTA of 128 threads per block, thread = row (d = 128: the block moves
+// through shared memory by TMA both ways; d = 64: direct loads).  The rotation is the fast
 // Walsh-Hadamard transform (log2 d butterfly stages of a+b, a-b in fp32, in
 // registers) followed by one multiply by fp32(1/sqrt(d)); it equals H_d z in
 // exact arithmetic and differs from the fp64 product by a few fp32 ulps.
@@ -95,6 +96,109 @@ __global__ void __launch_bounds__(128) quant_fp8_kernel(const uint4* __restrict_
   }
 }
 
+// d = 128 with TMA: the block (128 rows x 256 B, two 128-byte swizzled
+// panels) arrives in shared memory by one bulk copy; thread r reads row r
+// chunk by chunk at the swizzled position (no bank conflicts); the codes go
+// back through a 16 KB swizzled tile and one TMA store.
+template <bool ROT>
+__global__ void __launch_bounds__(128) quant_fp8_tma_kernel(const __grid_constant__ QuantParams p) {
+  constexpr int D = 128;
+  // dynamic shared memory only (no static variables ahead of it): input
+  // tile 32 KB | code tile 16 KB | mbarrier | abort flag | 4 warp maxima
+  extern __shared__ __align__(1024) uint8_t qsm[];
+  const uint32_t sbase = smem_u32(qsm);
+  const uint32_t in = sbase, out = sbase + 2 * 16384, bar = sbase + 3 * 16384;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(qsm + 3 * 16384 + 8);
+  float* warp_max = reinterpret_cast<float*>(qsm + 3 * 16384 + 16);
+  const int bh = blockIdx.x / p.nblk;
+  const int blk = blockIdx.x % p.nblk;
+  const int r = threadIdx.x;
+  if (r == 0) {
+    *abort_flag = 0;
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (sbase & 1023u) {                  // swizzled tiles need a 1024-byte aligned base
+    if (r == 0) atomicCAS(p.status, 0u, FA_ERR_LAUNCH);
+    return;
+  }
+  if (r == 0) {
+    mbar_arrive_expect_tx(bar, 2 * 16384);
+    tma_load_3d(in, &p.tm_x, bar, 0, blk * 128, bh);
+    tma_load_3d(in + 16384, &p.tm_x, bar, 64, blk * 128, bh);
+  }
+  const Abort ab{abort_flag, p.status};
+  // Bounded wait; on failure the copy is still waited for (bounded) before exit.
+  const bool ok = __syncthreads_and(mbar_wait(bar, 0, ab, 32) ? 1 : 0) != 0;
+  if (!ok) {
+    volatile int never = 0;
+    const Abort drain{&never, p.status};
+    mbar_wait(bar, 0, drain, 33);
+    return;
+  }
+  float v[D];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {        // 16-byte chunk c of the row = elements 8c .. 8c+7
+    const uint32_t addr = in + (c / 8) * 16384 + r * 128 + (((c % 8) ^ (r & 7)) << 4);
+    uint32_t w0, w1, w2, w3;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3) : "r"(addr));
+    const uint32_t ww[4] = {w0, w1, w2, w3};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[8 * c + 2 * k] = __uint_as_float(ww[k] << 16);
+      v[8 * c + 2 * k + 1] = __uint_as_float(ww[k] & 0xFFFF0000u);
+    }
+  }
+  if constexpr (ROT) {
+#pragma unroll
+    for (int i = 0; i < D; ++i) v[i] *= p.signs[i];
+#pragma unroll
+    for (int st = 0; st < 7; ++st) {
+      const int h = 1 << st;
+#pragma unroll
+      for (int bf = 0; bf < D / 2; ++bf) {
+        const int lo = (bf >> st) * 2 * h + (bf & (h - 1));
+        const float a = v[lo], b = v[lo + h];
+        v[lo] = a + b;
+        v[lo + h] = a - b;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < D; ++i) v[i] *= 0.08838834764831845f;
+  }
+  float am = 0.f;
+#pragma unroll
+  for (int i = 0; i < D; ++i) am = fmaxf(am, fabsf(v[i]));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
+  if ((r & 31) == 0) warp_max[r >> 5] = am;
+  __syncthreads();
+  am = fmaxf(fmaxf(warp_max[0], warp_max[1]), fmaxf(warp_max[2], warp_max[3]));
+  const float scale = am > 0.f ? __fdiv_rn(am, 448.f) : 1.f;
+  if (r == 0) p.scales[static_cast<size_t>(bh) * p.nblk + blk] = scale;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {         // 16 codes per chunk
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = 16 * c + 4 * k;
+      w[k] = e4m3x4(__fdiv_rn(v[i], scale), __fdiv_rn(v[i + 1], scale), __fdiv_rn(v[i + 2], scale),
+                    __fdiv_rn(v[i + 3], scale));
+    }
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(out + r * 128 + ((c ^ (r & 7)) << 4)),
+                 "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+                 : "memory");
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (r == 0) {                          // rows past N are clipped by the store
+    tma_store_3d(&p.tm_x8, out, 0, blk * 128, bh);
+    tma_store_commit();
+    tma_store_wait_all();
+  }
+}
+
 template <int D, bool ROT>
 cudaError_t launch_q(const uint16_t* x, uint8_t* x8, float* scales, const float* signs, int BH, int N,
                      cudaStream_t stream) {
@@ -106,6 +210,21 @@ cudaError_t launch_q(const uint16_t* x, uint8_t* x8, float* scales, const float*
 }
 
 }  // namespace
+
+cudaError_t launch_quant_fp8_tma(const QuantParams& q, int BH, cudaStream_t stream) {
+  const unsigned grid = static_cast<unsigned>(BH) * static_cast<unsigned>(q.nblk);
+  const int smem = 3 * 16384 + 64;
+  if (q.signs) {
+    cudaError_t e = cudaFuncSetAttribute(quant_fp8_tma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    quant_fp8_tma_kernel<true><<<grid, 128, smem, stream>>>(q);
+  } else {
+    cudaError_t e = cudaFuncSetAttribute(quant_fp8_tma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    quant_fp8_tma_kernel<false><<<grid, 128, smem, stream>>>(q);
+  }
+  return cudaGetLastError();
+}
 
 cudaError_t launch_quant_fp8(const uint16_t* x, uint8_t* x8, float* scales, const float* signs,
                              int BH, int N, int d, cudaStream_t stream) {

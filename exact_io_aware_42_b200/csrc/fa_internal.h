@@ -43,14 +43,26 @@ cudaError_t launch_fwd_bf16(const FwdParams& p, int d, bool causal, cudaStream_t
 // E4M3 forward (d = 128): tm_q/tm_k/tm_v are uint8 maps, sq/sk/sv block scales.
 cudaError_t launch_fwd_fp8(const FwdParams& p, bool causal, cudaStream_t stream);
 // Block quantisation of one bf16 tensor to E4M3 (signs == nullptr: no rotation).
+struct QuantParams {
+  CUtensorMap tm_x;     // bf16 [BH, N, 128], box {64, 128, 1}, 128-byte swizzle
+  CUtensorMap tm_x8;    // e4m3 [BH, N, 128], box {128, 128, 1}, 128-byte swizzle
+  float* scales;        // [BH, nblk]
+  const float* signs;   // d values or nullptr
+  unsigned int* status;
+  int N;
+  int nblk;
+};
 cudaError_t launch_quant_fp8(const uint16_t* x, uint8_t* x8, float* scales, const float* signs,
                              int BH, int N, int d, cudaStream_t stream);
+// d = 128 variant staged through TMA (tensor maps in ``q``).
+cudaError_t launch_quant_fp8_tma(const QuantParams& q, int BH, cudaStream_t stream);
 
 struct BwdParams {
   CUtensorMap tm_q;     // bf16 [BH, N, d], box {64, 128, 1}
   CUtensorMap tm_k;
   CUtensorMap tm_v;
   CUtensorMap tm_do;
+  CUtensorMap tm_dqacc; // fp32 [BH, N, d] accumulator, box {32, 128, 1}, for TMA reduce-add
   const float* lse;     // [BH, N], natural log
   const float* delta;   // [BH, N], D = rowsum(dO o O)
   float* dq_acc;        // [BH, N, d] fp32, zeroed by the preprocess kernel
@@ -63,7 +75,10 @@ struct BwdParams {
   int n_q;              // ceil(N / 128): query blocks
   float scale_log2;     // scale * log2(e)
   float scale;
+  int poly_groups;      // of every 4 groups of 4 columns, how many use the FMA-pipe exp2
 };
+
+constexpr int kDefaultBwdPolyGroups = 0;
 
 // D = rowsum(dO o O) per row, and dq_acc <- 0.
 cudaError_t launch_bwd_preprocess(const uint16_t* o, const uint16_t* dout, float* delta,
