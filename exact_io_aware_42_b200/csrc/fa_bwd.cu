@@ -64,8 +64,6 @@ struct BwdCfg {
   // X = 128 * (idx & 1) holds S^T, then P^T (bf16), then dQ_i; region
   // Y = 128 - X holds dP^T, then dS^T (bf16).  S^T of the next block goes into
   // the previous Y, so it never waits for the dQ reduction of the last block.
-  static constexpr uint32_t kColS = 0;
-  static constexpr uint32_t kColDP = 128;
   static constexpr uint32_t kColDV = 256;
   static constexpr uint32_t kColDK = 256 + D;
 };
@@ -157,8 +155,10 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
   const int B_KV = 0;
   auto B_QF = [](int s) { return 1 + s; };
   auto B_QE = [](int s) { return 1 + NS + s; };
+  // B_DQFREE: dQ_i has left TMEM (its region may take the next dP^T);
+  // B_DQSMEM: the dS buffer, used to stage dQ_i, is free again.
   const int B_S = 1 + 2 * NS, B_DP = B_S + 1, B_P = B_S + 2, B_DS = B_S + 3, B_DQ = B_S + 4,
-            B_DQFREE = B_S + 5, B_FINAL = B_S + 6, B_DRAIN = B_S + 7;
+            B_DQFREE = B_S + 5, B_FINAL = B_S + 6, B_DRAIN = B_S + 7, B_DQSMEM = B_S + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -184,6 +184,7 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
     mbar_init(bar(B_DS), 256);
     mbar_init(bar(B_DQ), 1);
     mbar_init(bar(B_DQFREE), 128);
+    mbar_init(bar(B_DQSMEM), 128);
     mbar_init(bar(B_FINAL), 1);
     mbar_init(bar(B_DRAIN), 1);
     *abort_flag = 0;
@@ -367,7 +368,7 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
       if (!(ok = mbar_wait_warp(bar(B_DP), idx & 1, ab, kSiteBSmDP))) break;
       // the dS buffer doubles as the dQ staging area: wait until the dQ
       // reduction of the previous block has left it
-      if (idx > 0 && !(ok = mbar_wait_warp(bar(B_DQFREE), (idx - 1) & 1, ab, kSiteBSmDQ))) break;
+      if (idx > 0 && !(ok = mbar_wait_warp(bar(B_DQSMEM), (idx - 1) & 1, ab, kSiteBSmDQ))) break;
       tc_fence_after();
       {
         uint32_t dp[64], pp[32], ds[32];
@@ -429,11 +430,12 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
     }
   } else if (warp < 12) {
     // ------------------------------------------------------------ dQ reduction (thread = query row)
-    // dQ_i leaves TMEM through the dS buffer (free once the dQ MMA has read
-    // it): two passes of 64 head-dim columns, each written as two 128-byte
-    // swizzled boxes of 32 fp32 columns and added into the fp32 accumulator
-    // by TMA bulk reductions (bulk L2 traffic instead of one reduction per
-    // 16 bytes from every thread).
+    // dQ_i leaves TMEM at once: head-dim columns [0, 64) go to the dS buffer
+    // (free once the dQ MMA has read it) as two 128-byte swizzled boxes of 32
+    // fp32 columns, columns [64, d) into registers; then the TMEM region is
+    // released (the next dP^T may start), the staged half is added into the
+    // fp32 accumulator by TMA bulk reductions, the register half is staged and
+    // reduced the same way, and finally the dS buffer is released.
     const int r = threadIdx.x - 256;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     bool ok = true;
@@ -443,30 +445,53 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
       // all four warps agree before any of them enters the named barriers below
       if (!(ok = named_bar_and(2, 128, ok))) break;
       tc_fence_after();
+      const uint32_t src = tmem + 128u * (idx & 1) + lane_off;
 #pragma unroll
-      for (int h = 0; h < D / 64; ++h) {
+      for (int b = 0; b < 2; ++b) {
+        uint32_t u[32];
+        tmem_ld32(src + 32 * b, u);
+        const uint32_t srow = dsAddr + b * 16384 + r * 128;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          st_shared_v4b(srow + ((q ^ (r & 7)) << 4), u[4 * q], u[4 * q + 1], u[4 * q + 2], u[4 * q + 3]);
+      }
+      uint32_t hi[D > 64 ? D - 64 : 1];
+      if constexpr (D > 64) {
+        tmem_ld32(src + 64, *reinterpret_cast<uint32_t(*)[32]>(&hi[0]));
+        tmem_ld32(src + 96, *reinterpret_cast<uint32_t(*)[32]>(&hi[32]));
+      }
+      tc_fence_before();
+      mbar_arrive(bar(B_DQFREE));
+      fence_proxy_async_smem();
+      named_bar_sync(2, 128);
+      if (r == 0) {
+#pragma unroll
+        for (int b = 0; b < 2; ++b) tma_reduce_add_3d(&p.tm_dqacc, dsAddr + b * 16384, 32 * b, i * 128, bh);
+        tma_store_commit();
+      }
+      if constexpr (D > 64) {
+        if (r == 0) tma_store_wait_read_all();
+        named_bar_sync(2, 128);
 #pragma unroll
         for (int b = 0; b < 2; ++b) {
-          uint32_t u[32];
-          tmem_ld32(tmem + 128u * (idx & 1) + lane_off + 64 * h + 32 * b, u);
-          const uint32_t row = dsAddr + b * 16384 + r * 128;
+          const uint32_t srow = dsAddr + b * 16384 + r * 128;
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            st_shared_v4b(row + ((q ^ (r & 7)) << 4), u[4 * q], u[4 * q + 1], u[4 * q + 2], u[4 * q + 3]);
+            st_shared_v4b(srow + ((q ^ (r & 7)) << 4), hi[32 * b + 4 * q], hi[32 * b + 4 * q + 1],
+                          hi[32 * b + 4 * q + 2], hi[32 * b + 4 * q + 3]);
         }
         fence_proxy_async_smem();
         named_bar_sync(2, 128);
         if (r == 0) {
 #pragma unroll
           for (int b = 0; b < 2; ++b)
-            tma_reduce_add_3d(&p.tm_dqacc, dsAddr + b * 16384, 64 * h + 32 * b, i * 128, bh);
+            tma_reduce_add_3d(&p.tm_dqacc, dsAddr + b * 16384, 64 + 32 * b, i * 128, bh);
           tma_store_commit();
-          tma_store_wait_read_all();       // staging buffer may be rewritten
         }
-        named_bar_sync(2, 128);
       }
-      tc_fence_before();
-      mbar_arrive(bar(B_DQFREE));
+      if (r == 0) tma_store_wait_read_all();   // staging buffer may be rewritten
+      named_bar_sync(2, 128);
+      mbar_arrive(bar(B_DQSMEM));
     }
     if (r == 0) tma_store_wait_all();      // every reduction has landed
   }
