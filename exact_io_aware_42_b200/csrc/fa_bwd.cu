@@ -14,14 +14,14 @@
 //   postprocess dQ = bf16(scale * dQ accumulator) (memory-bound)
 //
 // Main kernel, per query block i (TMEM lanes are the CTA's 128 keys):
-//   S^T  = K_j Q_i^T            tcgen05 SS   -> TMEM [0,128)
-//   dP^T = V_j dO_i^T           tcgen05 SS   -> TMEM [128,256)
+//   S^T  = K_j Q_i^T            tcgen05 SS   -> TMEM [0,128)  (region A)
+//   dP^T = V_j dO_i^T           tcgen05 SS   -> TMEM [128,256) (region B)
 //   P^T  = 2^(S^T c - L log2 e) softmax warps, bf16 back into TMEM
 //   dV  += P^T dO_i             tcgen05 TS   (A = P^T from TMEM)
 //   dS^T = P^T o (dP^T - D)     softmax warps, bf16 into TMEM and
 //                               into shared memory (MN-major, 128-B swizzle)
 //   dK  += dS^T Q_i             tcgen05 TS
-//   dQ_i = dS K_j               tcgen05 SS (A = dS, MN-major) -> TMEM [0,d)
+//   dQ_i = dS K_j               tcgen05 SS (A = dS, MN-major) -> region B
 //   dQ accumulator += dQ_i      dQ warps: TMEM -> shared -> TMA bulk reduce-add
 // dV and dK accumulate in TMEM [256,256+d) and [256+d,256+2d) over all i and
 // are written once at the end.  dQ accumulation: every key block adds its
@@ -56,14 +56,15 @@ struct BwdCfg {
   static constexpr int kOffDS = kOffQ + kStages * 2 * kTileBytes;   // dS^T, 128 x 128 bf16
   static constexpr int kOffLD = kOffDS + 128 * 128 * 2;             // + s * 1024: L2[128], D[128]
   static constexpr int kOffBar = kOffLD + kStages * 1024;
-  static constexpr int kNumBars = 1 + 2 * kStages + 9;
+  static constexpr int kNumBars = 1 + 2 * kStages + 10;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
   static constexpr uint32_t kTmemCols = 512;
-  // Two 128-column regions alternate roles per query block idx: region
-  // X = 128 * (idx & 1) holds S^T, then P^T (bf16), then dQ_i; region
-  // Y = 128 - X holds dP^T, then dS^T (bf16).  S^T of the next block goes into
-  // the previous Y, so it never waits for the dQ reduction of the last block.
+  // TMEM: columns [0,128) hold S^T, then P^T (bf16); [128,256) hold dP^T,
+  // then dS^T (bf16), then dQ_i.  S^T of the next block is issued right after
+  // dK of this one, before dQ, so the next P phase overlaps dQ and its drain.
+  static constexpr uint32_t kColA = 0;
+  static constexpr uint32_t kColB = 128;
   static constexpr uint32_t kColDV = 256;
   static constexpr uint32_t kColDK = 256 + D;
 };
@@ -155,10 +156,12 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
   const int B_KV = 0;
   auto B_QF = [](int s) { return 1 + s; };
   auto B_QE = [](int s) { return 1 + NS + s; };
+  // B_DS: dS^T is in TMEM (for dK); B_DSSM: dS is in shared memory (for dQ);
   // B_DQFREE: dQ_i has left TMEM (its region may take the next dP^T);
   // B_DQSMEM: the dS buffer, used to stage dQ_i, is free again.
   const int B_S = 1 + 2 * NS, B_DP = B_S + 1, B_P = B_S + 2, B_DS = B_S + 3, B_DQ = B_S + 4,
-            B_DQFREE = B_S + 5, B_FINAL = B_S + 6, B_DRAIN = B_S + 7, B_DQSMEM = B_S + 8;
+            B_DQFREE = B_S + 5, B_FINAL = B_S + 6, B_DRAIN = B_S + 7, B_DQSMEM = B_S + 8,
+            B_DSSM = B_S + 9;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -182,6 +185,7 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
     mbar_init(bar(B_DP), 1);
     mbar_init(bar(B_P), 256);
     mbar_init(bar(B_DS), 256);
+    mbar_init(bar(B_DSSM), 256);
     mbar_init(bar(B_DQ), 1);
     mbar_init(bar(B_DQFREE), 128);
     mbar_init(bar(B_DQSMEM), 128);
@@ -277,28 +281,37 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
                      (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(bar(B_KV), 0, ab, kSiteBMmaKV);
+      if (ok && n_i > 0 && (ok = mbar_wait(bar(B_QF(0)), 0, ab, kSiteBMmaQ))) {
+        tc_fence_after();
+        gemm_kk(C::kColA, kAddr, qAddr(0));                      // S^T(0) = K Q^T
+        tc_commit(bar(B_S));
+      }
       for (int idx = 0; idx < n_i && ok; ++idx) {
         const int s = idx % NS;
-        if (!(ok = mbar_wait(bar(B_QF(s)), (idx / NS) & 1, ab, kSiteBMmaQ))) break;
-        tc_fence_after();
-        const uint32_t X = 128u * (idx & 1), Y = 128u - X;
-        gemm_kk(X, kAddr, qAddr(s));                             // S^T = K Q^T
-        tc_commit(bar(B_S));
-        if (idx > 0) {   // the dQ reduction of block idx-1 has drained region Y
+        if (idx > 0) {   // dQ of the previous block has left region B
           if (!(ok = mbar_wait(bar(B_DQFREE), (idx - 1) & 1, ab, kSiteBMmaFree))) break;
           tc_fence_after();
         }
-        gemm_kk(Y, vAddr, doAddr(s));                            // dP^T = V dO^T
+        gemm_kk(C::kColB, vAddr, doAddr(s));                     // dP^T = V dO^T
         tc_commit(bar(B_DP));
         if (!(ok = mbar_wait(bar(B_P), idx & 1, ab, kSiteBMmaP))) break;
         tc_fence_after();
-        gemm_ts(C::kColDV, X, doAddr(s), idx > 0);               // dV += P^T dO
+        gemm_ts(C::kColDV, C::kColA, doAddr(s), idx > 0);        // dV += P^T dO
         if (!(ok = mbar_wait(bar(B_DS), idx & 1, ab, kSiteBMmaDS))) break;
         tc_fence_after();
-        gemm_ts(C::kColDK, Y, qAddr(s), idx > 0);                // dK += dS^T Q
+        gemm_ts(C::kColDK, C::kColB, qAddr(s), idx > 0);         // dK += dS^T Q
+        if (idx + 1 < n_i) {                                     // S^T of the next block
+          const int s1 = (idx + 1) % NS;
+          if (!(ok = mbar_wait(bar(B_QF(s1)), ((idx + 1) / NS) & 1, ab, kSiteBMmaQ))) break;
+          tc_fence_after();
+          gemm_kk(C::kColA, kAddr, qAddr(s1));
+          tc_commit(bar(B_S));
+        }
+        if (!(ok = mbar_wait(bar(B_DSSM), idx & 1, ab, kSiteBMmaDS))) break;
+        tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)                           // dQ_i = dS K  -> X
-          mma_f16_ss(tmem + X, smem_desc_sw128(dsAddr + kk * 2048, C::kPanelBytes, 1024),
+        for (int kk = 0; kk < 8; ++kk)                           // dQ_i = dS K  -> region B
+          mma_f16_ss(tmem + C::kColB, smem_desc_sw128(dsAddr + kk * 2048, C::kPanelBytes, 1024),
                      smem_desc_sw128(kAddr + kk * 2048, C::kPanelBytes, 1024), kIdescQ,
                      kk > 0 ? 1u : 0u);
         tc_commit(bar(B_DQ));
@@ -331,8 +344,8 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
       const float4* L4 = reinterpret_cast<const float4*>(smem + C::kOffLD + s * 1024) + 16 * wg;
       const float4* D4 = L4 + 32;
       const bool diag = CAUSAL && i == j;
-      const uint32_t tS = tmem + 128u * (idx & 1) + lane_off + col_half;           // region X
-      const uint32_t tDP = tmem + 128u - 128u * (idx & 1) + lane_off + col_half;   // region Y
+      const uint32_t tS = tmem + C::kColA + lane_off + col_half;
+      const uint32_t tDP = tmem + C::kColB + lane_off + col_half;
       if (!(ok = mbar_wait_warp(bar(B_S), idx & 1, ab, kSiteBSmS))) break;
       tc_fence_after();
       {
@@ -366,12 +379,10 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
       tc_fence_before();
       mbar_arrive(bar(B_P));
       if (!(ok = mbar_wait_warp(bar(B_DP), idx & 1, ab, kSiteBSmDP))) break;
-      // the dS buffer doubles as the dQ staging area: wait until the dQ
-      // reduction of the previous block has left it
-      if (idx > 0 && !(ok = mbar_wait_warp(bar(B_DQSMEM), (idx - 1) & 1, ab, kSiteBSmDQ))) break;
       tc_fence_after();
+      uint32_t ds[32];
       {
-        uint32_t dp[64], pp[32], ds[32];
+        uint32_t dp[64], pp[32];
         tmem_ld64(tDP, dp);
         tmem_ld32(tS, pp);
 #pragma unroll
@@ -388,15 +399,21 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
           }
         }
         tmem_st32(tDP, ds);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(B_DS));
+      // the dS buffer doubles as the dQ staging area: wait until the dQ
+      // reduction of the previous block has left it
+      if (idx > 0 && !(ok = mbar_wait_warp(bar(B_DQSMEM), (idx - 1) & 1, ab, kSiteBSmDQ))) break;
+      {
         const uint32_t row = dsAddr + wg * C::kPanelBytes + r * 128;
 #pragma unroll
         for (int q = 0; q < 8; ++q)
           st_shared_v4b(row + ((q ^ (r & 7)) << 4), ds[4 * q], ds[4 * q + 1], ds[4 * q + 2], ds[4 * q + 3]);
       }
-      tmem_st_wait();
       fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar(B_DS));
+      mbar_arrive(bar(B_DSSM));
     }
     if (ok) ok = mbar_wait_warp(bar(B_FINAL), 0, ab, kSiteBEpi);
     ok = named_bar_and(1, 256, ok);
@@ -445,7 +462,7 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
       // all four warps agree before any of them enters the named barriers below
       if (!(ok = named_bar_and(2, 128, ok))) break;
       tc_fence_after();
-      const uint32_t src = tmem + 128u * (idx & 1) + lane_off;
+      const uint32_t src = tmem + C::kColB + lane_off;
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
         uint32_t u[32];
