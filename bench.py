@@ -38,8 +38,27 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-WORKLOAD = dict(name="attn_B4_H16_N4096_d128_causal", B=4, H=16, N=4096, d=128, causal=True,
-                seed=2)
+DEFAULT_WORKLOAD = "attn_B4_H16_N4096_d128_causal"
+
+
+def workloads():
+    """Every timed configuration: the default (the one the headline metric is
+    quoted on), the small and FP8 workloads and the sequence-length sweep,
+    each causal and non-causal."""
+    from exact_io_aware_42_b200 import inputs
+    out = {DEFAULT_WORKLOAD: dict(B=4, H=16, N=4096, d=128, causal=True, seed=2),
+           "attn_B4_H16_N4096_d128_noncausal": dict(B=4, H=16, N=4096, d=128, causal=False, seed=2)}
+    for w in (inputs.TINY, inputs.SMALL, inputs.FP8) + inputs.sweep():
+        for c in w.causal:
+            name = w.name.replace("attn_fwd_", "attn_").replace("attn_fp8_", "attn_fp8_") + \
+                ("_causal" if c else "_noncausal")
+            out[name] = dict(B=w.B, H=w.H, N=w.N, d=w.d, causal=c, seed=w.seed)
+    for name, w in out.items():
+        w["name"] = name
+    return out
+
+
+WORKLOAD = None   # set in main()
 
 
 def fwd_flops(B, H, N, d, causal):
@@ -179,8 +198,9 @@ def build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs):
                                                       sc8["v"], causal=causal, out=o8, lse=lse8)
 
     f = fwd_flops(B, H, N, d, causal)
-    stages = [("fwd_bf16", s_fwd, f, 1), ("bwd_bf16", s_bwd, 2.5 * f, 3),
-              ("quant_fp8", s_quant, 0.0, 3), ("fwd_fp8", s_fwd8, f, 1)]
+    stages = [("fwd_bf16", s_fwd, f, 1), ("bwd_bf16", s_bwd, 2.5 * f, 3)]
+    if d == 128:   # the FP8 forward exists for d = 128 only
+        stages += [("quant_fp8", s_quant, 0.0, 3), ("fwd_fp8", s_fwd8, f, 1)]
     return stages, state
 
 
@@ -204,6 +224,22 @@ def time_stages(torch, stages, steps, stream):
 
 
 _ORACLE_INPUTS = {}
+
+
+def reduce_max(x: float, dist, device, world: int) -> float:
+    """Max of a per-rank scalar over all ranks (the slowest rank's time)."""
+    if world == 1:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world: int, step_flops: float, ms_per_step: float) -> float:
+    """Weak scaling: every rank runs its own copy of the workload, so the job
+    processes world x step_flops per (max-over-ranks) step time."""
+    return world * step_flops / (ms_per_step * 1e-3) / 1e12
 
 
 def oracle_sample(budget_s: float, B, H, N, d, causal, with_bwd: bool):
@@ -280,8 +316,10 @@ def config_block():
     return {"workload": w["name"], "B": w["B"], "H": w["H"], "N": w["N"], "d": w["d"],
             "causal": w["causal"], "global_batch": w["B"], "seq_len": w["N"],
             "parallelism": "independent replicas per GPU (heads), no collective",
-            "l2": "inputs 4 x 64 MiB > 126 MB L2, no flush",
-            "step": "fwd_bf16 + bwd_bf16 + quant_fp8 (Q, K rotated; V) + fwd_fp8",
+            "l2": (f"inputs 4 x {w['B'] * w['H'] * w['N'] * w['d'] * 2 / 2**20:.0f} MiB > 126 MB L2, no flush"
+                   if 4 * w["B"] * w["H"] * w["N"] * w["d"] * 2 > 126e6 else
+                   "inputs smaller than L2: timed warm in L2 (latency-bound workload)"),
+            "step": "fwd_bf16 + bwd_bf16" + (" + quant_fp8 (Q, K rotated; V) + fwd_fp8" if w["d"] == 128 else ""),
             "fp8": "quantisation and forward in E4M3 (kind::f8f6f4), counted at forward FLOPs"}
 
 
@@ -317,11 +355,7 @@ def run_ours(args):
         torch.cuda.synchronize()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, dist, dev, world)
 
     for _ in range(args.warmup):
         for s in stages:
@@ -334,7 +368,7 @@ def run_ours(args):
     total_ms = max_over_ranks(total_ms)
     per_stage = [max_over_ranks(x) for x in per_stage]
     ms_step = total_ms / args.steps
-    value = world * step_flops / (ms_step * 1e-3) / 1e12
+    value = whole_job_tflops(world, step_flops, ms_step)
 
     # end to end through the public API, host buffers in and out
     pin = {n: t.pin_memory() for n, t in (("q", hq), ("k", hk), ("v", hv), ("do", hdo))}
@@ -384,11 +418,13 @@ def run_ours(args):
                         "nominal_2250": value / world / 2250.0},
         "stages": {s[0]: {"ms": per_stage[i], "tflops": s[2] / (per_stage[i] * 1e-3) / 1e12}
                    for i, s in enumerate(stages)},
-        "roofline": dict(roof("bwd_bf16", "bwd_main_kernel<128, causal> (+ pre/post kernels in the timed call)",
-                              bwd_bytes(B, H, N, d)), traffic=profiled_traffic("bwd")),
-        "roofline_fwd": dict(roof("fwd_bf16", "fwd_kernel<128, causal, bf16>", fwd_bytes(B, H, N, d)),
-                             traffic=profiled_traffic("fwd")),
-        "e2e": {"value": world * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+        "roofline": dict(roof("bwd_bf16", f"bwd_main_kernel<{d}, {'causal' if causal else 'non-causal'}> "
+                              "(+ pre/post kernels in the timed call)", bwd_bytes(B, H, N, d)),
+                         traffic=profiled_traffic("bwd") if w["name"] == DEFAULT_WORKLOAD else None),
+        "roofline_fwd": dict(roof("fwd_bf16", f"fwd_kernel<{d}, {'causal' if causal else 'non-causal'}, bf16>",
+                                  fwd_bytes(B, H, N, d)),
+                             traffic=profiled_traffic("fwd") if w["name"] == DEFAULT_WORKLOAD else None),
+        "e2e": {"value": whole_job_tflops(world, step_flops, e2e_ms), "unit": "TFLOPS",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
@@ -413,7 +449,11 @@ def main():
     ap.add_argument("--ref-seconds", type=float, default=12.0,
                     help="host-core seconds of oracle work per reference step / cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads()),
+                    help="configuration to time (default: the one the headline metric is quoted on)")
     args = ap.parse_args()
+    global WORKLOAD
+    WORKLOAD = workloads()[args.workload]
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

@@ -28,6 +28,7 @@ SIGNATURES = {
     "fa_quant_fp8": (c_int, [_P, _P, _P, c_int, c_int, c_int, c_int, _P, _P]),
     "fa_fwd_fp8": (c_int, [_P, _P, _P, _P, _P, _P, _P, _P, c_int, c_int, c_int, c_int, c_float,
                            c_int, _P]),
+    "fa_selftest_wait_timeout": (c_int, [_P]),
     "fa_get_status": (c_uint, []),
     "fa_clear_status": (None, []),
     "fa_status_string": (ctypes.c_char_p, [c_int]),

@@ -310,6 +310,17 @@ extern "C" fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, 
   return FA_OK;
 }
 
+extern "C" fa_status fa_selftest_wait_timeout(void* stream) {
+  DeviceInfo* di = nullptr;
+  fa_status st = current_device(&di);
+  if (st != FA_OK) return st;
+  if (launch_selftest_wait(di->status, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+  }
+  return FA_OK;
+}
+
 extern "C" unsigned int fa_get_status(void) {
   unsigned int v = 0;
   if (cudaMemcpyFromSymbol(&v, fa::g_status, sizeof(v)) != cudaSuccess) {

@@ -40,6 +40,8 @@ constexpr int kDefaultPolyPairsD128 = 0;
 constexpr int kDefaultPolyPairsD64 = 4;
 
 cudaError_t launch_fwd_bf16(const FwdParams& p, int d, bool causal, cudaStream_t stream);
+// One CTA waiting on an mbarrier nothing arrives on (failure-path self-test).
+cudaError_t launch_selftest_wait(unsigned int* status, cudaStream_t stream);
 // E4M3 forward (d = 128): tm_q/tm_k/tm_v are uint8 maps, sq/sk/sv block scales.
 cudaError_t launch_fwd_fp8(const FwdParams& p, bool causal, cudaStream_t stream);
 // Block quantisation of one bf16 tensor to E4M3 (signs == nullptr: no rotation).

@@ -76,14 +76,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Wait for the phase of ``bar`` with the given parity.  Returns false (after
 // recording the failure) if the wait outlasts kWaitTimeoutNs or another role
 // of the CTA has already failed.
+// A second, independent bound: the number of polls (each try_wait may
+// suspend the thread for a short, hardware-defined time).
+constexpr uint32_t kWaitMaxPolls = 1u << 24;
+
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const Abort& ab,
                                           unsigned int where) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  while (true) {
+  for (uint32_t polls = 0;; ++polls) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*ab.flag) return false;
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+    if (global_timer_ns() - t0 > kWaitTimeoutNs || polls >= kWaitMaxPolls) {
       record_failure(ab, FA_ERR_PIPELINE_TIMEOUT | (where << 8));
       return false;
     }

@@ -156,6 +156,15 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float
 unsigned int fa_get_status(void);
 void fa_clear_status(void);
 
+/*
+ * Self-test of the failure path (not part of the attention computation):
+ * launches one CTA whose pipeline wait can never complete.  After the bounded
+ * wait (~2 s) it records FA_ERR_PIPELINE_TIMEOUT (site 0x7F) in the status
+ * word and returns; nothing is faulted or trapped and the context stays
+ * usable.  Synchronise, then read fa_get_status() and fa_clear_status().
+ */
+fa_status fa_selftest_wait_timeout(void* stream);
+
 /* Static, human-readable name of a status code. */
 const char* fa_status_string(int status);
 

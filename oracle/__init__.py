@@ -23,6 +23,7 @@ Modules:
 """
 from .attention_ref import (  # noqa: F401
     attn_fwd_ref,
+    attn_fwd_rows_ref,
     attn_bwd_ref,
     online_softmax_ref,
     attn_fwd_online_ref,

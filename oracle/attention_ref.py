@@ -113,6 +113,27 @@ def attn_fwd_ref(q, k, v, scale: float, causal: bool):
     return o, lse
 
 
+def attn_fwd_rows_ref(q, k, v, scale: float, causal: bool, rows):
+    """The forward definition for selected query rows of one head.
+
+    q, k, v: [N, d] (one head); ``rows``: query indices.  Row i sees keys
+    j <= i when causal.  Returns (O [len(rows), d], L [len(rows)]), fp64.
+    Used where a whole head is too large to materialise (N up to 16K).
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    rows = np.asarray(rows, dtype=np.int64)
+    o = np.zeros((rows.size, v.shape[1]))
+    lse = np.zeros(rows.size)
+    for n, i in enumerate(rows):
+        kk, vv = (k[: i + 1], v[: i + 1]) if causal else (k, v)
+        srow = float(scale) * (kk @ q[i])
+        m = np.max(srow)
+        e = np.exp(srow - m)
+        o[n] = (e / e.sum()) @ vv
+        lse[n] = m + np.log(e.sum())
+    return o, lse
+
+
 class BwdResult(NamedTuple):
     dq: np.ndarray
     dk: np.ndarray

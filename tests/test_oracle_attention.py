@@ -328,3 +328,16 @@ def test_planted_mistakes(kind):
         except AssertionError:
             caught.append(pin.__name__)
     assert caught, f"planted mistake {kind!r} passed every pin"
+
+
+def test_rows_oracle_matches_full_definition():
+    rng = np.random.default_rng(8)
+    q, k, v = (rng.standard_normal((1, 1, 50, 8)) for _ in range(3))
+    rows = [0, 1, 17, 49]
+    for causal in (False, True):
+        o, lse = oracle.attn_fwd_ref(q, k, v, 0.6, causal)
+        o_r, l_r = oracle.attn_fwd_rows_ref(q[0, 0], k[0, 0], v[0, 0], 0.6, causal, rows)
+        np.testing.assert_allclose(o_r, o[0, 0, rows], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(l_r, lse[0, 0, rows], rtol=1e-12, atol=1e-13)
+        ob = [brute_fwd(q[0, 0].tolist(), k[0, 0].tolist(), v[0, 0].tolist(), 0.6, causal)]
+        np.testing.assert_allclose(o_r, ob[0][0][rows], rtol=1e-12, atol=1e-12)
