@@ -525,7 +525,7 @@ template <int D, bool CAUSAL, int NPOLY>
 cudaError_t launch_main_impl(const BwdParams& p, cudaStream_t stream) {
   using C = BwdCfg<D>;
   auto kern = bwd_main_kernel<D, CAUSAL, NPOLY>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  cudaError_t e = set_smem_once<bwd_main_kernel<D, CAUSAL, NPOLY>>(C::kSmemBytes);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(p.n_kv) * static_cast<unsigned>(p.BH);
   kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(p);

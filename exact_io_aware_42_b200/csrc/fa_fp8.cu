@@ -27,6 +27,20 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
+// x / s rounded to nearest, by Markstein's correction step (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990): with y = RN(1/s),
+// q0 = RN(x y), r = x - q0 s (exact by FMA), q = RN(q0 + r y).  This gives
+// the correctly rounded quotient for normal operands and results; the only
+// quotients here outside that range are below 2^-126 in magnitude, which
+// round to E4M3 zero either way.  Checked bit for bit against IEEE division
+// by the quantisation tests.
+__device__ __forceinline__ float div_rn(float x, float s, float y) {
+  const float q0 = x * y;
+  const float r = fmaf(-q0, s, x);
+  return fmaf(r, y, q0);
+}
+
 template <int D, bool ROT>
 __global__ void __launch_bounds__(128) quant_fp8_kernel(const uint4* __restrict__ x,
                                                         uint4* __restrict__ x8,
@@ -80,6 +94,7 @@ __global__ void __launch_bounds__(128) quant_fp8_kernel(const uint4* __restrict_
   __syncthreads();
   am = fmaxf(fmaxf(warp_max[0], warp_max[1]), fmaxf(warp_max[2], warp_max[3]));
   const float scale = am > 0.f ? __fdiv_rn(am, 448.f) : 1.f;
+  const float inv = __frcp_rn(scale);
   if (r == 0) scales[static_cast<size_t>(bh) * nblk + blk] = scale;
   if (valid) {
 #pragma unroll
@@ -88,8 +103,8 @@ __global__ void __launch_bounds__(128) quant_fp8_kernel(const uint4* __restrict_
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int i = 16 * c16 + 4 * k;
-        w[k] = e4m3x4(__fdiv_rn(v[i], scale), __fdiv_rn(v[i + 1], scale), __fdiv_rn(v[i + 2], scale),
-                      __fdiv_rn(v[i + 3], scale));
+        w[k] = e4m3x4(div_rn(v[i], scale, inv), div_rn(v[i + 1], scale, inv), div_rn(v[i + 2], scale, inv),
+                      div_rn(v[i + 3], scale, inv));
       }
       x8[row_off * (D / 16) + c16] = make_uint4(w[0], w[1], w[2], w[3]);
     }
@@ -176,6 +191,7 @@ __global__ void __launch_bounds__(128) quant_fp8_tma_kernel(const __grid_constan
   __syncthreads();
   am = fmaxf(fmaxf(warp_max[0], warp_max[1]), fmaxf(warp_max[2], warp_max[3]));
   const float scale = am > 0.f ? __fdiv_rn(am, 448.f) : 1.f;
+  const float inv = __frcp_rn(scale);
   if (r == 0) p.scales[static_cast<size_t>(bh) * p.nblk + blk] = scale;
 #pragma unroll
   for (int c = 0; c < 8; ++c) {         // 16 codes per chunk
@@ -183,8 +199,8 @@ __global__ void __launch_bounds__(128) quant_fp8_tma_kernel(const __grid_constan
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int i = 16 * c + 4 * k;
-      w[k] = e4m3x4(__fdiv_rn(v[i], scale), __fdiv_rn(v[i + 1], scale), __fdiv_rn(v[i + 2], scale),
-                    __fdiv_rn(v[i + 3], scale));
+      w[k] = e4m3x4(div_rn(v[i], scale, inv), div_rn(v[i + 1], scale, inv), div_rn(v[i + 2], scale, inv),
+                    div_rn(v[i + 3], scale, inv));
     }
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(out + r * 128 + ((c ^ (r & 7)) << 4)),
                  "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
@@ -215,11 +231,11 @@ cudaError_t launch_quant_fp8_tma(const QuantParams& q, int BH, cudaStream_t stre
   const unsigned grid = static_cast<unsigned>(BH) * static_cast<unsigned>(q.nblk);
   const int smem = 3 * 16384 + 64;
   if (q.signs) {
-    cudaError_t e = cudaFuncSetAttribute(quant_fp8_tma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = set_smem_once<quant_fp8_tma_kernel<true>>(smem);
     if (e != cudaSuccess) return e;
     quant_fp8_tma_kernel<true><<<grid, 128, smem, stream>>>(q);
   } else {
-    cudaError_t e = cudaFuncSetAttribute(quant_fp8_tma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = set_smem_once<quant_fp8_tma_kernel<false>>(smem);
     if (e != cudaSuccess) return e;
     quant_fp8_tma_kernel<false><<<grid, 128, smem, stream>>>(q);
   }

@@ -61,7 +61,7 @@ struct FwdCfg {
   static constexpr int kOffBar = kOffRing + kStages * kTileBytes;
   static constexpr int kNumBars = 2 + 2 * kStages + 7;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // + base alignment slack
+  static constexpr int kSmemBytes = kOffMisc + 48 + 1024;   // + base alignment slack
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS = 0;       // + 128 * t
   static constexpr uint32_t kColO = 256;     // + D * t
@@ -290,10 +290,21 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
     const size_t sc_base = static_cast<size_t>(bh) * p.n_kv;
     float c_q = p.scale_log2;
     float v_max = 1.f;
+    float sk_next = 1.f, sv_next = 1.f;
     if constexpr (FP8) {
       c_q *= (qi < p.n_kv) ? p.sq[sc_base + qi] : 1.f;
-      v_max = 0.f;
-      for (int jj = 0; jj < p.n_kv; ++jj) v_max = fmaxf(v_max, p.sv[sc_base + jj]);
+      // max over this head's V block scales: strided over the warpgroup's
+      // 128 threads, then a shuffle and a shared-memory reduction
+      float vm = 0.f;
+      for (int jj = r; jj < p.n_kv; jj += 128) vm = fmaxf(vm, p.sv[sc_base + jj]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, off));
+      float* red = reinterpret_cast<float*>(smem + C::kOffMisc + 8) + 4 * t;   // 4 floats per tile
+      if (lane == 0) red[warp & 3] = vm;
+      named_bar_sync(1 + t, 128);
+      v_max = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+      sk_next = p.sk[sc_base];
+      sv_next = p.sv[sc_base];
     }
     constexpr float kTau = FP8 ? 0.f : kRescaleTau;
     float m_use = -INFINITY;
@@ -304,7 +315,14 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
       tc_fence_after();
       uint32_t u[128];
       tmem_ld128(tS, u);
-      const float c = FP8 ? c_q * p.sk[sc_base + j] : c_q;
+      const float c = c_q * sk_next;   // FP8: dequantise with s_q(i) s_k(j); bf16: sk_next = 1
+      const float sv_j = sv_next;
+      if constexpr (FP8) {             // next tile's scales, loaded while this one is processed
+        if (j + 1 < n) {
+          sk_next = p.sk[sc_base + j + 1];
+          sv_next = p.sv[sc_base + j + 1];
+        }
+      }
       const bool masked = (CAUSAL && j == qi) || ((j + 1) * kBlockN > p.N);
       if (masked) {
         // scaled scores with -inf where the key is hidden or past N
@@ -340,7 +358,7 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
       const float neg_m = -m_use;
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
       if constexpr (FP8) {
-        const float f8 = 256.f * p.sv[sc_base + j] / v_max;
+        const float f8 = 256.f * sv_j / v_max;
         const uint64_t c2 = f2_pack(c, c);
         const uint64_t nm2 = f2_pack(neg_m, neg_m);
         float keep0 = 0.f, keep1 = 0.f;
@@ -462,7 +480,7 @@ template <int D, bool CAUSAL, int NPOLY, bool FP8>
 cudaError_t launch_impl(const FwdParams& p, cudaStream_t stream) {
   using C = FwdCfg<D, FP8>;
   auto kern = fwd_kernel<D, CAUSAL, NPOLY, 3, FP8>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  cudaError_t e = set_smem_once<fwd_kernel<D, CAUSAL, NPOLY, 3, FP8>>(C::kSmemBytes);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(p.n_pairs) * static_cast<unsigned>(p.BH);
   kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(p);

@@ -8,6 +8,20 @@
 
 namespace fa {
 
+// Raise a kernel's dynamic shared-memory limit once per device and kernel
+// (the template parameter is the kernel itself, so every instantiation has
+// its own flags).
+template <auto Kernel>
+cudaError_t set_smem_once(int bytes) {
+  static bool done[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (done[dev]) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done[dev] = true;
+  return e;
+}
+
 constexpr int kBlockM = 128;      // query rows per tile (one TMEM lane per row)
 constexpr int kBlockN = 128;      // keys per K/V tile
 constexpr float kRescaleTau = 8.0f;   // log2 units; see the forward kernel
