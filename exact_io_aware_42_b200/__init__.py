@@ -6,6 +6,7 @@ does not load the library; the first call does, and raises if it is missing.
 """
 from .api import (  # noqa: F401
     bwd,
+    bwd_noalloc,
     bwd_workspace_size,
     clear_status,
     fwd,

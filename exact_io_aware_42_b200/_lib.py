@@ -23,6 +23,9 @@ SIGNATURES = {
     "fa_bwd_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int]),
     "fa_bwd": (c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, c_int, c_int, c_int, c_int, c_float,
                        c_int, _P, c_size_t, _P]),
+    "fa_bwd_deterministic_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int]),
+    "fa_bwd_deterministic": (c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, c_int, c_int, c_int, c_int,
+                                     c_float, c_int, _P, c_size_t, _P]),
     "fa_bwd_noalloc": (c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, c_int, c_int, c_int, c_int,
                                c_float, c_int, _P]),
     "fa_quant_fp8": (c_int, [_P, _P, _P, c_int, c_int, c_int, c_int, _P, _P]),

@@ -4,7 +4,7 @@ torch provides device memory and the current CUDA stream; every step of the
 computation runs in the library's kernels.  Functions mirror include/fa.h:
 
 * ``fwd(q, k, v, causal, scale)``            -> (o, lse)
-* ``bwd(q, k, v, o, do, lse, causal, scale)`` -> (dq, dk, dv)
+* ``bwd(q, k, v, o, do, lse, causal, scale, deterministic=False)`` -> (dq, dk, dv)
 * ``quant_fp8(x, signs=None)``               -> (x8 as uint8, block scales)
 * ``fwd_fp8(q8, k8, v8, sq, sk, sv, causal, scale)`` -> (o, lse)
 """
@@ -17,7 +17,7 @@ import torch
 
 from ._lib import check, lib
 
-__all__ = ["fwd", "bwd", "bwd_workspace_size", "quant_fp8", "fwd_fp8", "get_status",
+__all__ = ["fwd", "bwd", "bwd_workspace_size", "bwd_noalloc", "quant_fp8", "fwd_fp8", "get_status",
            "clear_status", "n_blocks"]
 
 
@@ -61,13 +61,19 @@ def fwd(q, k, v, causal: bool = False, scale: Optional[float] = None, out=None, 
     return o, lse_t
 
 
-def bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
+def bwd_workspace_size(B: int, H: int, N: int, d: int, deterministic: bool = False) -> int:
+    if deterministic:
+        return int(lib().fa_bwd_deterministic_workspace_size(B, H, N, d))
     return int(lib().fa_bwd_workspace_size(B, H, N, d))
 
 
 def bwd(q, k, v, o, do, lse, causal: bool = False, scale: Optional[float] = None,
-        workspace: Optional[torch.Tensor] = None, dq=None, dk=None, dv=None):
-    """Attention backward (bf16).  Returns (dq, dk, dv)."""
+        workspace: Optional[torch.Tensor] = None, dq=None, dk=None, dv=None,
+        deterministic: bool = False):
+    """Attention backward (bf16).  Returns (dq, dk, dv).
+
+    ``deterministic=True`` calls fa_bwd_deterministic: bitwise reproducible
+    gradients (dQ by a separate query-block-major kernel)."""
     _check_bhnd("q", q, torch.bfloat16)
     B, H, N, d = q.shape
     for name, t in (("k", k), ("v", v), ("o", o), ("do", do)):
@@ -76,16 +82,17 @@ def bwd(q, k, v, o, do, lse, causal: bool = False, scale: Optional[float] = None
         raise ValueError("lse must be a contiguous fp32 [B, H, N] tensor")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    ws_bytes = bwd_workspace_size(B, H, N, d)
+    ws_bytes = bwd_workspace_size(B, H, N, d, deterministic)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    code = lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
-                        _ptr(dk), _ptr(dv), B, H, N, d, float(scale), int(bool(causal)),
-                        _ptr(workspace), workspace.numel(), _stream())
-    check("fa_bwd", code)
+    name = "fa_bwd_deterministic" if deterministic else "fa_bwd"
+    code = getattr(lib(), name)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
+                                _ptr(dk), _ptr(dv), B, H, N, d, float(scale), int(bool(causal)),
+                                _ptr(workspace), workspace.numel(), _stream())
+    check(name, code)
     return dq, dk, dv
 
 

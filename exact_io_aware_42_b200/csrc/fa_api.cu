@@ -177,10 +177,21 @@ extern "C" size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   return up(rows * d * sizeof(float)) + up(rows * sizeof(float));
 }
 
-extern "C" fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o,
-                            const void* dout, const float* lse, void* dq, void* dk, void* dv,
-                            int B, int H, int N, int d, float scale, int causal, void* workspace,
-                            size_t workspace_bytes, void* stream) {
+extern "C" size_t fa_bwd_deterministic_workspace_size(int B, int H, int N, int d) {
+  if (B < 0 || H < 0 || N < 0 || (d != 64 && d != 128)) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  return (rows * sizeof(float) + 255) & ~static_cast<size_t>(255);
+}
+
+namespace {
+
+// Both backward variants: shared argument checks and tensor maps; the
+// atomic one accumulates dQ in fp32 scratch by TMA reductions, the
+// deterministic one runs the main kernel without dQ and the dQ kernel.
+fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                     const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                     float scale, int causal, void* workspace, size_t workspace_bytes, void* stream,
+                     bool deterministic) {
   fa_status st = check_shape(B, H, N, d, scale);
   if (st != FA_OK) return st;
   if (static_cast<long long>(B) * H * N == 0) return FA_OK;
@@ -188,7 +199,8 @@ extern "C" fa_status fa_bwd(const void* q, const void* k, const void* v, const v
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))
     return FA_ERR_MISALIGNED;
-  const size_t need = fa_bwd_workspace_size(B, H, N, d);
+  const size_t need = deterministic ? fa_bwd_deterministic_workspace_size(B, H, N, d)
+                                    : fa_bwd_workspace_size(B, H, N, d);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return FA_ERR_WORKSPACE;
   DeviceInfo* di = nullptr;
@@ -196,14 +208,18 @@ extern "C" fa_status fa_bwd(const void* q, const void* k, const void* v, const v
 
   const int BH = B * H;
   const long long rows = static_cast<long long>(BH) * N;
-  float* dq_acc = static_cast<float*>(workspace);
-  float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                          ((static_cast<size_t>(rows) * d * 4 + 255) & ~static_cast<size_t>(255)));
+  float* dq_acc = deterministic ? nullptr : static_cast<float*>(workspace);
+  float* delta = deterministic
+                     ? static_cast<float*>(workspace)
+                     : reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                                ((static_cast<size_t>(rows) * d * 4 + 255) & ~static_cast<size_t>(255)));
   BwdParams p;
   std::memset(&p, 0, sizeof(p));
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   if (!encode_3d(&p.tm_q, q, bf, 2, d, N, BH, 64, 128) || !encode_3d(&p.tm_k, k, bf, 2, d, N, BH, 64, 128) ||
-      !encode_3d(&p.tm_v, v, bf, 2, d, N, BH, 64, 128) || !encode_3d(&p.tm_do, dout, bf, 2, d, N, BH, 64, 128) ||
+      !encode_3d(&p.tm_v, v, bf, 2, d, N, BH, 64, 128) || !encode_3d(&p.tm_do, dout, bf, 2, d, N, BH, 64, 128))
+    return FA_ERR_INVALID_ARG;
+  if (!deterministic &&
       !encode_3d(&p.tm_dqacc, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, N, BH, 32, 128))
     return FA_ERR_INVALID_ARG;
   p.lse = lse;
@@ -211,6 +227,7 @@ extern "C" fa_status fa_bwd(const void* q, const void* k, const void* v, const v
   p.dq_acc = dq_acc;
   p.dk = static_cast<uint16_t*>(dk);
   p.dv = static_cast<uint16_t*>(dv);
+  p.dq = static_cast<uint16_t*>(dq);
   p.status = di->status;
   p.N = N;
   p.BH = BH;
@@ -222,13 +239,37 @@ extern "C" fa_status fa_bwd(const void* q, const void* k, const void* v, const v
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = launch_bwd_preprocess(static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout),
                                         delta, dq_acc, rows, d, s);
-  if (e == cudaSuccess) e = launch_bwd_main(p, d, causal != 0, s);
-  if (e == cudaSuccess) e = launch_bwd_postprocess(dq_acc, static_cast<uint16_t*>(dq), rows * d, scale, s);
+  if (e == cudaSuccess) e = launch_bwd_main(p, d, causal != 0, !deterministic, s);
+  if (e == cudaSuccess) {
+    if (deterministic)
+      e = launch_bwd_dq(p, d, causal != 0, s);
+    else
+      e = launch_bwd_postprocess(dq_acc, static_cast<uint16_t*>(dq), rows * d, scale, s);
+  }
   if (e != cudaSuccess) {
     cudaGetLastError();
     return FA_ERR_LAUNCH;
   }
   return FA_OK;
+}
+
+}  // namespace
+
+extern "C" fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o,
+                            const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                            int B, int H, int N, int d, float scale, int causal, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace,
+                    workspace_bytes, stream, false);
+}
+
+extern "C" fa_status fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,
+                                          const void* dout, const float* lse, void* dq, void* dk,
+                                          void* dv, int B, int H, int N, int d, float scale,
+                                          int causal, void* workspace, size_t workspace_bytes,
+                                          void* stream) {
+  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace,
+                    workspace_bytes, stream, true);
 }
 
 extern "C" fa_status fa_quant_fp8(const void* x, void* x8, float* scales, int B, int H, int N,

@@ -109,6 +109,7 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const uint4* __rest
     for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (valid) {
       if (sub == 0) delta[row] = acc;
+      if (dq_acc == nullptr) continue;
       const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
       dq_acc[row * (D / 4) + 2 * sub] = z;
       dq_acc[row * (D / 4) + 2 * sub + 1] = z;
@@ -141,8 +142,11 @@ __device__ __forceinline__ void st_global_v4(void* dst, uint32_t a, uint32_t b, 
 }
 
 // NPOLY of every 4 groups of 4 query columns take the FMA-pipe exp2
-// (fa_exp2.cuh) in the P phase, the rest the SFU.
-template <int D, bool CAUSAL, int NPOLY>
+// (fa_exp2.cuh) in the P phase, the rest the SFU.  DQ = false builds the
+// kernel without its dQ product (dK and dV only; the deterministic dQ
+// kernel computes dQ): no dS staging in shared memory, no dQ warps' work,
+// and the MMA issuer waits on nothing of dQ.
+template <int D, bool CAUSAL, int NPOLY, bool DQ>
 __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant__ BwdParams p) {
   using C = BwdCfg<D>;
   constexpr int NS = C::kStages;
@@ -288,7 +292,7 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
       }
       for (int idx = 0; idx < n_i && ok; ++idx) {
         const int s = idx % NS;
-        if (idx > 0) {   // dQ of the previous block has left region B
+        if (DQ && idx > 0) {   // dQ of the previous block has left region B
           if (!(ok = mbar_wait(bar(B_DQFREE), (idx - 1) & 1, ab, kSiteBMmaFree))) break;
           tc_fence_after();
         }
@@ -307,14 +311,18 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
           gemm_kk(C::kColA, kAddr, qAddr(s1));
           tc_commit(bar(B_S));
         }
-        if (!(ok = mbar_wait(bar(B_DSSM), idx & 1, ab, kSiteBMmaDS))) break;
-        tc_fence_after();
+        if constexpr (DQ) {
+          if (!(ok = mbar_wait(bar(B_DSSM), idx & 1, ab, kSiteBMmaDS))) break;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)                           // dQ_i = dS K  -> region B
-          mma_f16_ss(tmem + C::kColB, smem_desc_sw128(dsAddr + kk * 2048, C::kPanelBytes, 1024),
-                     smem_desc_sw128(kAddr + kk * 2048, C::kPanelBytes, 1024), kIdescQ,
-                     kk > 0 ? 1u : 0u);
-        tc_commit(bar(B_DQ));
+          for (int kk = 0; kk < 8; ++kk)                         // dQ_i = dS K  -> region B
+            mma_f16_ss(tmem + C::kColB, smem_desc_sw128(dsAddr + kk * 2048, C::kPanelBytes, 1024),
+                       smem_desc_sw128(kAddr + kk * 2048, C::kPanelBytes, 1024), kIdescQ,
+                       kk > 0 ? 1u : 0u);
+          tc_commit(bar(B_DQ));
+        }
+        // Without dQ, region B takes dP^T of the next block after this dK in
+        // issue order, and its completion (B_DP) implies dK has read dS^T.
         tc_commit(bar(B_QE(s)));
       }
       tc_commit(bar(B_FINAL));
@@ -403,6 +411,7 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(B_DS));
+      if constexpr (!DQ) continue;
       // the dS buffer doubles as the dQ staging area: wait until the dQ
       // reduction of the previous block has left it
       if (idx > 0 && !(ok = mbar_wait_warp(bar(B_DQSMEM), (idx - 1) & 1, ab, kSiteBSmDQ))) break;
@@ -445,7 +454,7 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
         }
       }
     }
-  } else if (warp < 12) {
+  } else if (DQ && warp < 12) {
     // ------------------------------------------------------------ dQ reduction (thread = query row)
     // dQ_i leaves TMEM at once: head-dim columns [0, 64) go to the dS buffer
     // (free once the dQ MMA has read it) as two 128-byte swizzled boxes of 32
@@ -521,11 +530,11 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
   }
 }
 
-template <int D, bool CAUSAL, int NPOLY>
+template <int D, bool CAUSAL, int NPOLY, bool DQ>
 cudaError_t launch_main_impl(const BwdParams& p, cudaStream_t stream) {
   using C = BwdCfg<D>;
-  auto kern = bwd_main_kernel<D, CAUSAL, NPOLY>;
-  cudaError_t e = set_smem_once<bwd_main_kernel<D, CAUSAL, NPOLY>>(C::kSmemBytes);
+  auto kern = bwd_main_kernel<D, CAUSAL, NPOLY, DQ>;
+  cudaError_t e = set_smem_once<bwd_main_kernel<D, CAUSAL, NPOLY, DQ>>(C::kSmemBytes);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(p.n_kv) * static_cast<unsigned>(p.BH);
   kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(p);
@@ -554,17 +563,19 @@ cudaError_t launch_bwd_preprocess(const uint16_t* o, const uint16_t* dout, float
 }
 
 template <int D, bool CAUSAL>
-cudaError_t launch_main_np(const BwdParams& p, cudaStream_t stream) {
+cudaError_t launch_main_np(const BwdParams& p, bool with_dq, cudaStream_t stream) {
+  if (!with_dq) return launch_main_impl<D, CAUSAL, 0, false>(p, stream);
   switch (p.poly_groups) {
-    case 1: return launch_main_impl<D, CAUSAL, 1>(p, stream);
-    case 2: return launch_main_impl<D, CAUSAL, 2>(p, stream);
-    default: return launch_main_impl<D, CAUSAL, 0>(p, stream);
+    case 1: return launch_main_impl<D, CAUSAL, 1, true>(p, stream);
+    case 2: return launch_main_impl<D, CAUSAL, 2, true>(p, stream);
+    default: return launch_main_impl<D, CAUSAL, 0, true>(p, stream);
   }
 }
 
-cudaError_t launch_bwd_main(const BwdParams& p, int d, bool causal, cudaStream_t stream) {
-  if (d == 64) return causal ? launch_main_np<64, true>(p, stream) : launch_main_np<64, false>(p, stream);
-  return causal ? launch_main_np<128, true>(p, stream) : launch_main_np<128, false>(p, stream);
+cudaError_t launch_bwd_main(const BwdParams& p, int d, bool causal, bool with_dq, cudaStream_t stream) {
+  if (d == 64)
+    return causal ? launch_main_np<64, true>(p, with_dq, stream) : launch_main_np<64, false>(p, with_dq, stream);
+  return causal ? launch_main_np<128, true>(p, with_dq, stream) : launch_main_np<128, false>(p, with_dq, stream);
 }
 
 cudaError_t launch_bwd_postprocess(const float* dq_acc, uint16_t* dq, long long n, float scale,

@@ -84,6 +84,7 @@ struct BwdParams {
   float* dq_acc;        // [BH, N, d] fp32, zeroed by the preprocess kernel
   uint16_t* dk;         // bf16 [BH, N, d]
   uint16_t* dv;
+  uint16_t* dq;         // bf16 [BH, N, d]: written directly by the deterministic dQ kernel
   unsigned int* status;
   int N;
   int BH;
@@ -96,10 +97,13 @@ struct BwdParams {
 
 constexpr int kDefaultBwdPolyGroups = 0;
 
-// D = rowsum(dO o O) per row, and dq_acc <- 0.
+// D = rowsum(dO o O) per row, and dq_acc <- 0 (dq_acc == nullptr: D only).
 cudaError_t launch_bwd_preprocess(const uint16_t* o, const uint16_t* dout, float* delta,
                                   float* dq_acc, long long rows, int d, cudaStream_t stream);
-cudaError_t launch_bwd_main(const BwdParams& p, int d, bool causal, cudaStream_t stream);
+// with_dq: also accumulate dQ into dq_acc (atomic order); without: dK, dV only.
+cudaError_t launch_bwd_main(const BwdParams& p, int d, bool causal, bool with_dq, cudaStream_t stream);
+// Deterministic dQ: one CTA per query block, key blocks in ascending order.
+cudaError_t launch_bwd_dq(const BwdParams& p, int d, bool causal, cudaStream_t stream);
 // dq <- bf16(scale * dq_acc)
 cudaError_t launch_bwd_postprocess(const float* dq_acc, uint16_t* dq, long long n, float scale,
                                    cudaStream_t stream);

@@ -94,6 +94,32 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  float scale, int causal, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Bytes of scratch fa_bwd_deterministic needs (fp32 D [B, H, N], rounded up
+ * to 256 bytes).  Returns 0 for an unsupported d or a negative size.
+ */
+size_t fa_bwd_deterministic_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Deterministic backward: same arguments, layouts and results as fa_bwd,
+ * with a workspace of at least fa_bwd_deterministic_workspace_size() bytes
+ * (256-byte aligned).  dQ, dK and dV are bitwise identical from run to run
+ * on the same device.  fa_bwd adds each key block's share of dQ into an fp32
+ * buffer from many thread blocks, in an order that varies; here one kernel
+ * produces dK and dV (one thread block per key block, as in fa_bwd) and a
+ * second owns each 128-row query block, recomputes S and dP for it
+ * (the same recomputation from L, "How it works") and sums dS K over the
+ * key blocks in ascending order.  The extra recomputation costs two more
+ * tile products per (query block, key block) pair; no dQ reductions go to
+ * memory.  The pages fix only that the backward recomputes P from L; how
+ * dQ is accumulated is this library's design, and this is its reproducible
+ * form.
+ */
+fa_status fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,
+                               const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                               int B, int H, int N, int d, float scale, int causal,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Allocation-free backward.  No counterpart in the papers: it exists for
  * callers that cannot allocate device memory themselves (code inside a host
  * framework that owns all device memory through its own pool, or a
