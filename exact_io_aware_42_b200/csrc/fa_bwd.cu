@@ -41,34 +41,44 @@
 namespace fa {
 namespace {
 
-template <int D>
+template <int D, bool DQ>
 struct BwdCfg {
   static constexpr int kPanels = D / 64;
   static constexpr int kPanelBytes = 128 * 128;
   static constexpr int kTileBytes = 128 * D * 2;       // one 128 x D bf16 tile
-  static constexpr int kStages = (D == 128) ? 2 : 3;   // (Q_i, dO_i) ring depth
-  static constexpr int kThreads = 448;
+  // Ring depths: (dO_i, L_i, D_i) and Q_i.  Q_i is read first (S^T) and last
+  // (dK), so its ring is one stage deeper where the dS buffer's space is free
+  // (no dQ product); the next block's S^T then never waits for its Q tile.
+  static constexpr int kStagesD = (D == 128) ? 2 : 3;
+  static constexpr int kStagesQ = kStagesD + (DQ ? 0 : 1);
+  // 14 warps with the dQ drain warps, 10 without (the roles keep their
+  // order: P/dS 0-7, [dQ 8-11], producer, MMA).
+  static constexpr int kThreads = DQ ? 448 : 320;
   // All swizzled tiles are 1024-byte aligned offsets from the (1024-aligned)
   // dynamic shared memory base.
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kTileBytes;
-  static constexpr int kOffQ = 2 * kTileBytes;          // + s * 2 * kTileBytes
-  static constexpr int kOffDS = kOffQ + kStages * 2 * kTileBytes;   // dS^T, 128 x 128 bf16
-  static constexpr int kOffLD = kOffDS + 128 * 128 * 2;             // + s * 1024: L2[128], D[128]
-  static constexpr int kOffBar = kOffLD + kStages * 1024;
-  static constexpr int kNumBars = 1 + 2 * kStages + 10;
+  static constexpr int kOffQ = 2 * kTileBytes;                        // + s * kTileBytes
+  static constexpr int kOffDO = kOffQ + kStagesQ * kTileBytes;        // + s * kTileBytes
+  static constexpr int kOffDS = kOffDO + kStagesD * kTileBytes;       // dS^T, 128 x 128 bf16 (dQ only)
+  static constexpr int kOffL = kOffDS + (DQ ? 128 * 128 * 2 : 0);     // + s * 512: L log2 e [128], Q ring
+  static constexpr int kOffDl = kOffL + kStagesQ * 512;               // + s * 512: D [128], dO ring
+  static constexpr int kOffBar = kOffDl + kStagesD * 512;
+  static constexpr int kNumBars = 1 + 2 * kStagesQ + 2 * kStagesD + 10;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
   static constexpr uint32_t kTmemCols = 512;
   // TMEM: columns [0,128) hold S^T, then P^T (bf16); [128,256) hold dP^T,
   // then dS^T (bf16), then dQ_i.  S^T of the next block is issued right after
-  // dK of this one, before dQ, so the next P phase overlaps dQ and its drain.
+  // dV of this one, so the next P phase overlaps dK, dQ and the dQ drain.
   static constexpr uint32_t kColA = 0;
   static constexpr uint32_t kColB = 128;
   static constexpr uint32_t kColDV = 256;
   static constexpr uint32_t kColDK = 256 + D;
 };
-static_assert(BwdCfg<128>::kSmemBytes <= 232448, "backward d=128 shared memory");
+static_assert(BwdCfg<128, true>::kSmemBytes <= 232448, "backward d=128 shared memory");
+static_assert(BwdCfg<128, false>::kSmemBytes <= 232448, "backward d=128 shared memory");
+static_assert(BwdCfg<64, false>::kSmemBytes <= 232448, "backward d=64 shared memory");
 
 enum : unsigned int { kSiteBProd = 16, kSiteBMmaKV, kSiteBMmaQ, kSiteBMmaFree, kSiteBMmaP, kSiteBMmaDS,
                       kSiteBSmS, kSiteBSmDP, kSiteBSmDQ, kSiteBDq, kSiteBEpi, kSiteBDrain, kSiteBAlign };
@@ -147,9 +157,10 @@ __device__ __forceinline__ void st_global_v4(void* dst, uint32_t a, uint32_t b, 
 // kernel computes dQ): no dS staging in shared memory, no dQ warps' work,
 // and the MMA issuer waits on nothing of dQ.
 template <int D, bool CAUSAL, int NPOLY, bool DQ>
-__global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant__ BwdParams p) {
-  using C = BwdCfg<D>;
-  constexpr int NS = C::kStages;
+__global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(const __grid_constant__ BwdParams p) {
+  using C = BwdCfg<D, DQ>;
+  constexpr int NQ = C::kStagesQ;
+  constexpr int ND = C::kStagesD;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   if (sbase & 1023u) {   // the swizzled layouts below need a 1024-byte aligned base
@@ -158,12 +169,14 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
   }
   auto bar = [&](int i) -> uint32_t { return sbase + C::kOffBar + 8 * i; };
   const int B_KV = 0;
-  auto B_QF = [](int s) { return 1 + s; };
-  auto B_QE = [](int s) { return 1 + NS + s; };
+  auto B_QF = [](int s) { return 1 + s; };             // Q_i landed (L_i written)
+  auto B_QE = [](int s) { return 1 + NQ + s; };        // Q_i's slot free
+  auto B_DF = [](int s) { return 1 + 2 * NQ + s; };    // dO_i landed (D_i written)
+  auto B_DE = [](int s) { return 1 + 2 * NQ + ND + s; };
   // B_DS: dS^T is in TMEM (for dK); B_DSSM: dS is in shared memory (for dQ);
   // B_DQFREE: dQ_i has left TMEM (its region may take the next dP^T);
   // B_DQSMEM: the dS buffer, used to stage dQ_i, is free again.
-  const int B_S = 1 + 2 * NS, B_DP = B_S + 1, B_P = B_S + 2, B_DS = B_S + 3, B_DQ = B_S + 4,
+  const int B_S = 1 + 2 * NQ + 2 * ND, B_DP = B_S + 1, B_P = B_S + 2, B_DS = B_S + 3, B_DQ = B_S + 4,
             B_DQFREE = B_S + 5, B_FINAL = B_S + 6, B_DRAIN = B_S + 7, B_DQSMEM = B_S + 8,
             B_DSSM = B_S + 9;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
@@ -171,6 +184,8 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  constexpr int kWarpProd = DQ ? 12 : 8;
+  constexpr int kWarpMma = kWarpProd + 1;
   // Head-major order: the CTAs resident at any time cover a few heads, so
   // their dQ accumulators (and K, V, Q, dO) stay in L2.  Within a head the
   // key blocks with the most query blocks (small j, causal) go first.
@@ -181,9 +196,13 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_KV), 1);
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < NQ; ++s) {
       mbar_init(bar(B_QF(s)), 1);
       mbar_init(bar(B_QE(s)), 1);
+    }
+    for (int s = 0; s < ND; ++s) {
+      mbar_init(bar(B_DF(s)), 1);
+      mbar_init(bar(B_DE(s)), 1);
     }
     mbar_init(bar(B_S), 1);
     mbar_init(bar(B_DP), 1);
@@ -198,7 +217,7 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 13) {
+  if (warp == kWarpMma) {
     tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
     tmem_relinquish();
   }
@@ -208,12 +227,12 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
   const uint32_t tmem = *tmem_slot;
   const Abort ab{abort_flag, p.status};
   const uint32_t kAddr = sbase + C::kOffK, vAddr = sbase + C::kOffV, dsAddr = sbase + C::kOffDS;
-  auto qAddr = [&](int s) -> uint32_t { return sbase + C::kOffQ + s * 2 * C::kTileBytes; };
-  auto doAddr = [&](int s) -> uint32_t { return qAddr(s) + C::kTileBytes; };
+  auto qAddr = [&](int s) -> uint32_t { return sbase + C::kOffQ + s * C::kTileBytes; };
+  auto doAddr = [&](int s) -> uint32_t { return sbase + C::kOffDO + s * C::kTileBytes; };
 
-  if (warp == 12) {
+  if (warp == kWarpProd) {
     // ------------------------------------------------------------ producer
-    int issued = 0;
+    int issued_q = 0, issued_d = 0;
     bool ok = true;
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_q);
@@ -224,46 +243,53 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
         tma_load_3d(vAddr + pn * C::kPanelBytes, &p.tm_v, bar(B_KV), pn * 64, j * 128, bh);
       }
     }
-    for (int idx = 0; idx < n_i && ok; ++idx) {
-      const int i = i0 + idx;
-      const int s = idx % NS;
-      const uint32_t ph = (idx / NS) & 1;
-      bool w = true;
-      if (lane == 0) w = mbar_wait(bar(B_QE(s)), ph ^ 1, ab, kSiteBProd);
-      ok = __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
-      if (!ok) break;
-      // L (in log2 units) and D of the 128 query rows, +inf / 0 past N
-      float* ld = reinterpret_cast<float*>(smem + C::kOffLD + s * 1024);
-      float lv[4], dv4[4];
+    // Per query block: L_i (log2 units, +inf past N) beside Q_i, D_i (0 past
+    // N) beside dO_i; each is written by the warp before the arrive that
+    // publishes its slot.
+    auto stage_rows = [&](float* dst, const float* src, int i, float mul, float pad) {
+      float v4[4];
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         const int q = i * 128 + lane * 4 + t;
-        const bool in = q < p.N;
-        const size_t g = static_cast<size_t>(bh) * p.N + q;
-        lv[t] = in ? p.lse[g] * 1.4426950408889634f : INFINITY;
-        dv4[t] = in ? p.delta[g] : 0.f;
+        v4[t] = q < p.N ? src[static_cast<size_t>(bh) * p.N + q] * mul : pad;
       }
-      reinterpret_cast<float4*>(ld)[lane] = make_float4(lv[0], lv[1], lv[2], lv[3]);
-      reinterpret_cast<float4*>(ld + 128)[lane] = make_float4(dv4[0], dv4[1], dv4[2], dv4[3]);
+      reinterpret_cast<float4*>(dst)[lane] = make_float4(v4[0], v4[1], v4[2], v4[3]);
       __syncwarp();
+    };
+    for (int idx = 0; idx < n_i && ok; ++idx) {
+      const int i = i0 + idx;
+      const int sq = idx % NQ, sd = idx % ND;
+      bool w = true;
+      if (lane == 0) w = mbar_wait(bar(B_QE(sq)), ((idx / NQ) & 1) ^ 1, ab, kSiteBProd);
+      if (!(ok = __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0)) break;
+      stage_rows(reinterpret_cast<float*>(smem + C::kOffL + sq * 512), p.lse, i, 1.4426950408889634f, INFINITY);
       if (lane == 0) {
-        mbar_arrive_expect_tx(bar(B_QF(s)), 2 * C::kTileBytes);
-        for (int pn = 0; pn < C::kPanels; ++pn) {
-          tma_load_3d(qAddr(s) + pn * C::kPanelBytes, &p.tm_q, bar(B_QF(s)), pn * 64, i * 128, bh);
-          tma_load_3d(doAddr(s) + pn * C::kPanelBytes, &p.tm_do, bar(B_QF(s)), pn * 64, i * 128, bh);
-        }
+        mbar_arrive_expect_tx(bar(B_QF(sq)), C::kTileBytes);
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_3d(qAddr(sq) + pn * C::kPanelBytes, &p.tm_q, bar(B_QF(sq)), pn * 64, i * 128, bh);
+        ++issued_q;
+        w = mbar_wait(bar(B_DE(sd)), ((idx / ND) & 1) ^ 1, ab, kSiteBProd);
       }
-      ++issued;
+      if (!(ok = __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0)) break;
+      stage_rows(reinterpret_cast<float*>(smem + C::kOffDl + sd * 512), p.delta, i, 1.f, 0.f);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar(B_DF(sd)), C::kTileBytes);
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_3d(doAddr(sd) + pn * C::kPanelBytes, &p.tm_do, bar(B_DF(sd)), pn * 64, i * 128, bh);
+        ++issued_d;
+      }
     }
-    if (lane == 0 && *abort_flag) {
+    if (lane == 0 && *abort_flag) {   // let the copies in flight land before the CTA leaves
       volatile int never = 0;
       const Abort drain{&never, p.status};
       mbar_wait(bar(B_KV), 0, drain, kSiteBDrain);
-      const int first = issued > NS ? issued - NS : 0;
-      for (int q = first; q < issued; ++q) mbar_wait(bar(B_QF(q % NS)), (q / NS) & 1, drain, kSiteBDrain);
+      for (int q = (issued_q > NQ ? issued_q - NQ : 0); q < issued_q; ++q)
+        mbar_wait(bar(B_QF(q % NQ)), (q / NQ) & 1, drain, kSiteBDrain);
+      for (int q = (issued_d > ND ? issued_d - ND : 0); q < issued_d; ++q)
+        mbar_wait(bar(B_DF(q % ND)), (q / ND) & 1, drain, kSiteBDrain);
     }
     __syncwarp();
-  } else if (warp == 13) {
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdescKK = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
@@ -291,26 +317,30 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
         tc_commit(bar(B_S));
       }
       for (int idx = 0; idx < n_i && ok; ++idx) {
-        const int s = idx % NS;
+        const int sq = idx % NQ, sd = idx % ND;
         if (DQ && idx > 0) {   // dQ of the previous block has left region B
           if (!(ok = mbar_wait(bar(B_DQFREE), (idx - 1) & 1, ab, kSiteBMmaFree))) break;
-          tc_fence_after();
         }
-        gemm_kk(C::kColB, vAddr, doAddr(s));                     // dP^T = V dO^T
+        if (!(ok = mbar_wait(bar(B_DF(sd)), (idx / ND) & 1, ab, kSiteBMmaQ))) break;
+        tc_fence_after();
+        gemm_kk(C::kColB, vAddr, doAddr(sd));                    // dP^T = V dO^T
         tc_commit(bar(B_DP));
         if (!(ok = mbar_wait(bar(B_P), idx & 1, ab, kSiteBMmaP))) break;
         tc_fence_after();
-        gemm_ts(C::kColDV, C::kColA, doAddr(s), idx > 0);        // dV += P^T dO
-        if (!(ok = mbar_wait(bar(B_DS), idx & 1, ab, kSiteBMmaDS))) break;
-        tc_fence_after();
-        gemm_ts(C::kColDK, C::kColB, qAddr(s), idx > 0);         // dK += dS^T Q
-        if (idx + 1 < n_i) {                                     // S^T of the next block
-          const int s1 = (idx + 1) % NS;
-          if (!(ok = mbar_wait(bar(B_QF(s1)), ((idx + 1) / NS) & 1, ab, kSiteBMmaQ))) break;
+        gemm_ts(C::kColDV, C::kColA, doAddr(sd), idx > 0);       // dV += P^T dO
+        // S^T of the next block goes to region A right behind dV, which is
+        // the last reader of P^T there (the dS phase keeps its own copy of P
+        // in registers), so the next P phase overlaps dK and dP.
+        if (idx + 1 < n_i) {
+          const int s1 = (idx + 1) % NQ;
+          if (!(ok = mbar_wait(bar(B_QF(s1)), ((idx + 1) / NQ) & 1, ab, kSiteBMmaQ))) break;
           tc_fence_after();
           gemm_kk(C::kColA, kAddr, qAddr(s1));
           tc_commit(bar(B_S));
         }
+        if (!(ok = mbar_wait(bar(B_DS), idx & 1, ab, kSiteBMmaDS))) break;
+        tc_fence_after();
+        gemm_ts(C::kColDK, C::kColB, qAddr(sq), idx > 0);        // dK += dS^T Q
         if constexpr (DQ) {
           if (!(ok = mbar_wait(bar(B_DSSM), idx & 1, ab, kSiteBMmaDS))) break;
           tc_fence_after();
@@ -323,7 +353,10 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
         }
         // Without dQ, region B takes dP^T of the next block after this dK in
         // issue order, and its completion (B_DP) implies dK has read dS^T.
-        tc_commit(bar(B_QE(s)));
+        // dK is the last reader of Q_i, and it follows the dS phase, the last
+        // reader of L_i and D_i: both slots are free once it completes.
+        tc_commit(bar(B_QE(sq)));
+        tc_commit(bar(B_DE(sd)));
       }
       tc_commit(bar(B_FINAL));
       tc_commit(bar(B_DRAIN));
@@ -348,14 +381,14 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
     bool ok = true;
     for (int idx = 0; idx < n_i && ok; ++idx) {
       const int i = i0 + idx;
-      const int s = idx % NS;
-      const float4* L4 = reinterpret_cast<const float4*>(smem + C::kOffLD + s * 1024) + 16 * wg;
-      const float4* D4 = L4 + 32;
+      const float4* L4 = reinterpret_cast<const float4*>(smem + C::kOffL + (idx % NQ) * 512) + 16 * wg;
+      const float4* D4 = reinterpret_cast<const float4*>(smem + C::kOffDl + (idx % ND) * 512) + 16 * wg;
       const bool diag = CAUSAL && i == j;
       const uint32_t tS = tmem + C::kColA + lane_off + col_half;
       const uint32_t tDP = tmem + C::kColB + lane_off + col_half;
       if (!(ok = mbar_wait_warp(bar(B_S), idx & 1, ab, kSiteBSmS))) break;
       tc_fence_after();
+      uint32_t pp[32];   // this thread's P^T row, packed bf16: the dS phase reads it here
       {
         uint32_t u[64];
         tmem_ld64(tS, u);
@@ -381,7 +414,9 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
           u[2 * c4] = pack_bf16x2(pv[0], pv[1]);
           u[2 * c4 + 1] = pack_bf16x2(pv[2], pv[3]);
         }
-        tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pp[c] = u[c];
+        tmem_st32(tS, pp);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -389,25 +424,25 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
       if (!(ok = mbar_wait_warp(bar(B_DP), idx & 1, ab, kSiteBSmDP))) break;
       tc_fence_after();
       uint32_t ds[32];
-      {
-        uint32_t dp[64], pp[32];
-        tmem_ld64(tDP, dp);
-        tmem_ld32(tS, pp);
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
+      for (int h = 0; h < 2; ++h) {                      // 32 dP^T columns at a time
+        uint32_t dp[32];
+        tmem_ld32(tDP + 32 * h, dp);
+#pragma unroll
+        for (int c4 = 8 * h; c4 < 8 * h + 8; ++c4) {
           const float4 d4 = D4[c4];
           const float dq[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
           for (int t2 = 0; t2 < 2; ++t2) {
             const int c2 = 2 * c4 + t2;                  // packed pair index
             const float p0 = __uint_as_float(pp[c2] << 16), p1 = __uint_as_float(pp[c2] & 0xFFFF0000u);
-            const float d0 = p0 * (__uint_as_float(dp[2 * c2]) - dq[2 * t2]);
-            const float d1 = p1 * (__uint_as_float(dp[2 * c2 + 1]) - dq[2 * t2 + 1]);
+            const float d0 = p0 * (__uint_as_float(dp[2 * c2 - 32 * h]) - dq[2 * t2]);
+            const float d1 = p1 * (__uint_as_float(dp[2 * c2 + 1 - 32 * h]) - dq[2 * t2 + 1]);
             ds[c2] = pack_bf16x2(d0, d1);
           }
         }
-        tmem_st32(tDP, ds);
       }
+      tmem_st32(tDP, ds);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(B_DS));
@@ -524,7 +559,7 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 13) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
@@ -532,7 +567,7 @@ __global__ void __launch_bounds__(448, 1) bwd_main_kernel(const __grid_constant_
 
 template <int D, bool CAUSAL, int NPOLY, bool DQ>
 cudaError_t launch_main_impl(const BwdParams& p, cudaStream_t stream) {
-  using C = BwdCfg<D>;
+  using C = BwdCfg<D, DQ>;
   auto kern = bwd_main_kernel<D, CAUSAL, NPOLY, DQ>;
   cudaError_t e = set_smem_once<bwd_main_kernel<D, CAUSAL, NPOLY, DQ>>(C::kSmemBytes);
   if (e != cudaSuccess) return e;
