@@ -4,6 +4,7 @@ torch provides device memory and the current CUDA stream; every step of the
 computation runs in the library's kernels.  Functions mirror include/fa.h:
 
 * ``fwd(q, k, v, causal, scale)``            -> (o, lse)
+  (k, v may have fewer heads than q: grouped K/V heads, H a multiple of H_kv)
 * ``bwd(q, k, v, o, do, lse, causal, scale, deterministic=False)`` -> (dq, dk, dv)
 * ``quant_fp8(x, signs=None)``               -> (x8 as uint8, block scales)
 * ``fwd_fp8(q8, k8, v8, sq, sk, sv, causal, scale)`` -> (o, lse)
@@ -29,6 +30,17 @@ def _stream() -> int:
     return torch.cuda.current_stream().cuda_stream
 
 
+def _kv_shape(name: str, q_shape, kv: torch.Tensor):
+    """[B, H_kv, N, d] with H_kv dividing H; returns H_kv."""
+    B, H, N, d = q_shape
+    if kv.dim() != 4 or kv.shape[0] != B or kv.shape[2] != N or kv.shape[3] != d:
+        raise ValueError(f"{name} has shape {tuple(kv.shape)}, expected [B, H_kv, N, d] = [{B}, H_kv, {N}, {d}]")
+    h_kv = kv.shape[1]
+    if h_kv < 1 or H % h_kv != 0:
+        raise ValueError(f"{name} has {h_kv} heads, which does not divide H = {H}")
+    return h_kv
+
+
 def _check_bhnd(name: str, t: torch.Tensor, dtype, shape=None) -> None:
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
@@ -49,15 +61,21 @@ def fwd(q, k, v, causal: bool = False, scale: Optional[float] = None, out=None, 
     """Exact attention forward (bf16).  Returns (o bf16 [B,H,N,d], lse fp32 [B,H,N])."""
     _check_bhnd("q", q, torch.bfloat16)
     B, H, N, d = q.shape
-    _check_bhnd("k", k, torch.bfloat16, q.shape)
-    _check_bhnd("v", v, torch.bfloat16, q.shape)
+    h_kv = _kv_shape("k", q.shape, k)
+    _check_bhnd("k", k, torch.bfloat16, (B, h_kv, N, d))
+    _check_bhnd("v", v, torch.bfloat16, (B, h_kv, N, d))
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     o = torch.empty_like(q) if out is None else out
     lse_t = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
-    code = lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), B, H, N, d, float(scale),
-                        int(bool(causal)), _stream())
-    check("fa_fwd", code)
+    if h_kv == H:
+        code = lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), B, H, N, d, float(scale),
+                            int(bool(causal)), _stream())
+        check("fa_fwd", code)
+    else:
+        code = lib().fa_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), B, H, h_kv, N, d,
+                                float(scale), int(bool(causal)), _stream())
+        check("fa_fwd_gqa", code)
     return o, lse_t
 
 
@@ -76,7 +94,10 @@ def bwd(q, k, v, o, do, lse, causal: bool = False, scale: Optional[float] = None
     gradients (dQ by a separate query-block-major kernel)."""
     _check_bhnd("q", q, torch.bfloat16)
     B, H, N, d = q.shape
-    for name, t in (("k", k), ("v", v), ("o", o), ("do", do)):
+    h_kv = _kv_shape("k", q.shape, k)
+    for name, t in (("k", k), ("v", v)):
+        _check_bhnd(name, t, torch.bfloat16, (B, h_kv, N, d))
+    for name, t in (("o", o), ("do", do)):
         _check_bhnd(name, t, torch.bfloat16, q.shape)
     if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous fp32 [B, H, N] tensor")
@@ -88,10 +109,16 @@ def bwd(q, k, v, o, do, lse, causal: bool = False, scale: Optional[float] = None
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    name = "fa_bwd_deterministic" if deterministic else "fa_bwd"
-    code = getattr(lib(), name)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
-                                _ptr(dk), _ptr(dv), B, H, N, d, float(scale), int(bool(causal)),
-                                _ptr(workspace), workspace.numel(), _stream())
+    if h_kv == H:
+        name = "fa_bwd_deterministic" if deterministic else "fa_bwd"
+        code = getattr(lib(), name)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
+                                    _ptr(dk), _ptr(dv), B, H, N, d, float(scale), int(bool(causal)),
+                                    _ptr(workspace), workspace.numel(), _stream())
+    else:
+        name = "fa_bwd_gqa"
+        code = lib().fa_bwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
+                                _ptr(dk), _ptr(dv), B, H, h_kv, N, d, float(scale), int(bool(causal)),
+                                int(bool(deterministic)), _ptr(workspace), workspace.numel(), _stream())
     check(name, code)
     return dq, dk, dv
 
@@ -116,18 +143,20 @@ def fwd_fp8(q8, k8, v8, sq, sk, sv, causal: bool = False, scale: Optional[float]
     """FP8 attention forward on quantised inputs.  Returns (o bf16, lse fp32)."""
     _check_bhnd("q8", q8, torch.uint8)
     B, H, N, d = q8.shape
-    _check_bhnd("k8", k8, torch.uint8, q8.shape)
-    _check_bhnd("v8", v8, torch.uint8, q8.shape)
-    for name, s in (("sq", sq), ("sk", sk), ("sv", sv)):
-        if s.dtype != torch.float32 or tuple(s.shape) != (B, H, n_blocks(N)) or not s.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous fp32 [B, H, ceil(N/128)] tensor")
+    h_kv = _kv_shape("k8", q8.shape, k8)
+    _check_bhnd("k8", k8, torch.uint8, (B, h_kv, N, d))
+    _check_bhnd("v8", v8, torch.uint8, (B, h_kv, N, d))
+    for name, s, h in (("sq", sq, H), ("sk", sk, h_kv), ("sv", sv, h_kv)):
+        if s.dtype != torch.float32 or tuple(s.shape) != (B, h, n_blocks(N)) or not s.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous fp32 [B, {h}, ceil(N/128)] tensor")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q8.device) if out is None else out
     lse_t = torch.empty((B, H, N), dtype=torch.float32, device=q8.device) if lse is None else lse
-    code = lib().fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk), _ptr(sv), _ptr(o),
-                            _ptr(lse_t), B, H, N, d, float(scale), int(bool(causal)), _stream())
-    check("fa_fwd_fp8", code)
+    code = lib().fa_fwd_fp8_gqa(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk), _ptr(sv), _ptr(o),
+                                _ptr(lse_t), B, H, h_kv, N, d, float(scale), int(bool(causal)),
+                                _stream())
+    check("fa_fwd_fp8_gqa", code)
     return o, lse_t
 
 

@@ -127,15 +127,23 @@ fa_status check_shape(int B, int H, int N, int d, float scale) {
   return FA_OK;
 }
 
+// Grouped K/V heads: 1 <= H_kv, H a multiple of H_kv.
+fa_status check_kv_heads(int H, int H_kv) {
+  if (H_kv < 1 || H % H_kv != 0) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
 }  // namespace
 }  // namespace fa
 
 using namespace fa;
 
-extern "C" fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
-                            int B, int H, int N, int d, float scale, int causal, void* stream) {
+extern "C" fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
+                                int B, int H, int H_kv, int N, int d, float scale, int causal,
+                                void* stream) {
   fa_status st = check_shape(B, H, N, d, scale);
   if (st != FA_OK) return st;
+  if (H > 0 && (st = check_kv_heads(H, H_kv)) != FA_OK) return st;
   if (static_cast<long long>(B) * H * N == 0) return FA_OK;
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
@@ -148,15 +156,17 @@ extern "C" fa_status fa_fwd(const void* q, const void* k, const void* v, void* o
   std::memset(&p, 0, sizeof(p));
   const int BH = B * H;
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const int BHkv = B * H_kv;
   if (!encode_3d(&p.tm_q, q, bf, 2, d, N, BH, 64, kBlockM) ||
-      !encode_3d(&p.tm_k, k, bf, 2, d, N, BH, 64, kBlockN) ||
-      !encode_3d(&p.tm_v, v, bf, 2, d, N, BH, 64, kBlockN) ||
+      !encode_3d(&p.tm_k, k, bf, 2, d, N, BHkv, 64, kBlockN) ||
+      !encode_3d(&p.tm_v, v, bf, 2, d, N, BHkv, 64, kBlockN) ||
       !encode_3d(&p.tm_o, o, bf, 2, d, N, BH, 64, kBlockM))
     return FA_ERR_INVALID_ARG;
   p.lse = lse;
   p.status = di->status;
   p.N = N;
   p.BH = BH;
+  p.kv_group = H / H_kv;
   p.n_kv = (N + kBlockN - 1) / kBlockN;
   p.n_pairs = ((N + kBlockM - 1) / kBlockM + 1) / 2;
   p.scale = scale;
@@ -168,6 +178,11 @@ extern "C" fa_status fa_fwd(const void* q, const void* k, const void* v, void* o
     return FA_ERR_LAUNCH;
   }
   return FA_OK;
+}
+
+extern "C" fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                            int B, int H, int N, int d, float scale, int causal, void* stream) {
+  return fa_fwd_gqa(q, k, v, o, lse, B, H, H, N, d, scale, causal, stream);
 }
 
 extern "C" size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
@@ -189,11 +204,12 @@ namespace {
 // atomic one accumulates dQ in fp32 scratch by TMA reductions, the
 // deterministic one runs the main kernel without dQ and the dQ kernel.
 fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                     const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
-                     float scale, int causal, void* workspace, size_t workspace_bytes, void* stream,
-                     bool deterministic) {
+                     const float* lse, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N,
+                     int d, float scale, int causal, void* workspace, size_t workspace_bytes,
+                     void* stream, bool deterministic) {
   fa_status st = check_shape(B, H, N, d, scale);
   if (st != FA_OK) return st;
+  if (H > 0 && (st = check_kv_heads(H, H_kv)) != FA_OK) return st;
   if (static_cast<long long>(B) * H * N == 0) return FA_OK;
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
@@ -216,8 +232,9 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   BwdParams p;
   std::memset(&p, 0, sizeof(p));
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  if (!encode_3d(&p.tm_q, q, bf, 2, d, N, BH, 64, 128) || !encode_3d(&p.tm_k, k, bf, 2, d, N, BH, 64, 128) ||
-      !encode_3d(&p.tm_v, v, bf, 2, d, N, BH, 64, 128) || !encode_3d(&p.tm_do, dout, bf, 2, d, N, BH, 64, 128))
+  const int BHkv = B * H_kv;
+  if (!encode_3d(&p.tm_q, q, bf, 2, d, N, BH, 64, 128) || !encode_3d(&p.tm_k, k, bf, 2, d, N, BHkv, 64, 128) ||
+      !encode_3d(&p.tm_v, v, bf, 2, d, N, BHkv, 64, 128) || !encode_3d(&p.tm_do, dout, bf, 2, d, N, BH, 64, 128))
     return FA_ERR_INVALID_ARG;
   if (!deterministic &&
       !encode_3d(&p.tm_dqacc, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, N, BH, 32, 128))
@@ -233,6 +250,7 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   p.BH = BH;
   p.n_kv = (N + 127) / 128;
   p.n_q = (N + 127) / 128;
+  p.kv_group = H / H_kv;
   p.scale = scale;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.poly_groups = bwd_poly_groups();
@@ -259,7 +277,7 @@ extern "C" fa_status fa_bwd(const void* q, const void* k, const void* v, const v
                             const void* dout, const float* lse, void* dq, void* dk, void* dv,
                             int B, int H, int N, int d, float scale, int causal, void* workspace,
                             size_t workspace_bytes, void* stream) {
-  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace,
+  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, H, N, d, scale, causal, workspace,
                     workspace_bytes, stream, false);
 }
 
@@ -268,8 +286,17 @@ extern "C" fa_status fa_bwd_deterministic(const void* q, const void* k, const vo
                                           void* dv, int B, int H, int N, int d, float scale,
                                           int causal, void* workspace, size_t workspace_bytes,
                                           void* stream) {
-  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, workspace,
+  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, H, N, d, scale, causal, workspace,
                     workspace_bytes, stream, true);
+}
+
+extern "C" fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
+                                const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                                int B, int H, int H_kv, int N, int d, float scale, int causal,
+                                int deterministic, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, H_kv, N, d, scale, causal, workspace,
+                    workspace_bytes, stream, deterministic != 0);
 }
 
 extern "C" fa_status fa_quant_fp8(const void* x, void* x8, float* scales, int B, int H, int N,
@@ -309,11 +336,13 @@ extern "C" fa_status fa_quant_fp8(const void* x, void* x8, float* scales, int B,
   return FA_OK;
 }
 
-extern "C" fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* sq,
-                                const float* sk, const float* sv, void* o, float* lse, int B, int H,
-                                int N, int d, float scale, int causal, void* stream) {
+extern "C" fa_status fa_fwd_fp8_gqa(const void* q8, const void* k8, const void* v8, const float* sq,
+                                    const float* sk, const float* sv, void* o, float* lse, int B,
+                                    int H, int H_kv, int N, int d, float scale, int causal,
+                                    void* stream) {
   fa_status st = check_shape(B, H, N, d, scale);
   if (st != FA_OK) return st;
+  if (H > 0 && (st = check_kv_heads(H, H_kv)) != FA_OK) return st;
   if (d != 128) return FA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H * N == 0) return FA_OK;
   if (!q8 || !k8 || !v8 || !sq || !sk || !sv || !o || !lse) return FA_ERR_INVALID_ARG;
@@ -327,9 +356,10 @@ extern "C" fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, 
   std::memset(&p, 0, sizeof(p));
   const int BH = B * H;
   const CUtensorMapDataType u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const int BHkv = B * H_kv;
   if (!encode_3d(&p.tm_q, q8, u8, 1, d, N, BH, 128, kBlockM) ||
-      !encode_3d(&p.tm_k, k8, u8, 1, d, N, BH, 128, kBlockN) ||
-      !encode_3d(&p.tm_v, v8, u8, 1, d, N, BH, 128, kBlockN) ||
+      !encode_3d(&p.tm_k, k8, u8, 1, d, N, BHkv, 128, kBlockN) ||
+      !encode_3d(&p.tm_v, v8, u8, 1, d, N, BHkv, 128, kBlockN) ||
       !encode_3d(&p.tm_o, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, BH, 64, kBlockM))
     return FA_ERR_INVALID_ARG;
   p.lse = lse;
@@ -339,6 +369,7 @@ extern "C" fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, 
   p.sv = sv;
   p.N = N;
   p.BH = BH;
+  p.kv_group = H / H_kv;
   p.n_kv = (N + kBlockN - 1) / kBlockN;
   p.n_pairs = ((N + kBlockM - 1) / kBlockM + 1) / 2;
   p.scale = scale;
@@ -349,6 +380,12 @@ extern "C" fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, 
     return FA_ERR_LAUNCH;
   }
   return FA_OK;
+}
+
+extern "C" fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* sq,
+                                const float* sk, const float* sv, void* o, float* lse, int B, int H,
+                                int N, int d, float scale, int causal, void* stream) {
+  return fa_fwd_fp8_gqa(q8, k8, v8, sq, sk, sv, o, lse, B, H, H, N, d, scale, causal, stream);
 }
 
 extern "C" fa_status fa_selftest_wait_timeout(void* stream) {

@@ -189,10 +189,16 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
   // Head-major order: the CTAs resident at any time cover a few heads, so
   // their dQ accumulators (and K, V, Q, dO) stay in L2.  Within a head the
   // key blocks with the most query blocks (small j, causal) go first.
-  const int bh = blockIdx.x / p.n_kv;
+  // kvh is the K/V head (flattened [B * H_kv]); with grouped K/V heads the
+  // CTA visits the query blocks of its G query heads one head after the
+  // other, so dK and dV sum over the group in TMEM.
+  const int kvh = blockIdx.x / p.n_kv;
   const int j = blockIdx.x % p.n_kv;
   const int i0 = CAUSAL ? j : 0;
-  const int n_i = p.n_q - i0;
+  const int n_i = p.n_q - i0;               // query blocks per query head (>= 1)
+  const int n_it = n_i * p.kv_group;
+  auto q_block = [&](int idx) { return i0 + idx % n_i; };
+  auto q_head = [&](int idx) { return kvh * p.kv_group + idx / n_i; };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_KV), 1);
@@ -239,43 +245,43 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
       tma_prefetch_desc(&p.tm_do);
       mbar_arrive_expect_tx(bar(B_KV), 2 * C::kTileBytes);
       for (int pn = 0; pn < C::kPanels; ++pn) {
-        tma_load_3d(kAddr + pn * C::kPanelBytes, &p.tm_k, bar(B_KV), pn * 64, j * 128, bh);
-        tma_load_3d(vAddr + pn * C::kPanelBytes, &p.tm_v, bar(B_KV), pn * 64, j * 128, bh);
+        tma_load_3d(kAddr + pn * C::kPanelBytes, &p.tm_k, bar(B_KV), pn * 64, j * 128, kvh);
+        tma_load_3d(vAddr + pn * C::kPanelBytes, &p.tm_v, bar(B_KV), pn * 64, j * 128, kvh);
       }
     }
     // Per query block: L_i (log2 units, +inf past N) beside Q_i, D_i (0 past
     // N) beside dO_i; each is written by the warp before the arrive that
     // publishes its slot.
-    auto stage_rows = [&](float* dst, const float* src, int i, float mul, float pad) {
+    auto stage_rows = [&](float* dst, const float* src, int qh, int i, float mul, float pad) {
       float v4[4];
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         const int q = i * 128 + lane * 4 + t;
-        v4[t] = q < p.N ? src[static_cast<size_t>(bh) * p.N + q] * mul : pad;
+        v4[t] = q < p.N ? src[static_cast<size_t>(qh) * p.N + q] * mul : pad;
       }
       reinterpret_cast<float4*>(dst)[lane] = make_float4(v4[0], v4[1], v4[2], v4[3]);
       __syncwarp();
     };
-    for (int idx = 0; idx < n_i && ok; ++idx) {
-      const int i = i0 + idx;
+    for (int idx = 0; idx < n_it && ok; ++idx) {
+      const int i = q_block(idx), qh = q_head(idx);
       const int sq = idx % NQ, sd = idx % ND;
       bool w = true;
       if (lane == 0) w = mbar_wait(bar(B_QE(sq)), ((idx / NQ) & 1) ^ 1, ab, kSiteBProd);
       if (!(ok = __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0)) break;
-      stage_rows(reinterpret_cast<float*>(smem + C::kOffL + sq * 512), p.lse, i, 1.4426950408889634f, INFINITY);
+      stage_rows(reinterpret_cast<float*>(smem + C::kOffL + sq * 512), p.lse, qh, i, 1.4426950408889634f, INFINITY);
       if (lane == 0) {
         mbar_arrive_expect_tx(bar(B_QF(sq)), C::kTileBytes);
         for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_3d(qAddr(sq) + pn * C::kPanelBytes, &p.tm_q, bar(B_QF(sq)), pn * 64, i * 128, bh);
+          tma_load_3d(qAddr(sq) + pn * C::kPanelBytes, &p.tm_q, bar(B_QF(sq)), pn * 64, i * 128, qh);
         ++issued_q;
         w = mbar_wait(bar(B_DE(sd)), ((idx / ND) & 1) ^ 1, ab, kSiteBProd);
       }
       if (!(ok = __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0)) break;
-      stage_rows(reinterpret_cast<float*>(smem + C::kOffDl + sd * 512), p.delta, i, 1.f, 0.f);
+      stage_rows(reinterpret_cast<float*>(smem + C::kOffDl + sd * 512), p.delta, qh, i, 1.f, 0.f);
       if (lane == 0) {
         mbar_arrive_expect_tx(bar(B_DF(sd)), C::kTileBytes);
         for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_3d(doAddr(sd) + pn * C::kPanelBytes, &p.tm_do, bar(B_DF(sd)), pn * 64, i * 128, bh);
+          tma_load_3d(doAddr(sd) + pn * C::kPanelBytes, &p.tm_do, bar(B_DF(sd)), pn * 64, i * 128, qh);
         ++issued_d;
       }
     }
@@ -311,12 +317,12 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
                      (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(bar(B_KV), 0, ab, kSiteBMmaKV);
-      if (ok && n_i > 0 && (ok = mbar_wait(bar(B_QF(0)), 0, ab, kSiteBMmaQ))) {
+      if (ok && n_it > 0 && (ok = mbar_wait(bar(B_QF(0)), 0, ab, kSiteBMmaQ))) {
         tc_fence_after();
         gemm_kk(C::kColA, kAddr, qAddr(0));                      // S^T(0) = K Q^T
         tc_commit(bar(B_S));
       }
-      for (int idx = 0; idx < n_i && ok; ++idx) {
+      for (int idx = 0; idx < n_it && ok; ++idx) {
         const int sq = idx % NQ, sd = idx % ND;
         if (DQ && idx > 0) {   // dQ of the previous block has left region B
           if (!(ok = mbar_wait(bar(B_DQFREE), (idx - 1) & 1, ab, kSiteBMmaFree))) break;
@@ -331,7 +337,7 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
         // S^T of the next block goes to region A right behind dV, which is
         // the last reader of P^T there (the dS phase keeps its own copy of P
         // in registers), so the next P phase overlaps dK and dP.
-        if (idx + 1 < n_i) {
+        if (idx + 1 < n_it) {
           const int s1 = (idx + 1) % NQ;
           if (!(ok = mbar_wait(bar(B_QF(s1)), ((idx + 1) / NQ) & 1, ab, kSiteBMmaQ))) break;
           tc_fence_after();
@@ -379,8 +385,8 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
     const uint32_t col_half = 64u * wg;
     const float cs = p.scale_log2;
     bool ok = true;
-    for (int idx = 0; idx < n_i && ok; ++idx) {
-      const int i = i0 + idx;
+    for (int idx = 0; idx < n_it && ok; ++idx) {
+      const int i = q_block(idx);
       const float4* L4 = reinterpret_cast<const float4*>(smem + C::kOffL + (idx % NQ) * 512) + 16 * wg;
       const float4* D4 = reinterpret_cast<const float4*>(smem + C::kOffDl + (idx % ND) * 512) + 16 * wg;
       const bool diag = CAUSAL && i == j;
@@ -466,7 +472,7 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
       // global stores depend on the key being inside the sequence.  wg 0
       // writes head-dim columns [0, d/2), wg 1 [d/2, d).
       tc_fence_after();
-      const size_t g = (static_cast<size_t>(bh) * p.N + (key_ok ? key : 0)) * D;
+      const size_t g = (static_cast<size_t>(kvh) * p.N + (key_ok ? key : 0)) * D;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {      // 0: dV, 1: dK (times scale)
         const uint32_t src = tmem + (which ? C::kColDK : C::kColDV) + lane_off;
@@ -500,8 +506,8 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
     const int r = threadIdx.x - 256;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     bool ok = true;
-    for (int idx = 0; idx < n_i && ok; ++idx) {
-      const int i = i0 + idx;
+    for (int idx = 0; idx < n_it && ok; ++idx) {
+      const int i = q_block(idx), qh = q_head(idx);
       ok = mbar_wait_warp(bar(B_DQ), idx & 1, ab, kSiteBDq);
       // all four warps agree before any of them enters the named barriers below
       if (!(ok = named_bar_and(2, 128, ok))) break;
@@ -527,7 +533,7 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
       named_bar_sync(2, 128);
       if (r == 0) {
 #pragma unroll
-        for (int b = 0; b < 2; ++b) tma_reduce_add_3d(&p.tm_dqacc, dsAddr + b * 16384, 32 * b, i * 128, bh);
+        for (int b = 0; b < 2; ++b) tma_reduce_add_3d(&p.tm_dqacc, dsAddr + b * 16384, 32 * b, i * 128, qh);
         tma_store_commit();
       }
       if constexpr (D > 64) {
@@ -546,7 +552,7 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
         if (r == 0) {
 #pragma unroll
           for (int b = 0; b < 2; ++b)
-            tma_reduce_add_3d(&p.tm_dqacc, dsAddr + b * 16384, 64 + 32 * b, i * 128, bh);
+            tma_reduce_add_3d(&p.tm_dqacc, dsAddr + b * 16384, 64 + 32 * b, i * 128, qh);
           tma_store_commit();
         }
       }
@@ -571,7 +577,7 @@ cudaError_t launch_main_impl(const BwdParams& p, cudaStream_t stream) {
   auto kern = bwd_main_kernel<D, CAUSAL, NPOLY, DQ>;
   cudaError_t e = set_smem_once<bwd_main_kernel<D, CAUSAL, NPOLY, DQ>>(C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>(p.n_kv) * static_cast<unsigned>(p.BH);
+  const unsigned grid = static_cast<unsigned>(p.n_kv) * static_cast<unsigned>(p.BH / p.kv_group);
   kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(p);
   return cudaGetLastError();
 }

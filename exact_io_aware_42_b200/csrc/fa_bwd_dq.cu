@@ -91,6 +91,7 @@ __global__ void __launch_bounds__(320, 1) bwd_dq_kernel(const __grid_constant__ 
   const int bh = blockIdx.x / p.n_q;
   const int i = CAUSAL ? p.n_q - 1 - static_cast<int>(blockIdx.x % p.n_q) : static_cast<int>(blockIdx.x % p.n_q);
   const int n_j = CAUSAL ? i + 1 : p.n_kv;
+  const int kvh = bh / p.kv_group;   // grouped K/V heads: see the forward kernel
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QDO), 1);
@@ -142,12 +143,12 @@ __global__ void __launch_bounds__(320, 1) bwd_dq_kernel(const __grid_constant__ 
         if (!(ok = mbar_wait(bar(B_KE(sk)), ((j / NK) & 1) ^ 1, ab, kSiteDProd))) break;
         mbar_arrive_expect_tx(bar(B_KF(sk)), C::kTileBytes);
         for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_3d(kAddr(sk) + pn * C::kPanelBytes, &p.tm_k, bar(B_KF(sk)), pn * 64, j * 128, bh);
+          tma_load_3d(kAddr(sk) + pn * C::kPanelBytes, &p.tm_k, bar(B_KF(sk)), pn * 64, j * 128, kvh);
         ++nk;
         if (!(ok = mbar_wait(bar(B_VE(sv)), ((j / NV) & 1) ^ 1, ab, kSiteDProd))) break;
         mbar_arrive_expect_tx(bar(B_VF(sv)), C::kTileBytes);
         for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_3d(vAddr(sv) + pn * C::kPanelBytes, &p.tm_v, bar(B_VF(sv)), pn * 64, j * 128, bh);
+          tma_load_3d(vAddr(sv) + pn * C::kPanelBytes, &p.tm_v, bar(B_VF(sv)), pn * 64, j * 128, kvh);
         ++nv;
       }
       if (*abort_flag) {   // let the copies in flight land before the CTA leaves

@@ -119,6 +119,9 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
   // few heads whose K and V stay in L2.  Both orders measured on B200.
   const int bh = CAUSAL ? blockIdx.x % p.BH : blockIdx.x / p.n_pairs;
   const int pair = CAUSAL ? p.n_pairs - 1 - blockIdx.x / p.BH : blockIdx.x % p.n_pairs;
+  // Grouped K/V heads: query head h of batch b reads K/V head b * H_kv + h / G,
+  // which in the flattened [B * H] index is bh / G.
+  const int kvh = bh / p.kv_group;
   const int qt0 = 2 * pair;
   int n_t[2];
 #pragma unroll
@@ -174,7 +177,7 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
           const CUtensorMap* m = (w == 0) ? &p.tm_k : &p.tm_v;
           for (int pn = 0; pn < C::kPanels; ++pn)
             tma_load_3d(sbase + C::kOffRing + s * C::kTileBytes + pn * C::kPanelBytes, m,
-                        bar(bar_full<NS>(s)), pn * C::kPanelElems, j * kBlockN, bh);
+                        bar(bar_full<NS>(s)), pn * C::kPanelElems, j * kBlockN, kvh);
           ++seq;
         }
       }
@@ -287,7 +290,8 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
     // stored as E4M3 times 256 * s_v(j) / max_j s_v(j), which folds V's block
     // scale into P (p <= 1 because FP8 rescales on every max increase), and O
     // is multiplied back by max s_v / 256 at the end.
-    const size_t sc_base = static_cast<size_t>(bh) * p.n_kv;
+    const size_t sc_base = static_cast<size_t>(bh) * p.n_kv;      // Q's block scales
+    const size_t kv_base = static_cast<size_t>(kvh) * p.n_kv;     // K's and V's
     float c_q = p.scale_log2;
     float v_max = 1.f;
     float sk_next = 1.f, sv_next = 1.f;
@@ -296,15 +300,15 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
       // max over this head's V block scales: strided over the warpgroup's
       // 128 threads, then a shuffle and a shared-memory reduction
       float vm = 0.f;
-      for (int jj = r; jj < p.n_kv; jj += 128) vm = fmaxf(vm, p.sv[sc_base + jj]);
+      for (int jj = r; jj < p.n_kv; jj += 128) vm = fmaxf(vm, p.sv[kv_base + jj]);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, off));
       float* red = reinterpret_cast<float*>(smem + C::kOffMisc + 8) + 4 * t;   // 4 floats per tile
       if (lane == 0) red[warp & 3] = vm;
       named_bar_sync(1 + t, 128);
       v_max = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-      sk_next = p.sk[sc_base];
-      sv_next = p.sv[sc_base];
+      sk_next = p.sk[kv_base];
+      sv_next = p.sv[kv_base];
     }
     constexpr float kTau = FP8 ? 0.f : kRescaleTau;
     float m_use = -INFINITY;
@@ -319,8 +323,8 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
       const float sv_j = sv_next;
       if constexpr (FP8) {             // next tile's scales, loaded while this one is processed
         if (j + 1 < n) {
-          sk_next = p.sk[sc_base + j + 1];
-          sv_next = p.sv[sc_base + j + 1];
+          sk_next = p.sk[kv_base + j + 1];
+          sv_next = p.sv[kv_base + j + 1];
         }
       }
       const bool masked = (CAUSAL && j == qi) || ((j + 1) * kBlockN > p.N);

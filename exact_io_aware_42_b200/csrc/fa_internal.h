@@ -40,6 +40,7 @@ struct FwdParams {
   int BH;
   int n_pairs;          // ceil(ceil(N/128) / 2): CTAs per (b, h)
   int n_kv;             // ceil(N / 128)
+  int kv_group;         // G = H / H_kv query heads per K/V head (1: no grouping)
   float scale_log2;     // scale * log2(e)
   float scale;
   int poly_pairs;       // of every 8 column pairs, how many use the FMA-pipe exp2
@@ -90,6 +91,7 @@ struct BwdParams {
   int BH;
   int n_kv;             // ceil(N / 128): key blocks = CTAs per (b, h)
   int n_q;              // ceil(N / 128): query blocks
+  int kv_group;         // G = H / H_kv query heads per K/V head (1: no grouping)
   float scale_log2;     // scale * log2(e)
   float scale;
   int poly_groups;      // of every 4 groups of 4 columns, how many use the FMA-pipe exp2

@@ -80,6 +80,21 @@ def make_qkv(B: int, H: int, N: int, d: int, seed: int, with_do: bool = False,
     return out
 
 
+def make_gqa(B: int, H: int, H_kv: int, N: int, d: int, seed: int, with_do: bool = False,
+             outliers: bool = False):
+    """CPU bf16 (q, k, v[, do]) with grouped K/V heads: q, do [B, H, N, d];
+    k, v [B, H_kv, N, d]."""
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    shapes = {"q": (B, H, N, d), "k": (B, H_kv, N, d), "v": (B, H_kv, N, d), "do": (B, H, N, d)}
+    names = ["q", "k", "v"] + (["do"] if with_do else [])
+    t = {n: torch.randn(shapes[n], dtype=torch.float32, generator=g) for n in names}
+    if outliers:
+        for n in ("q", "k", "v"):
+            mask = torch.rand(shapes[n], generator=g) < 1e-3
+            t[n] = torch.where(mask, t[n] * 20.0, t[n])
+    return tuple(t[n].to(torch.bfloat16) for n in names)
+
+
 def make_workload(w: Workload):
     return make_qkv(w.B, w.H, w.N, w.d, w.seed, with_do=w.backward, outliers=w.fp8)
 

@@ -174,6 +174,35 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float
                      int d, float scale, int causal, void* stream);
 
 /*
+ * Grouped K/V heads (GQA; MQA when H_kv = 1).  The librarian page lists
+ * GQA/MQA as natively supported ("Cases where FlashAttention does not
+ * help"); the pages give no formula, so the reading here is the usual one:
+ * query head h of batch b attends with K/V head h / G of the same batch,
+ * G = H / H_kv.
+ *  k, v (k8, v8)   : [B, H_kv, N, d]; q, o, dout, dq : [B, H, N, d].
+ *  sk, sv           : [B, H_kv, ceil(N / 128)] block scales (FP8).
+ *  dk, dv           : [B, H_kv, N, d]: the sum over the group's G query
+ *                     heads of each head's gradient.
+ *  H_kv             : 1 <= H_kv, H a multiple of H_kv, else
+ *                     FA_ERR_INVALID_ARG.
+ * H_kv = H is exactly fa_fwd / fa_bwd / fa_bwd_deterministic / fa_fwd_fp8.
+ * fa_bwd_gqa takes the workspace of fa_bwd_workspace_size(B, H, N, d)
+ * (deterministic = 0) or fa_bwd_deterministic_workspace_size(B, H, N, d)
+ * (deterministic != 0), sized by the query heads.  In the backward one
+ * thread block per (K/V head, key block) visits the query blocks of all G
+ * query heads in turn, so dK and dV are summed on chip, in a fixed order.
+ */
+fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                     int H_kv, int N, int d, float scale, int causal, void* stream);
+fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                     const float* lse, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N,
+                     int d, float scale, int causal, int deterministic, void* workspace,
+                     size_t workspace_bytes, void* stream);
+fa_status fa_fwd_fp8_gqa(const void* q8, const void* k8, const void* v8, const float* sq,
+                         const float* sk, const float* sv, void* o, float* lse, int B, int H,
+                         int H_kv, int N, int d, float scale, int causal, void* stream);
+
+/*
  * Device status word of the current device: FA_OK, or the first in-kernel
  * failure (FA_ERR_PIPELINE_TIMEOUT, with the failing wait's site in bits
  * 8..15) since the last fa_clear_status().  Synchronises with the device

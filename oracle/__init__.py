@@ -17,7 +17,7 @@ Sources are cited by page title and section:
 Modules:
 
 * ``attention_ref``  -- forward (O, L), backward (dQ, dK, dV), the online
-  softmax recurrence.  Every function is pinned by ``tests/test_oracle_*.py``.
+  softmax recurrence, and grouped K/V heads (GQA / MQA).  Every function is pinned by ``tests/test_oracle_*.py``.
 * ``fp8_ref``        -- Sylvester Hadamard rotation, per-128-row block scale,
   a table-driven E4M3 (OCP e4m3fn) encoder/decoder.  Pinned likewise.
 """
@@ -25,6 +25,8 @@ from .attention_ref import (  # noqa: F401
     attn_fwd_ref,
     attn_fwd_rows_ref,
     attn_bwd_ref,
+    attn_fwd_gqa_ref,
+    attn_bwd_gqa_ref,
     online_softmax_ref,
     attn_fwd_online_ref,
     softmax_ref,

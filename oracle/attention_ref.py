@@ -242,3 +242,60 @@ def attn_fwd_online_ref(q, k, v, scale: float, causal: bool, block_sizes: Sequen
         o[i] = acc / ell
         lse[i] = m + np.log(ell)
     return o, lse
+
+
+def attn_fwd_gqa_ref(q, k, v, scale: float, causal: bool):
+    """Attention with grouped K/V heads, fp64.  q: [B, H, N, d]; k, v: [B, H_kv, N, d].
+
+    The librarian page lists GQA/MQA among the variants FlashAttention
+    supports ("Cases where FlashAttention does not help") without a formula;
+    the reading used: query head h of batch b uses K/V head h // G, G = H / H_kv.
+    Each query head is then plain attention (``attn_fwd_ref``'s definition).
+    Returns (O [B, H, N, d], L [B, H, N]).
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, H, N, d = q.shape
+    h_kv = k.shape[1]
+    if H % h_kv:
+        raise ValueError("H must be a multiple of H_kv")
+    g = H // h_kv
+    o = np.zeros((B, H, N, v.shape[-1]))
+    lse = np.zeros((B, H, N))
+    for b in range(B):
+        for h in range(H):
+            kk, vv = k[b, h // g], v[b, h // g]
+            s = scores_ref(q[b, h], kk, scale, causal)
+            m = np.max(s, axis=1)
+            e = np.exp(s - m[:, None])
+            ell = np.sum(e, axis=1)
+            o[b, h] = (e / ell[:, None]) @ vv
+            lse[b, h] = m + np.log(ell)
+    return o, lse
+
+
+def attn_bwd_gqa_ref(q, k, v, do, scale: float, causal: bool):
+    """Gradients of sum(O * dO) for grouped K/V heads, fp64.
+
+    dQ of head h is that of plain attention with K/V head h // G; since a
+    K/V head feeds G query heads, its dK and dV are the sums of the G heads'
+    gradients (the chain rule over the shared input).  Returns (dq, dk, dv)
+    with dk, dv of shape [B, H_kv, N, d].
+    """
+    q, k, v, do = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(do)
+    B, H, N, d = q.shape
+    h_kv = k.shape[1]
+    g = H // h_kv
+    _, lse = attn_fwd_gqa_ref(q, k, v, scale, causal)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for h in range(H):
+            kk, vv = k[b, h // g], v[b, h // g]
+            p = np.exp(scores_ref(q[b, h], kk, scale, causal) - lse[b, h][:, None])
+            dp = do[b, h] @ vv.T
+            ds = p * (dp - np.sum(p * dp, axis=1)[:, None])
+            dq[b, h] = float(scale) * (ds @ kk)
+            dk[b, h // g] += float(scale) * (ds.T @ q[b, h])
+            dv[b, h // g] += p.T @ do[b, h]
+    return dq, dk, dv
