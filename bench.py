@@ -21,6 +21,10 @@ weak scaling.
 
 ``--impl reference`` times the fp64 CPU oracle (the only other code this
 script may run) on a bounded sample of the same workload on the host cores.
+
+``--bwd deterministic`` times the reproducible backward (dK, dV kernel plus
+the query-block-major dQ kernel) in place of the atomic one; the ``gqa_`` /
+``mqa_`` workloads have fewer K/V heads than query heads (grouped K/V).
 """
 from __future__ import annotations
 
@@ -53,8 +57,13 @@ def workloads():
             name = w.name.replace("attn_fwd_", "attn_").replace("attn_fp8_", "attn_fp8_") + \
                 ("_causal" if c else "_noncausal")
             out[name] = dict(B=w.B, H=w.H, N=w.N, d=w.d, causal=c, seed=w.seed)
+    # grouped K/V heads: FLOPs as for H query heads, K/V (and dK, dV) of H_kv heads
+    out["gqa_B4_H32_Hkv8_N4096_d128_causal"] = dict(B=4, H=32, H_kv=8, N=4096, d=128, causal=True, seed=5)
+    out["gqa_B4_H32_Hkv8_N4096_d128_noncausal"] = dict(B=4, H=32, H_kv=8, N=4096, d=128, causal=False, seed=5)
+    out["mqa_B4_H16_Hkv1_N4096_d128_causal"] = dict(B=4, H=16, H_kv=1, N=4096, d=128, causal=True, seed=6)
     for name, w in out.items():
         w["name"] = name
+        w.setdefault("H_kv", w["H"])
     return out
 
 
@@ -66,13 +75,17 @@ def fwd_flops(B, H, N, d, causal):
     return f / 2 if causal else f
 
 
-def fwd_bytes(B, H, N, d):
+def fwd_bytes(B, H, N, d, H_kv=None):
     """Algorithmic bytes of the forward: Q, K, V read once, O written, LSE written."""
-    return 3 * B * H * N * d * 2 + B * H * N * d * 2 + B * H * N * 4
+    H_kv = H if H_kv is None else H_kv
+    return (B * H + 2 * B * H_kv) * N * d * 2 + B * H * N * d * 2 + B * H * N * 4
 
 
-def bwd_bytes(B, H, N, d):
-    return 5 * B * H * N * d * 2 + 2 * B * H * N * 4 + 3 * B * H * N * d * 2
+def bwd_bytes(B, H, N, d, H_kv=None):
+    """Q, O, dO read and dQ written (query heads); K, V read and dK, dV
+    written (K/V heads); L and D read."""
+    H_kv = H if H_kv is None else H_kv
+    return (3 * B * H + 2 * B * H_kv) * N * d * 2 + 2 * B * H * N * 4 + (B * H + 2 * B * H_kv) * N * d * 2
 
 
 def measured_peaks():
@@ -166,12 +179,13 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs):
+def build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs, deterministic=False):
     """The hot path as a list of (stage name, callable, FLOPs, kernel launches)."""
     state = {}
 
-    ws = torch.empty(fa.bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=q.device)
-    bufs = {n: torch.empty_like(q) for n in ("o", "dq", "dk", "dv")}
+    ws = torch.empty(fa.bwd_workspace_size(B, H, N, d, deterministic), dtype=torch.uint8, device=q.device)
+    bufs = {n: torch.empty_like(q) for n in ("o", "dq")}
+    bufs.update({n: torch.empty_like(k) for n in ("dk", "dv")})
     bufs["lse"] = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
 
     def s_fwd():
@@ -180,11 +194,12 @@ def build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs):
     def s_bwd():
         state["dq"], state["dk"], state["dv"] = fa.bwd(
             q, k, v, bufs["o"], do, bufs["lse"], causal=causal, workspace=ws,
-            dq=bufs["dq"], dk=bufs["dk"], dv=bufs["dv"])
+            dq=bufs["dq"], dk=bufs["dk"], dv=bufs["dv"], deterministic=deterministic)
 
-    q8 = {n: torch.empty(q.shape, dtype=torch.uint8, device=q.device) for n in ("q", "k", "v")}
-    sc8 = {n: torch.empty((B, H, fa.n_blocks(N)), dtype=torch.float32, device=q.device)
-           for n in ("q", "k", "v")}
+    src = {"q": q, "k": k, "v": v}
+    q8 = {n: torch.empty(t.shape, dtype=torch.uint8, device=q.device) for n, t in src.items()}
+    sc8 = {n: torch.empty((B, t.shape[1], fa.n_blocks(N)), dtype=torch.float32, device=q.device)
+           for n, t in src.items()}
     o8 = torch.empty_like(q)
     lse8 = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
 
@@ -198,6 +213,7 @@ def build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs):
                                                       sc8["v"], causal=causal, out=o8, lse=lse8)
 
     f = fwd_flops(B, H, N, d, causal)
+    # backward launches: preprocess, main, and postprocess (atomic) or dQ (deterministic)
     stages = [("fwd_bf16", s_fwd, f, 1), ("bwd_bf16", s_bwd, 2.5 * f, 3)]
     if d == 128:   # the FP8 forward exists for d = 128 only
         stages += [("quant_fp8", s_quant, 0.0, 3), ("fwd_fp8", s_fwd8, f, 1)]
@@ -252,25 +268,28 @@ def oracle_sample(budget_s: float, B, H, N, d, causal, with_bwd: bool):
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
     except Exception:  # noqa: BLE001
         cores = os.cpu_count()
-    key = (B, H, N, d)
+    H_kv = WORKLOAD.get("H_kv", H)
+    key = (B, H, H_kv, N, d)
     if key not in _ORACLE_INPUTS:
-        _ORACLE_INPUTS[key] = inputs.make_qkv(B, H, N, d, WORKLOAD["seed"], with_do=True)
+        _ORACLE_INPUTS[key] = inputs.make_gqa(B, H, H_kv, N, d, WORKLOAD["seed"], with_do=True)
     q, k, v, do = _ORACLE_INPUTS[key]
     sc = 1.0 / math.sqrt(d)
     flops, heads, t0 = 0.0, 0, time.perf_counter()
     for idx in range(B * H):
         b, h = divmod(idx, H)
         sl = (slice(b, b + 1), slice(h, h + 1))
-        oracle.attn_fwd_ref(q[sl], k[sl], v[sl], sc, causal)
+        kh = h // (H // H_kv)           # the K/V head of query head h
+        kl = (slice(b, b + 1), slice(kh, kh + 1))
+        oracle.attn_fwd_ref(q[sl], k[kl], v[kl], sc, causal)
         flops += fwd_flops(1, 1, N, d, causal)
         if with_bwd:
-            oracle.attn_bwd_ref(q[sl], k[sl], v[sl], do[sl], sc, causal)
+            oracle.attn_bwd_ref(q[sl], k[kl], v[kl], do[sl], sc, causal)
             flops += 2.5 * fwd_flops(1, 1, N, d, causal)
             # FP8 rows: block quantisation (Q, K rotated; V) and attention on the
             # dequantised values
             sg = inputs.signs(d).numpy()
-            deq = [oracle.dequant_fp8_ref(*oracle.quant_fp8_ref(x[sl].double().numpy(), rot, sg))
-                   for x, rot in ((q, True), (k, True), (v, False))]
+            deq = [oracle.dequant_fp8_ref(*oracle.quant_fp8_ref(x[s_].double().numpy(), rot, sg))
+                   for x, s_, rot in ((q, sl, True), (k, kl, True), (v, kl, False))]
             oracle.attn_fwd_ref(deq[0], deq[1], deq[2], sc, causal)
             flops += fwd_flops(1, 1, N, d, causal)
         heads += 1
@@ -309,15 +328,18 @@ def run_reference(args):
 
 METRIC = "attention fwd/bwd TFLOPS (BF16 causal+non-causal) and % of B200 tensor peak"
 STAGES_WITH_BWD = True
+BWD_MODE = "atomic"   # set in main()
 
 
 def config_block():
     w = WORKLOAD
-    return {"workload": w["name"], "B": w["B"], "H": w["H"], "N": w["N"], "d": w["d"],
+    in_bytes = 2 * (w["H"] + w["H_kv"]) * w["B"] * w["N"] * w["d"] * 2
+    return {"workload": w["name"], "B": w["B"], "H": w["H"], "H_kv": w["H_kv"], "N": w["N"], "d": w["d"],
+            "bwd": BWD_MODE,
             "causal": w["causal"], "global_batch": w["B"], "seq_len": w["N"],
             "parallelism": "independent replicas per GPU (heads), no collective",
-            "l2": (f"inputs 4 x {w['B'] * w['H'] * w['N'] * w['d'] * 2 / 2**20:.0f} MiB > 126 MB L2, no flush"
-                   if 4 * w["B"] * w["H"] * w["N"] * w["d"] * 2 > 126e6 else
+            "l2": (f"inputs (Q, K, V, dO) {in_bytes / 2**20:.0f} MiB > 126 MB L2, no flush"
+                   if in_bytes > 126e6 else
                    "inputs smaller than L2: timed warm in L2 (latency-bound workload)"),
             "step": "fwd_bf16 + bwd_bf16" + (" + quant_fp8 (Q, K rotated; V) + fwd_fp8" if w["d"] == 128 else ""),
             "fp8": "quantisation and forward in E4M3 (kind::f8f6f4), counted at forward FLOPs"}
@@ -340,11 +362,12 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
     w = WORKLOAD
-    B, H, N, d, causal = w["B"], w["H"], w["N"], w["d"], w["causal"]
-    hq, hk, hv, hdo = inputs.make_qkv(B, H, N, d, w["seed"] + rank, with_do=True)
+    B, H, N, d, causal, H_kv = w["B"], w["H"], w["N"], w["d"], w["causal"], w["H_kv"]
+    hq, hk, hv, hdo = inputs.make_gqa(B, H, H_kv, N, d, w["seed"] + rank, with_do=True)
     signs = inputs.signs(d).to(dev)
     q, k, v, do = (t.to(dev) for t in (hq, hk, hv, hdo))
-    stages, state = build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs)
+    stages, state = build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs,
+                               deterministic=BWD_MODE == "deterministic")
     step_flops = sum(s[2] for s in stages)
     launches_per_step = sum(s[3] for s in stages)
 
@@ -418,11 +441,14 @@ def run_ours(args):
                         "nominal_2250": value / world / 2250.0},
         "stages": {s[0]: {"ms": per_stage[i], "tflops": s[2] / (per_stage[i] * 1e-3) / 1e12}
                    for i, s in enumerate(stages)},
-        "roofline": dict(roof("bwd_bf16", f"bwd_main_kernel<{d}, {'causal' if causal else 'non-causal'}> "
-                              "(+ pre/post kernels in the timed call)", bwd_bytes(B, H, N, d)),
-                         traffic=profiled_traffic("bwd") if w["name"] == DEFAULT_WORKLOAD else None),
+        "roofline": dict(roof("bwd_bf16", (f"bwd_main_kernel<{d}, {'causal' if causal else 'non-causal'}> "
+                              "(+ pre/post kernels in the timed call)") if BWD_MODE == "atomic" else
+                              (f"bwd_main_kernel<{d}, {'causal' if causal else 'non-causal'}, no dQ> + "
+                               "bwd_dq_kernel (+ preprocess) in the timed call"), bwd_bytes(B, H, N, d, H_kv)),
+                         traffic=profiled_traffic("bwd") if (w["name"] == DEFAULT_WORKLOAD and BWD_MODE == "atomic")
+                         else None),
         "roofline_fwd": dict(roof("fwd_bf16", f"fwd_kernel<{d}, {'causal' if causal else 'non-causal'}, bf16>",
-                                  fwd_bytes(B, H, N, d)),
+                                  fwd_bytes(B, H, N, d, H_kv)),
                              traffic=profiled_traffic("fwd") if w["name"] == DEFAULT_WORKLOAD else None),
         "e2e": {"value": whole_job_tflops(world, step_flops, e2e_ms), "unit": "TFLOPS",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
@@ -451,9 +477,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads()),
                     help="configuration to time (default: the one the headline metric is quoted on)")
+    ap.add_argument("--bwd", choices=["atomic", "deterministic"], default="atomic",
+                    help="backward variant timed in the step (default: atomic dQ accumulation)")
     args = ap.parse_args()
-    global WORKLOAD
+    global WORKLOAD, BWD_MODE
     WORKLOAD = workloads()[args.workload]
+    BWD_MODE = args.bwd
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
