@@ -61,18 +61,33 @@ def workloads():
     out["gqa_B4_H32_Hkv8_N4096_d128_causal"] = dict(B=4, H=32, H_kv=8, N=4096, d=128, causal=True, seed=5)
     out["gqa_B4_H32_Hkv8_N4096_d128_noncausal"] = dict(B=4, H=32, H_kv=8, N=4096, d=128, causal=False, seed=5)
     out["mqa_B4_H16_Hkv1_N4096_d128_causal"] = dict(B=4, H=16, H_kv=1, N=4096, d=128, causal=True, seed=6)
+    # causal sliding window of 1024 keys at N = 16384: FLOPs counted over the visible pairs only
+    out["window1024_B1_H16_N16384_d128"] = dict(B=1, H=16, N=16384, d=128, causal=True, seed=7, window=1024)
     for name, w in out.items():
         w["name"] = name
         w.setdefault("H_kv", w["H"])
+        w.setdefault("window", None)
     return out
 
 
 WORKLOAD = None   # set in main()
 
 
-def fwd_flops(B, H, N, d, causal):
-    f = 4.0 * B * H * N * N * d
-    return f / 2 if causal else f
+def visible_pairs(N, causal, window=None):
+    """(query, key) pairs the mask leaves visible."""
+    if not causal:
+        return N * N
+    if window is None or window >= N - 1:
+        return N * (N + 1) / 2
+    w = window   # row i sees min(i, w) + 1 keys
+    return (w + 1) * (w + 2) / 2 - (w + 1) + (N - w) * (w + 1) if N > w else N * (N + 1) / 2
+
+
+def fwd_flops(B, H, N, d, causal, window=None):
+    """4 B H d x visible pairs (x N^2 / 2 for plain causal, the usual count)."""
+    if causal and window is None:
+        return 4.0 * B * H * N * N * d / 2
+    return 4.0 * B * H * d * visible_pairs(N, causal, window)
 
 
 def fwd_bytes(B, H, N, d, H_kv=None):
@@ -179,7 +194,7 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs, deterministic=False):
+def build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs, deterministic=False, window=None):
     """The hot path as a list of (stage name, callable, FLOPs, kernel launches)."""
     state = {}
 
@@ -189,12 +204,13 @@ def build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs, deterministic=
     bufs["lse"] = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
 
     def s_fwd():
-        state["o"], state["lse"] = fa.fwd(q, k, v, causal=causal, out=bufs["o"], lse=bufs["lse"])
+        state["o"], state["lse"] = fa.fwd(q, k, v, causal=causal, out=bufs["o"], lse=bufs["lse"],
+                                          window=window)
 
     def s_bwd():
         state["dq"], state["dk"], state["dv"] = fa.bwd(
             q, k, v, bufs["o"], do, bufs["lse"], causal=causal, workspace=ws,
-            dq=bufs["dq"], dk=bufs["dk"], dv=bufs["dv"], deterministic=deterministic)
+            dq=bufs["dq"], dk=bufs["dk"], dv=bufs["dv"], deterministic=deterministic, window=window)
 
     src = {"q": q, "k": k, "v": v}
     q8 = {n: torch.empty(t.shape, dtype=torch.uint8, device=q.device) for n, t in src.items()}
@@ -210,9 +226,10 @@ def build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs, deterministic=
 
     def s_fwd8():
         state["o_fp8"], state["lse_fp8"] = fa.fwd_fp8(q8["q"], q8["k"], q8["v"], sc8["q"], sc8["k"],
-                                                      sc8["v"], causal=causal, out=o8, lse=lse8)
+                                                      sc8["v"], causal=causal, out=o8, lse=lse8,
+                                                      window=window)
 
-    f = fwd_flops(B, H, N, d, causal)
+    f = fwd_flops(B, H, N, d, causal, window)
     # backward launches: preprocess, main, and postprocess (atomic) or dQ (deterministic)
     stages = [("fwd_bf16", s_fwd, f, 1), ("bwd_bf16", s_bwd, 2.5 * f, 3)]
     if d == 128:   # the FP8 forward exists for d = 128 only
@@ -280,18 +297,19 @@ def oracle_sample(budget_s: float, B, H, N, d, causal, with_bwd: bool):
         sl = (slice(b, b + 1), slice(h, h + 1))
         kh = h // (H // H_kv)           # the K/V head of query head h
         kl = (slice(b, b + 1), slice(kh, kh + 1))
-        oracle.attn_fwd_ref(q[sl], k[kl], v[kl], sc, causal)
-        flops += fwd_flops(1, 1, N, d, causal)
+        win = WORKLOAD.get("window")
+        oracle.attn_fwd_gqa_ref(q[sl], k[kl], v[kl], sc, causal, window=win)
+        flops += fwd_flops(1, 1, N, d, causal, win)
         if with_bwd:
-            oracle.attn_bwd_ref(q[sl], k[kl], v[kl], do[sl], sc, causal)
-            flops += 2.5 * fwd_flops(1, 1, N, d, causal)
+            oracle.attn_bwd_gqa_ref(q[sl], k[kl], v[kl], do[sl], sc, causal, window=win)
+            flops += 2.5 * fwd_flops(1, 1, N, d, causal, win)
             # FP8 rows: block quantisation (Q, K rotated; V) and attention on the
             # dequantised values
             sg = inputs.signs(d).numpy()
             deq = [oracle.dequant_fp8_ref(*oracle.quant_fp8_ref(x[s_].double().numpy(), rot, sg))
                    for x, s_, rot in ((q, sl, True), (k, kl, True), (v, kl, False))]
-            oracle.attn_fwd_ref(deq[0], deq[1], deq[2], sc, causal)
-            flops += fwd_flops(1, 1, N, d, causal)
+            oracle.attn_fwd_gqa_ref(deq[0], deq[1], deq[2], sc, causal, window=win)
+            flops += fwd_flops(1, 1, N, d, causal, win)
         heads += 1
         if time.perf_counter() - t0 >= budget_s:
             break
@@ -335,7 +353,7 @@ def config_block():
     w = WORKLOAD
     in_bytes = 2 * (w["H"] + w["H_kv"]) * w["B"] * w["N"] * w["d"] * 2
     return {"workload": w["name"], "B": w["B"], "H": w["H"], "H_kv": w["H_kv"], "N": w["N"], "d": w["d"],
-            "bwd": BWD_MODE,
+            "bwd": BWD_MODE, "window": w["window"],
             "causal": w["causal"], "global_batch": w["B"], "seq_len": w["N"],
             "parallelism": "independent replicas per GPU (heads), no collective",
             "l2": (f"inputs (Q, K, V, dO) {in_bytes / 2**20:.0f} MiB > 126 MB L2, no flush"
@@ -367,7 +385,7 @@ def run_ours(args):
     signs = inputs.signs(d).to(dev)
     q, k, v, do = (t.to(dev) for t in (hq, hk, hv, hdo))
     stages, state = build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs,
-                               deterministic=BWD_MODE == "deterministic")
+                               deterministic=BWD_MODE == "deterministic", window=w["window"])
     step_flops = sum(s[2] for s in stages)
     launches_per_step = sum(s[3] for s in stages)
 

@@ -133,17 +133,26 @@ fa_status check_kv_heads(int H, int H_kv) {
   return FA_OK;
 }
 
+// Sliding window: -1 (none) or >= 0 with causal; returns the kernels' value.
+fa_status check_window(int window_left, int causal, int* window) {
+  if (window_left < -1 || (window_left >= 0 && !causal)) return FA_ERR_INVALID_ARG;
+  *window = window_left < 0 ? kNoWindow : window_left;
+  return FA_OK;
+}
+
 }  // namespace
 }  // namespace fa
 
 using namespace fa;
 
-extern "C" fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
-                                int B, int H, int H_kv, int N, int d, float scale, int causal,
-                                void* stream) {
+extern "C" fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                               int B, int H, int H_kv, int N, int d, float scale, int causal,
+                               int window_left, void* stream) {
   fa_status st = check_shape(B, H, N, d, scale);
   if (st != FA_OK) return st;
   if (H > 0 && (st = check_kv_heads(H, H_kv)) != FA_OK) return st;
+  int window = kNoWindow;
+  if ((st = check_window(window_left, causal, &window)) != FA_OK) return st;
   if (static_cast<long long>(B) * H * N == 0) return FA_OK;
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
@@ -167,6 +176,7 @@ extern "C" fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, voi
   p.N = N;
   p.BH = BH;
   p.kv_group = H / H_kv;
+  p.window = window;
   p.n_kv = (N + kBlockN - 1) / kBlockN;
   p.n_pairs = ((N + kBlockM - 1) / kBlockM + 1) / 2;
   p.scale = scale;
@@ -182,7 +192,7 @@ extern "C" fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, voi
 
 extern "C" fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                             int B, int H, int N, int d, float scale, int causal, void* stream) {
-  return fa_fwd_gqa(q, k, v, o, lse, B, H, H, N, d, scale, causal, stream);
+  return fa_fwd_ex(q, k, v, o, lse, B, H, H, N, d, scale, causal, -1, stream);
 }
 
 extern "C" size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
@@ -205,11 +215,13 @@ namespace {
 // deterministic one runs the main kernel without dQ and the dQ kernel.
 fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const void* dout,
                      const float* lse, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N,
-                     int d, float scale, int causal, void* workspace, size_t workspace_bytes,
-                     void* stream, bool deterministic) {
+                     int d, float scale, int causal, int window_left, void* workspace,
+                     size_t workspace_bytes, void* stream, bool deterministic) {
   fa_status st = check_shape(B, H, N, d, scale);
   if (st != FA_OK) return st;
   if (H > 0 && (st = check_kv_heads(H, H_kv)) != FA_OK) return st;
+  int window = kNoWindow;
+  if ((st = check_window(window_left, causal, &window)) != FA_OK) return st;
   if (static_cast<long long>(B) * H * N == 0) return FA_OK;
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
@@ -251,6 +263,7 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   p.n_kv = (N + 127) / 128;
   p.n_q = (N + 127) / 128;
   p.kv_group = H / H_kv;
+  p.window = window;
   p.scale = scale;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.poly_groups = bwd_poly_groups();
@@ -277,7 +290,7 @@ extern "C" fa_status fa_bwd(const void* q, const void* k, const void* v, const v
                             const void* dout, const float* lse, void* dq, void* dk, void* dv,
                             int B, int H, int N, int d, float scale, int causal, void* workspace,
                             size_t workspace_bytes, void* stream) {
-  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, H, N, d, scale, causal, workspace,
+  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, H, N, d, scale, causal, -1, workspace,
                     workspace_bytes, stream, false);
 }
 
@@ -286,17 +299,17 @@ extern "C" fa_status fa_bwd_deterministic(const void* q, const void* k, const vo
                                           void* dv, int B, int H, int N, int d, float scale,
                                           int causal, void* workspace, size_t workspace_bytes,
                                           void* stream) {
-  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, H, N, d, scale, causal, workspace,
+  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, H, N, d, scale, causal, -1, workspace,
                     workspace_bytes, stream, true);
 }
 
-extern "C" fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
-                                const void* dout, const float* lse, void* dq, void* dk, void* dv,
-                                int B, int H, int H_kv, int N, int d, float scale, int causal,
-                                int deterministic, void* workspace, size_t workspace_bytes,
-                                void* stream) {
-  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, H_kv, N, d, scale, causal, workspace,
-                    workspace_bytes, stream, deterministic != 0);
+extern "C" fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* o,
+                               const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                               int B, int H, int H_kv, int N, int d, float scale, int causal,
+                               int window_left, int deterministic, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, H_kv, N, d, scale, causal, window_left,
+                    workspace, workspace_bytes, stream, deterministic != 0);
 }
 
 extern "C" fa_status fa_quant_fp8(const void* x, void* x8, float* scales, int B, int H, int N,
@@ -336,13 +349,15 @@ extern "C" fa_status fa_quant_fp8(const void* x, void* x8, float* scales, int B,
   return FA_OK;
 }
 
-extern "C" fa_status fa_fwd_fp8_gqa(const void* q8, const void* k8, const void* v8, const float* sq,
-                                    const float* sk, const float* sv, void* o, float* lse, int B,
-                                    int H, int H_kv, int N, int d, float scale, int causal,
-                                    void* stream) {
+extern "C" fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v8, const float* sq,
+                                   const float* sk, const float* sv, void* o, float* lse, int B,
+                                   int H, int H_kv, int N, int d, float scale, int causal,
+                                   int window_left, void* stream) {
   fa_status st = check_shape(B, H, N, d, scale);
   if (st != FA_OK) return st;
   if (H > 0 && (st = check_kv_heads(H, H_kv)) != FA_OK) return st;
+  int window = kNoWindow;
+  if ((st = check_window(window_left, causal, &window)) != FA_OK) return st;
   if (d != 128) return FA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H * N == 0) return FA_OK;
   if (!q8 || !k8 || !v8 || !sq || !sk || !sv || !o || !lse) return FA_ERR_INVALID_ARG;
@@ -370,6 +385,7 @@ extern "C" fa_status fa_fwd_fp8_gqa(const void* q8, const void* k8, const void* 
   p.N = N;
   p.BH = BH;
   p.kv_group = H / H_kv;
+  p.window = window;
   p.n_kv = (N + kBlockN - 1) / kBlockN;
   p.n_pairs = ((N + kBlockM - 1) / kBlockM + 1) / 2;
   p.scale = scale;
@@ -385,7 +401,7 @@ extern "C" fa_status fa_fwd_fp8_gqa(const void* q8, const void* k8, const void* 
 extern "C" fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* sq,
                                 const float* sk, const float* sv, void* o, float* lse, int B, int H,
                                 int N, int d, float scale, int causal, void* stream) {
-  return fa_fwd_fp8_gqa(q8, k8, v8, sq, sk, sv, o, lse, B, H, H, N, d, scale, causal, stream);
+  return fa_fwd_fp8_ex(q8, k8, v8, sq, sk, sv, o, lse, B, H, H, N, d, scale, causal, -1, stream);
 }
 
 extern "C" fa_status fa_selftest_wait_timeout(void* stream) {

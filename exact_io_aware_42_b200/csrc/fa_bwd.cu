@@ -195,7 +195,9 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
   const int kvh = blockIdx.x / p.n_kv;
   const int j = blockIdx.x % p.n_kv;
   const int i0 = CAUSAL ? j : 0;
-  const int n_i = p.n_q - i0;               // query blocks per query head (>= 1)
+  // Sliding window (causal): the last query block that sees a key of block j.
+  const int i_last = CAUSAL ? min(p.n_q - 1, (j * 128 + 127 + p.window) / 128) : p.n_q - 1;
+  const int n_i = i_last - i0 + 1;          // query blocks per query head (>= 1)
   const int n_it = n_i * p.kv_group;
   auto q_block = [&](int idx) { return i0 + idx % n_i; };
   auto q_head = [&](int idx) { return kvh * p.kv_group + idx / n_i; };
@@ -389,7 +391,11 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
       const int i = q_block(idx);
       const float4* L4 = reinterpret_cast<const float4*>(smem + C::kOffL + (idx % NQ) * 512) + 16 * wg;
       const float4* D4 = reinterpret_cast<const float4*>(smem + C::kOffDl + (idx % ND) * 512) + 16 * wg;
-      const bool diag = CAUSAL && i == j;
+      // Visible query columns of this thread's key: c_lo <= column <= c_hi
+      // (column c is query i * 128 + c): after the key on the diagonal block,
+      // within the sliding window, and none at all for a key past N.
+      const int c_lo = (CAUSAL && i == j) ? r : 0;
+      const int c_hi = !key_ok ? -1 : (CAUSAL ? min(127, key + p.window - i * 128) : 127);
       const uint32_t tS = tmem + C::kColA + lane_off + col_half;
       const uint32_t tDP = tmem + C::kColB + lane_off + col_half;
       if (!(ok = mbar_wait_warp(bar(B_S), idx & 1, ab, kSiteBSmS))) break;
@@ -414,8 +420,8 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
           f2_unpack(p23, pv[2], pv[3]);
 #pragma unroll
           for (int t = 0; t < 4; ++t) {                  // query 64 wg + 4 c4 + t
-            const bool hidden = !key_ok || (diag && r > static_cast<int>(col_half) + 4 * c4 + t);
-            pv[t] = hidden ? 0.f : pv[t];                // key past N, or key after query
+            const int col = static_cast<int>(col_half) + 4 * c4 + t;
+            pv[t] = (col < c_lo || col > c_hi) ? 0.f : pv[t];
           }
           u[2 * c4] = pack_bf16x2(pv[0], pv[1]);
           u[2 * c4 + 1] = pack_bf16x2(pv[2], pv[3]);

@@ -90,7 +90,9 @@ __global__ void __launch_bounds__(320, 1) bwd_dq_kernel(const __grid_constant__ 
   // Head-major; within a head, causal query blocks with the most key blocks first.
   const int bh = blockIdx.x / p.n_q;
   const int i = CAUSAL ? p.n_q - 1 - static_cast<int>(blockIdx.x % p.n_q) : static_cast<int>(blockIdx.x % p.n_q);
-  const int n_j = CAUSAL ? i + 1 : p.n_kv;
+  // Sliding window (causal): key blocks wholly left of the window are skipped.
+  const int j_start = CAUSAL ? max(0, i * 128 - p.window) / 128 : 0;
+  const int n_j = (CAUSAL ? i + 1 : p.n_kv) - j_start;   // iterations; block = j_start + j
   const int kvh = bh / p.kv_group;   // grouped K/V heads: see the forward kernel
 
   if (threadIdx.x == 0) {
@@ -143,12 +145,12 @@ __global__ void __launch_bounds__(320, 1) bwd_dq_kernel(const __grid_constant__ 
         if (!(ok = mbar_wait(bar(B_KE(sk)), ((j / NK) & 1) ^ 1, ab, kSiteDProd))) break;
         mbar_arrive_expect_tx(bar(B_KF(sk)), C::kTileBytes);
         for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_3d(kAddr(sk) + pn * C::kPanelBytes, &p.tm_k, bar(B_KF(sk)), pn * 64, j * 128, kvh);
+          tma_load_3d(kAddr(sk) + pn * C::kPanelBytes, &p.tm_k, bar(B_KF(sk)), pn * 64, (j_start + j) * 128, kvh);
         ++nk;
         if (!(ok = mbar_wait(bar(B_VE(sv)), ((j / NV) & 1) ^ 1, ab, kSiteDProd))) break;
         mbar_arrive_expect_tx(bar(B_VF(sv)), C::kTileBytes);
         for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_3d(vAddr(sv) + pn * C::kPanelBytes, &p.tm_v, bar(B_VF(sv)), pn * 64, j * 128, kvh);
+          tma_load_3d(vAddr(sv) + pn * C::kPanelBytes, &p.tm_v, bar(B_VF(sv)), pn * 64, (j_start + j) * 128, kvh);
         ++nv;
       }
       if (*abort_flag) {   // let the copies in flight land before the CTA leaves
@@ -248,8 +250,10 @@ __global__ void __launch_bounds__(320, 1) bwd_dq_kernel(const __grid_constant__ 
       const int t = j & 1;
       const uint32_t tS = tmem + C::kColS + 128 * t + lane_off + 64 * wg;
       const uint32_t tDP = tmem + C::kColDP + lane_off + 64 * wg;
-      const int kbase = j * 128 + 64 * wg;
-      const bool edge = (CAUSAL && j == i) || kbase + 64 > p.N;   // warp-uniform
+      const int jb = j_start + j;
+      const int kbase = jb * 128 + 64 * wg;
+      // warp-uniform: a key past N, after the query (diagonal) or left of the window
+      const bool edge = (CAUSAL && (jb == i || kbase < i * 128 + 127 - p.window)) || kbase + 64 > p.N;
       if (!(ok = mbar_wait_warp(bar(B_S0 + t), (j >> 1) & 1, ab, kSiteDSmS))) break;
       tc_fence_after();
       uint32_t u[64];
@@ -267,7 +271,7 @@ __global__ void __launch_bounds__(320, 1) bwd_dq_kernel(const __grid_constant__ 
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const int key = kbase + c;
-          if (key >= p.N || (CAUSAL && key > q)) u[c] = 0u;
+          if (key >= p.N || (CAUSAL && (key > q || key < q - p.window))) u[c] = 0u;
         }
       }
       if (!(ok = mbar_wait_warp(bar(B_DP), j & 1, ab, kSiteDSmDP))) break;

@@ -123,9 +123,14 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
   // which in the flattened [B * H] index is bh / G.
   const int kvh = bh / p.kv_group;
   const int qt0 = 2 * pair;
+  // Sliding window (causal only): key j is visible to query i iff
+  // i - window <= j <= i.  Key blocks wholly left of tile 0's window are
+  // never loaded; both tiles start at the same block (tile 1's first block
+  // may then be fully masked for it, which the softmax handles).
+  const int j_start = CAUSAL ? max(0, qt0 * kBlockM - p.window) / kBlockN : 0;
   int n_t[2];
 #pragma unroll
-  for (int t = 0; t < 2; ++t) n_t[t] = CAUSAL ? min(qt0 + t + 1, p.n_kv) : p.n_kv;
+  for (int t = 0; t < 2; ++t) n_t[t] = (CAUSAL ? min(qt0 + t + 1, p.n_kv) : p.n_kv) - j_start;
   const int n_iter = n_t[1];
 
   if (threadIdx.x == 0) {
@@ -177,7 +182,7 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
           const CUtensorMap* m = (w == 0) ? &p.tm_k : &p.tm_v;
           for (int pn = 0; pn < C::kPanels; ++pn)
             tma_load_3d(sbase + C::kOffRing + s * C::kTileBytes + pn * C::kPanelBytes, m,
-                        bar(bar_full<NS>(s)), pn * C::kPanelElems, j * kBlockN, kvh);
+                        bar(bar_full<NS>(s)), pn * C::kPanelElems, (j_start + j) * kBlockN, kvh);
           ++seq;
         }
       }
@@ -307,14 +312,15 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
       if (lane == 0) red[warp & 3] = vm;
       named_bar_sync(1 + t, 128);
       v_max = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-      sk_next = p.sk[kv_base];
-      sv_next = p.sv[kv_base];
+      sk_next = p.sk[kv_base + j_start];
+      sv_next = p.sv[kv_base + j_start];
     }
     constexpr float kTau = FP8 ? 0.f : kRescaleTau;
     float m_use = -INFINITY;
     float l = 0.f;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
+      const int jb = j_start + j;      // key block; j counts this tile's iterations
       if (!(ok = mbar_wait_warp(bar(bar_s<NS>(t)), j & 1, ab, kSiteSmS))) break;
       tc_fence_after();
       uint32_t u[128];
@@ -323,18 +329,21 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
       const float sv_j = sv_next;
       if constexpr (FP8) {             // next tile's scales, loaded while this one is processed
         if (j + 1 < n) {
-          sk_next = p.sk[kv_base + j + 1];
-          sv_next = p.sv[kv_base + j + 1];
+          sk_next = p.sk[kv_base + jb + 1];
+          sv_next = p.sv[kv_base + jb + 1];
         }
       }
-      const bool masked = (CAUSAL && j == qi) || ((j + 1) * kBlockN > p.N);
+      const bool masked = (CAUSAL && (jb == qi || jb * kBlockN < qi * kBlockM + kBlockM - 1 - p.window)) ||
+                          ((jb + 1) * kBlockN > p.N);
       if (masked) {
-        // scaled scores with -inf where the key is hidden or past N
-        const int key0 = j * kBlockN;
+        // scaled scores with -inf where the key is hidden or past N: column i
+        // is visible iff lo <= i < hi
+        const int key0 = jb * kBlockN;
+        const int hi = (CAUSAL ? min(row + 1, p.N) : p.N) - key0;
+        const int lo = CAUSAL ? row - p.window - key0 : 0;
 #pragma unroll
         for (int i = 0; i < 128; ++i) {
-          const int key = key0 + i;
-          const bool vis = key < p.N && (!CAUSAL || key <= row);
+          const bool vis = i >= lo && i < hi;
           u[i] = __float_as_uint(vis ? __uint_as_float(u[i]) * c : -INFINITY);
         }
       }
@@ -359,7 +368,9 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
         alpha = ex2_sfu(m_use - m_new);
         m_use = m_new;
       }
-      const float neg_m = -m_use;
+      // a row that has seen only hidden keys so far (sliding window) keeps
+      // m = -inf; its p must be 0, not exp2(-inf + inf)
+      const float neg_m = m_use == -INFINITY ? 0.f : -m_use;
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
       if constexpr (FP8) {
         const float f8 = 256.f * sv_j / v_max;

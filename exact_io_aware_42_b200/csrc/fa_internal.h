@@ -25,6 +25,7 @@ cudaError_t set_smem_once(int bytes) {
 constexpr int kBlockM = 128;      // query rows per tile (one TMEM lane per row)
 constexpr int kBlockN = 128;      // keys per K/V tile
 constexpr float kRescaleTau = 8.0f;   // log2 units; see the forward kernel
+constexpr int kNoWindow = 1 << 30;    // window value meaning "no sliding window" (> any N + 128)
 
 struct FwdParams {
   CUtensorMap tm_q;     // [BH, N, d] bf16 or e4m3, box {64 or 128 elems, 128, 1}
@@ -41,6 +42,8 @@ struct FwdParams {
   int n_pairs;          // ceil(ceil(N/128) / 2): CTAs per (b, h)
   int n_kv;             // ceil(N / 128)
   int kv_group;         // G = H / H_kv query heads per K/V head (1: no grouping)
+  int window;           // causal sliding window: key j visible to query i iff i - window <= j <= i
+                        // (no window: kNoWindow)
   float scale_log2;     // scale * log2(e)
   float scale;
   int poly_pairs;       // of every 8 column pairs, how many use the FMA-pipe exp2
@@ -92,6 +95,7 @@ struct BwdParams {
   int n_kv;             // ceil(N / 128): key blocks = CTAs per (b, h)
   int n_q;              // ceil(N / 128): query blocks
   int kv_group;         // G = H / H_kv query heads per K/V head (1: no grouping)
+  int window;           // as in FwdParams
   float scale_log2;     // scale * log2(e)
   float scale;
   int poly_groups;      // of every 4 groups of 4 columns, how many use the FMA-pipe exp2

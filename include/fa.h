@@ -174,6 +174,8 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float
                      int d, float scale, int causal, void* stream);
 
 /*
+ * Extended entry points: grouped K/V heads and a causal sliding window.
+ *
  * Grouped K/V heads (GQA; MQA when H_kv = 1).  The librarian page lists
  * GQA/MQA as natively supported ("Cases where FlashAttention does not
  * help"); the pages give no formula, so the reading here is the usual one:
@@ -185,22 +187,32 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float
  *                     heads of each head's gradient.
  *  H_kv             : 1 <= H_kv, H a multiple of H_kv, else
  *                     FA_ERR_INVALID_ARG.
- * H_kv = H is exactly fa_fwd / fa_bwd / fa_bwd_deterministic / fa_fwd_fp8.
- * fa_bwd_gqa takes the workspace of fa_bwd_workspace_size(B, H, N, d)
- * (deterministic = 0) or fa_bwd_deterministic_workspace_size(B, H, N, d)
- * (deterministic != 0), sized by the query heads.  In the backward one
- * thread block per (K/V head, key block) visits the query blocks of all G
- * query heads in turn, so dK and dV are summed on chip, in a fixed order.
+ *
+ * Sliding window (the same page's list names it among the masks FA ships;
+ * again no formula).  Reading: with causal = 1 and window_left = w >= 0, key
+ * j is visible to query i iff i - w <= j <= i (w + 1 keys at most; w = 0
+ * keeps the diagonal only).  window_left = -1 means no window.  A window
+ * without causal, or window_left < -1, is FA_ERR_INVALID_ARG.  Key blocks
+ * wholly outside every row's window are skipped, not masked.
+ *
+ * H_kv = H with window_left = -1 is exactly fa_fwd / fa_bwd /
+ * fa_bwd_deterministic / fa_fwd_fp8.  fa_bwd_ex takes the workspace of
+ * fa_bwd_workspace_size(B, H, N, d) (deterministic = 0) or
+ * fa_bwd_deterministic_workspace_size(B, H, N, d) (deterministic != 0),
+ * sized by the query heads.  In the backward one thread block per (K/V
+ * head, key block) visits the query blocks of all G query heads in turn,
+ * so dK and dV are summed on chip, in a fixed order.
  */
-fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                     int H_kv, int N, int d, float scale, int causal, void* stream);
-fa_status fa_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                     const float* lse, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N,
-                     int d, float scale, int causal, int deterministic, void* workspace,
-                     size_t workspace_bytes, void* stream);
-fa_status fa_fwd_fp8_gqa(const void* q8, const void* k8, const void* v8, const float* sq,
-                         const float* sk, const float* sv, void* o, float* lse, int B, int H,
-                         int H_kv, int N, int d, float scale, int causal, void* stream);
+fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                    int H_kv, int N, int d, float scale, int causal, int window_left, void* stream);
+fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                    const float* lse, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N,
+                    int d, float scale, int causal, int window_left, int deterministic,
+                    void* workspace, size_t workspace_bytes, void* stream);
+fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v8, const float* sq,
+                        const float* sk, const float* sv, void* o, float* lse, int B, int H,
+                        int H_kv, int N, int d, float scale, int causal, int window_left,
+                        void* stream);
 
 /*
  * Device status word of the current device: FA_OK, or the first in-kernel

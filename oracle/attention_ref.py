@@ -71,6 +71,19 @@ def causal_mask(n_q: int, n_k: int) -> np.ndarray:
     return j <= i
 
 
+def window_mask(n_q: int, n_k: int, window: int) -> np.ndarray:
+    """Causal sliding window: True where i - window <= j <= i.
+
+    The librarian page names sliding-window masks among those FA ships
+    ("Cases where FlashAttention does not help") without a formula; the
+    reading is the left window of the causal mask, ``window`` keys before the
+    query plus the query's own key.
+    """
+    i = np.arange(n_q)[:, None]
+    j = np.arange(n_k)[None, :]
+    return (j <= i) & (j >= i - window)
+
+
 def softmax_ref(x: np.ndarray) -> np.ndarray:
     """Safe (max-subtracted) softmax along the last axis, fp64.
 
@@ -113,19 +126,21 @@ def attn_fwd_ref(q, k, v, scale: float, causal: bool):
     return o, lse
 
 
-def attn_fwd_rows_ref(q, k, v, scale: float, causal: bool, rows):
+def attn_fwd_rows_ref(q, k, v, scale: float, causal: bool, rows, window=None):
     """The forward definition for selected query rows of one head.
 
     q, k, v: [N, d] (one head); ``rows``: query indices.  Row i sees keys
-    j <= i when causal.  Returns (O [len(rows), d], L [len(rows)]), fp64.
-    Used where a whole head is too large to materialise (N up to 16K).
+    j <= i when causal (and j >= i - window with a sliding window).  Returns
+    (O [len(rows), d], L [len(rows)]), fp64.  Used where a whole head is too
+    large to materialise (N up to 16K).
     """
     q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
     rows = np.asarray(rows, dtype=np.int64)
     o = np.zeros((rows.size, v.shape[1]))
     lse = np.zeros(rows.size)
     for n, i in enumerate(rows):
-        kk, vv = (k[: i + 1], v[: i + 1]) if causal else (k, v)
+        lo = 0 if window is None else max(0, i - window)
+        kk, vv = (k[lo: i + 1], v[lo: i + 1]) if causal else (k, v)
         srow = float(scale) * (kk @ q[i])
         m = np.max(srow)
         e = np.exp(srow - m)
@@ -244,8 +259,16 @@ def attn_fwd_online_ref(q, k, v, scale: float, causal: bool, block_sizes: Sequen
     return o, lse
 
 
-def attn_fwd_gqa_ref(q, k, v, scale: float, causal: bool):
+def _scores_window(q2, k2, scale, causal, window):
+    s = scores_ref(q2, k2, scale, causal)
+    if window is not None:
+        s = np.where(window_mask(q2.shape[0], k2.shape[0], window), s, -np.inf)
+    return s
+
+
+def attn_fwd_gqa_ref(q, k, v, scale: float, causal: bool, window=None):
     """Attention with grouped K/V heads, fp64.  q: [B, H, N, d]; k, v: [B, H_kv, N, d].
+    ``window`` (causal only): the sliding window of ``window_mask``.
 
     The librarian page lists GQA/MQA among the variants FlashAttention
     supports ("Cases where FlashAttention does not help") without a formula;
@@ -264,7 +287,7 @@ def attn_fwd_gqa_ref(q, k, v, scale: float, causal: bool):
     for b in range(B):
         for h in range(H):
             kk, vv = k[b, h // g], v[b, h // g]
-            s = scores_ref(q[b, h], kk, scale, causal)
+            s = _scores_window(q[b, h], kk, scale, causal, window)
             m = np.max(s, axis=1)
             e = np.exp(s - m[:, None])
             ell = np.sum(e, axis=1)
@@ -273,7 +296,7 @@ def attn_fwd_gqa_ref(q, k, v, scale: float, causal: bool):
     return o, lse
 
 
-def attn_bwd_gqa_ref(q, k, v, do, scale: float, causal: bool):
+def attn_bwd_gqa_ref(q, k, v, do, scale: float, causal: bool, window=None):
     """Gradients of sum(O * dO) for grouped K/V heads, fp64.
 
     dQ of head h is that of plain attention with K/V head h // G; since a
@@ -285,14 +308,14 @@ def attn_bwd_gqa_ref(q, k, v, do, scale: float, causal: bool):
     B, H, N, d = q.shape
     h_kv = k.shape[1]
     g = H // h_kv
-    _, lse = attn_fwd_gqa_ref(q, k, v, scale, causal)
+    _, lse = attn_fwd_gqa_ref(q, k, v, scale, causal, window)
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
     for b in range(B):
         for h in range(H):
             kk, vv = k[b, h // g], v[b, h // g]
-            p = np.exp(scores_ref(q[b, h], kk, scale, causal) - lse[b, h][:, None])
+            p = np.exp(_scores_window(q[b, h], kk, scale, causal, window) - lse[b, h][:, None])
             dp = do[b, h] @ vv.T
             ds = p * (dp - np.sum(p * dp, axis=1)[:, None])
             dq[b, h] = float(scale) * (ds @ kk)

@@ -1,5 +1,5 @@
-"""GPU parity of grouped K/V heads (fa_fwd_gqa, fa_bwd_gqa, fa_fwd_fp8_gqa
-through the C ABI) against the fp64 grouped oracle.
+"""GPU parity of grouped K/V heads (fa_fwd_ex, fa_bwd_ex, fa_fwd_fp8_ex with
+H_kv < H, through the C ABI) against the fp64 grouped oracle.
 
 Also exact identities of the implementation: with the K/V heads repeated
 explicitly, the plain forward gives the same bits as the grouped one (same
@@ -130,9 +130,9 @@ def test_gqa_bad_head_counts():
         fa.fwd(q, k, k)
     lse = torch.zeros((1, 4, 128), dtype=torch.float32, device="cuda")
     from exact_io_aware_42_b200._lib import lib
-    code = lib().fa_fwd_gqa(q.data_ptr(), k.data_ptr(), k.data_ptr(), q.data_ptr(), lse.data_ptr(),
-                            1, 4, 3, 128, 64, 0.125, 0, None)
+    code = lib().fa_fwd_ex(q.data_ptr(), k.data_ptr(), k.data_ptr(), q.data_ptr(), lse.data_ptr(),
+                           1, 4, 3, 128, 64, 0.125, 0, -1, None)
     assert code == 1
-    code = lib().fa_fwd_gqa(q.data_ptr(), k.data_ptr(), k.data_ptr(), q.data_ptr(), lse.data_ptr(),
-                            1, 4, 0, 128, 64, 0.125, 0, None)
+    code = lib().fa_fwd_ex(q.data_ptr(), k.data_ptr(), k.data_ptr(), q.data_ptr(), lse.data_ptr(),
+                           1, 4, 0, 128, 64, 0.125, 0, -1, None)
     assert code == 1
