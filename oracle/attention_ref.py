@@ -259,16 +259,33 @@ def attn_fwd_online_ref(q, k, v, scale: float, causal: bool, block_sizes: Sequen
     return o, lse
 
 
-def _scores_window(q2, k2, scale, causal, window):
+def alibi_bias(n_q: int, n_k: int, slope: float) -> np.ndarray:
+    """ALiBi bias -slope * |i - j| added to the scaled scores.
+
+    The librarian page names ALiBi among the masks FA ships ("Cases where
+    FlashAttention does not help") without a formula; the reading is the
+    linear distance penalty of the ALiBi method, one non-negative slope per
+    query head, in the units of the scaled scores (natural log).  With the
+    causal mask |i - j| = i - j on every visible pair.
+    """
+    i = np.arange(n_q)[:, None]
+    j = np.arange(n_k)[None, :]
+    return -float(slope) * np.abs(i - j)
+
+
+def _scores_window(q2, k2, scale, causal, window, slope=None):
     s = scores_ref(q2, k2, scale, causal)
     if window is not None:
         s = np.where(window_mask(q2.shape[0], k2.shape[0], window), s, -np.inf)
+    if slope is not None:
+        s = s + alibi_bias(q2.shape[0], k2.shape[0], slope)
     return s
 
 
-def attn_fwd_gqa_ref(q, k, v, scale: float, causal: bool, window=None):
+def attn_fwd_gqa_ref(q, k, v, scale: float, causal: bool, window=None, alibi=None):
     """Attention with grouped K/V heads, fp64.  q: [B, H, N, d]; k, v: [B, H_kv, N, d].
-    ``window`` (causal only): the sliding window of ``window_mask``.
+    ``window`` (causal only): the sliding window of ``window_mask``;
+    ``alibi``: H slopes, the bias of ``alibi_bias`` for query head h.
 
     The librarian page lists GQA/MQA among the variants FlashAttention
     supports ("Cases where FlashAttention does not help") without a formula;
@@ -287,7 +304,7 @@ def attn_fwd_gqa_ref(q, k, v, scale: float, causal: bool, window=None):
     for b in range(B):
         for h in range(H):
             kk, vv = k[b, h // g], v[b, h // g]
-            s = _scores_window(q[b, h], kk, scale, causal, window)
+            s = _scores_window(q[b, h], kk, scale, causal, window, None if alibi is None else alibi[h])
             m = np.max(s, axis=1)
             e = np.exp(s - m[:, None])
             ell = np.sum(e, axis=1)
@@ -296,7 +313,7 @@ def attn_fwd_gqa_ref(q, k, v, scale: float, causal: bool, window=None):
     return o, lse
 
 
-def attn_bwd_gqa_ref(q, k, v, do, scale: float, causal: bool, window=None):
+def attn_bwd_gqa_ref(q, k, v, do, scale: float, causal: bool, window=None, alibi=None):
     """Gradients of sum(O * dO) for grouped K/V heads, fp64.
 
     dQ of head h is that of plain attention with K/V head h // G; since a
@@ -308,14 +325,15 @@ def attn_bwd_gqa_ref(q, k, v, do, scale: float, causal: bool, window=None):
     B, H, N, d = q.shape
     h_kv = k.shape[1]
     g = H // h_kv
-    _, lse = attn_fwd_gqa_ref(q, k, v, scale, causal, window)
+    _, lse = attn_fwd_gqa_ref(q, k, v, scale, causal, window, alibi)
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
     for b in range(B):
         for h in range(H):
             kk, vv = k[b, h // g], v[b, h // g]
-            p = np.exp(_scores_window(q[b, h], kk, scale, causal, window) - lse[b, h][:, None])
+            p = np.exp(_scores_window(q[b, h], kk, scale, causal, window,
+                                      None if alibi is None else alibi[h]) - lse[b, h][:, None])
             dp = do[b, h] @ vv.T
             ds = p * (dp - np.sum(p * dp, axis=1)[:, None])
             dq[b, h] = float(scale) * (ds @ kk)
