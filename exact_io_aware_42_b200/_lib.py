@@ -27,11 +27,11 @@ SIGNATURES = {
     "fa_bwd_deterministic": (c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, c_int, c_int, c_int, c_int,
                                      c_float, c_int, _P, c_size_t, _P]),
     "fa_fwd_ex": (c_int, [_P, _P, _P, _P, _P, c_int, c_int, c_int, c_int, c_int, c_float, c_int, c_int,
-                          _P]),
+                          _P, _P]),
     "fa_bwd_ex": (c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, c_int, c_int, c_int, c_int, c_int,
-                          c_float, c_int, c_int, c_int, _P, c_size_t, _P]),
+                          c_float, c_int, c_int, _P, c_int, _P, c_size_t, _P]),
     "fa_fwd_fp8_ex": (c_int, [_P, _P, _P, _P, _P, _P, _P, _P, c_int, c_int, c_int, c_int, c_int,
-                              c_float, c_int, c_int, _P]),
+                              c_float, c_int, c_int, _P, _P]),
     "fa_bwd_noalloc": (c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, c_int, c_int, c_int, c_int,
                                c_float, c_int, _P]),
     "fa_quant_fp8": (c_int, [_P, _P, _P, c_int, c_int, c_int, c_int, _P, _P]),

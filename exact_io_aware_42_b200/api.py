@@ -5,7 +5,8 @@ computation runs in the library's kernels.  Functions mirror include/fa.h:
 
 * ``fwd(q, k, v, causal, scale)``            -> (o, lse)
   (k, v may have fewer heads than q: grouped K/V heads, H a multiple of H_kv;
-  ``window=w`` with causal=True: key j visible to query i iff i - w <= j <= i)
+  ``window=w`` with causal=True: key j visible to query i iff i - w <= j <= i;
+  ``alibi=slopes``: a CUDA fp32 tensor of H slopes, bias -slope_h |i - j|)
 * ``bwd(q, k, v, o, do, lse, causal, scale, deterministic=False)`` -> (dq, dk, dv)
 * ``quant_fp8(x, signs=None)``               -> (x8 as uint8, block scales)
 * ``fwd_fp8(q8, k8, v8, sq, sk, sv, causal, scale)`` -> (o, lse)
@@ -50,6 +51,14 @@ def _window(window: Optional[int], causal: bool) -> int:
     return int(window)
 
 
+def _alibi(alibi: Optional[torch.Tensor], H: int):
+    if alibi is None:
+        return None
+    if not alibi.is_cuda or alibi.dtype != torch.float32 or alibi.numel() != H or not alibi.is_contiguous():
+        raise ValueError("alibi must be a contiguous CUDA fp32 tensor of H slopes")
+    return alibi
+
+
 def _check_bhnd(name: str, t: torch.Tensor, dtype, shape=None) -> None:
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
@@ -67,7 +76,7 @@ def n_blocks(N: int) -> int:
 
 
 def fwd(q, k, v, causal: bool = False, scale: Optional[float] = None, out=None, lse=None,
-        window: Optional[int] = None):
+        window: Optional[int] = None, alibi: Optional[torch.Tensor] = None):
     """Exact attention forward (bf16).  Returns (o bf16 [B,H,N,d], lse fp32 [B,H,N])."""
     wl = _window(window, causal)
     _check_bhnd("q", q, torch.bfloat16)
@@ -79,13 +88,14 @@ def fwd(q, k, v, causal: bool = False, scale: Optional[float] = None, out=None, 
         scale = 1.0 / math.sqrt(d)
     o = torch.empty_like(q) if out is None else out
     lse_t = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
-    if h_kv == H and wl < 0:
+    al = _alibi(alibi, H)
+    if h_kv == H and wl < 0 and al is None:
         code = lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), B, H, N, d, float(scale),
                             int(bool(causal)), _stream())
         check("fa_fwd", code)
     else:
         code = lib().fa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse_t), B, H, h_kv, N, d,
-                               float(scale), int(bool(causal)), wl, _stream())
+                               float(scale), int(bool(causal)), wl, _ptr(al), _stream())
         check("fa_fwd_ex", code)
     return o, lse_t
 
@@ -98,11 +108,12 @@ def bwd_workspace_size(B: int, H: int, N: int, d: int, deterministic: bool = Fal
 
 def bwd(q, k, v, o, do, lse, causal: bool = False, scale: Optional[float] = None,
         workspace: Optional[torch.Tensor] = None, dq=None, dk=None, dv=None,
-        deterministic: bool = False, window: Optional[int] = None):
+        deterministic: bool = False, window: Optional[int] = None,
+        alibi: Optional[torch.Tensor] = None):
     """Attention backward (bf16).  Returns (dq, dk, dv).
 
     ``deterministic=True`` calls fa_bwd_deterministic: bitwise reproducible
-    gradients (dQ by a separate query-block-major kernel).  ``window`` as in fwd."""
+    gradients (dQ by a separate query-block-major kernel).  ``window``, ``alibi`` as in fwd."""
     wl = _window(window, causal)
     _check_bhnd("q", q, torch.bfloat16)
     B, H, N, d = q.shape
@@ -121,7 +132,8 @@ def bwd(q, k, v, o, do, lse, causal: bool = False, scale: Optional[float] = None
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    if h_kv == H and wl < 0:
+    al = _alibi(alibi, H)
+    if h_kv == H and wl < 0 and al is None:
         name = "fa_bwd_deterministic" if deterministic else "fa_bwd"
         code = getattr(lib(), name)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
                                     _ptr(dk), _ptr(dv), B, H, N, d, float(scale), int(bool(causal)),
@@ -130,7 +142,8 @@ def bwd(q, k, v, o, do, lse, causal: bool = False, scale: Optional[float] = None
         name = "fa_bwd_ex"
         code = lib().fa_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
                                _ptr(dk), _ptr(dv), B, H, h_kv, N, d, float(scale), int(bool(causal)), wl,
-                               int(bool(deterministic)), _ptr(workspace), workspace.numel(), _stream())
+                               _ptr(al), int(bool(deterministic)), _ptr(workspace), workspace.numel(),
+                               _stream())
     check(name, code)
     return dq, dk, dv
 
@@ -151,7 +164,7 @@ def quant_fp8(x, signs: Optional[torch.Tensor] = None, out=None, scales=None):
 
 
 def fwd_fp8(q8, k8, v8, sq, sk, sv, causal: bool = False, scale: Optional[float] = None,
-            out=None, lse=None, window: Optional[int] = None):
+            out=None, lse=None, window: Optional[int] = None, alibi: Optional[torch.Tensor] = None):
     """FP8 attention forward on quantised inputs.  Returns (o bf16, lse fp32)."""
     wl = _window(window, causal)
     _check_bhnd("q8", q8, torch.uint8)
@@ -168,7 +181,7 @@ def fwd_fp8(q8, k8, v8, sq, sk, sv, causal: bool = False, scale: Optional[float]
     lse_t = torch.empty((B, H, N), dtype=torch.float32, device=q8.device) if lse is None else lse
     code = lib().fa_fwd_fp8_ex(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk), _ptr(sv), _ptr(o),
                                _ptr(lse_t), B, H, h_kv, N, d, float(scale), int(bool(causal)), wl,
-                               _stream())
+                               _ptr(_alibi(alibi, H)), _stream())
     check("fa_fwd_fp8_ex", code)
     return o, lse_t
 

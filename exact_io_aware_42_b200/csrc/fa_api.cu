@@ -147,8 +147,9 @@ using namespace fa;
 
 extern "C" fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
                                int B, int H, int H_kv, int N, int d, float scale, int causal,
-                               int window_left, void* stream) {
+                               int window_left, const float* alibi_slopes, void* stream) {
   fa_status st = check_shape(B, H, N, d, scale);
+  if (reinterpret_cast<uintptr_t>(alibi_slopes) & 3u) return FA_ERR_MISALIGNED;
   if (st != FA_OK) return st;
   if (H > 0 && (st = check_kv_heads(H, H_kv)) != FA_OK) return st;
   int window = kNoWindow;
@@ -177,6 +178,8 @@ extern "C" fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void
   p.BH = BH;
   p.kv_group = H / H_kv;
   p.window = window;
+  p.alibi = alibi_slopes;
+  p.H = H;
   p.n_kv = (N + kBlockN - 1) / kBlockN;
   p.n_pairs = ((N + kBlockM - 1) / kBlockM + 1) / 2;
   p.scale = scale;
@@ -192,7 +195,7 @@ extern "C" fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void
 
 extern "C" fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                             int B, int H, int N, int d, float scale, int causal, void* stream) {
-  return fa_fwd_ex(q, k, v, o, lse, B, H, H, N, d, scale, causal, -1, stream);
+  return fa_fwd_ex(q, k, v, o, lse, B, H, H, N, d, scale, causal, -1, nullptr, stream);
 }
 
 extern "C" size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
@@ -215,9 +218,10 @@ namespace {
 // deterministic one runs the main kernel without dQ and the dQ kernel.
 fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const void* dout,
                      const float* lse, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N,
-                     int d, float scale, int causal, int window_left, void* workspace,
-                     size_t workspace_bytes, void* stream, bool deterministic) {
+                     int d, float scale, int causal, int window_left, const float* alibi_slopes,
+                     void* workspace, size_t workspace_bytes, void* stream, bool deterministic) {
   fa_status st = check_shape(B, H, N, d, scale);
+  if (reinterpret_cast<uintptr_t>(alibi_slopes) & 3u) return FA_ERR_MISALIGNED;
   if (st != FA_OK) return st;
   if (H > 0 && (st = check_kv_heads(H, H_kv)) != FA_OK) return st;
   int window = kNoWindow;
@@ -264,6 +268,8 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   p.n_q = (N + 127) / 128;
   p.kv_group = H / H_kv;
   p.window = window;
+  p.alibi = alibi_slopes;
+  p.H = H;
   p.scale = scale;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.poly_groups = bwd_poly_groups();
@@ -290,8 +296,8 @@ extern "C" fa_status fa_bwd(const void* q, const void* k, const void* v, const v
                             const void* dout, const float* lse, void* dq, void* dk, void* dv,
                             int B, int H, int N, int d, float scale, int causal, void* workspace,
                             size_t workspace_bytes, void* stream) {
-  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, H, N, d, scale, causal, -1, workspace,
-                    workspace_bytes, stream, false);
+  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, H, N, d, scale, causal, -1, nullptr,
+                    workspace, workspace_bytes, stream, false);
 }
 
 extern "C" fa_status fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,
@@ -299,17 +305,17 @@ extern "C" fa_status fa_bwd_deterministic(const void* q, const void* k, const vo
                                           void* dv, int B, int H, int N, int d, float scale,
                                           int causal, void* workspace, size_t workspace_bytes,
                                           void* stream) {
-  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, H, N, d, scale, causal, -1, workspace,
-                    workspace_bytes, stream, true);
+  return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, H, N, d, scale, causal, -1, nullptr,
+                    workspace, workspace_bytes, stream, true);
 }
 
 extern "C" fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* o,
                                const void* dout, const float* lse, void* dq, void* dk, void* dv,
                                int B, int H, int H_kv, int N, int d, float scale, int causal,
-                               int window_left, int deterministic, void* workspace,
-                               size_t workspace_bytes, void* stream) {
+                               int window_left, const float* alibi_slopes, int deterministic,
+                               void* workspace, size_t workspace_bytes, void* stream) {
   return bwd_common(q, k, v, o, dout, lse, dq, dk, dv, B, H, H_kv, N, d, scale, causal, window_left,
-                    workspace, workspace_bytes, stream, deterministic != 0);
+                    alibi_slopes, workspace, workspace_bytes, stream, deterministic != 0);
 }
 
 extern "C" fa_status fa_quant_fp8(const void* x, void* x8, float* scales, int B, int H, int N,
@@ -352,8 +358,9 @@ extern "C" fa_status fa_quant_fp8(const void* x, void* x8, float* scales, int B,
 extern "C" fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v8, const float* sq,
                                    const float* sk, const float* sv, void* o, float* lse, int B,
                                    int H, int H_kv, int N, int d, float scale, int causal,
-                                   int window_left, void* stream) {
+                                   int window_left, const float* alibi_slopes, void* stream) {
   fa_status st = check_shape(B, H, N, d, scale);
+  if (reinterpret_cast<uintptr_t>(alibi_slopes) & 3u) return FA_ERR_MISALIGNED;
   if (st != FA_OK) return st;
   if (H > 0 && (st = check_kv_heads(H, H_kv)) != FA_OK) return st;
   int window = kNoWindow;
@@ -386,6 +393,8 @@ extern "C" fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v
   p.BH = BH;
   p.kv_group = H / H_kv;
   p.window = window;
+  p.alibi = alibi_slopes;
+  p.H = H;
   p.n_kv = (N + kBlockN - 1) / kBlockN;
   p.n_pairs = ((N + kBlockM - 1) / kBlockM + 1) / 2;
   p.scale = scale;
@@ -401,7 +410,8 @@ extern "C" fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v
 extern "C" fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* sq,
                                 const float* sk, const float* sv, void* o, float* lse, int B, int H,
                                 int N, int d, float scale, int causal, void* stream) {
-  return fa_fwd_fp8_ex(q8, k8, v8, sq, sk, sv, o, lse, B, H, H, N, d, scale, causal, -1, stream);
+  return fa_fwd_fp8_ex(q8, k8, v8, sq, sk, sv, o, lse, B, H, H, N, d, scale, causal, -1, nullptr,
+                       stream);
 }
 
 extern "C" fa_status fa_selftest_wait_timeout(void* stream) {

@@ -396,6 +396,9 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
       // within the sliding window, and none at all for a key past N.
       const int c_lo = (CAUSAL && i == j) ? r : 0;
       const int c_hi = !key_ok ? -1 : (CAUSAL ? min(127, key + p.window - i * 128) : 127);
+      // ALiBi: -slope log2(e) |query - key| for this block's query head
+      const float sl2 = p.alibi ? p.alibi[q_head(idx) % p.H] * 1.4426950408889634f : 0.f;
+      const float dq0 = static_cast<float>(i * 128 + static_cast<int>(col_half) - key);
       const uint32_t tS = tmem + C::kColA + lane_off + col_half;
       const uint32_t tDP = tmem + C::kColB + lane_off + col_half;
       if (!(ok = mbar_wait_warp(bar(B_S), idx & 1, ab, kSiteBSmS))) break;
@@ -409,10 +412,15 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
           const float4 l4 = L4[c4];
           const float lq[4] = {l4.x, l4.y, l4.z, l4.w};
           float pv[4];
+          float nl[4] = {-lq[0], -lq[1], -lq[2], -lq[3]};
+          if (p.alibi) {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) nl[t] -= sl2 * fabsf(dq0 + static_cast<float>(4 * c4 + t));
+          }
           const uint64_t x01 = f2_fma(f2_pack(__uint_as_float(u[4 * c4]), __uint_as_float(u[4 * c4 + 1])),
-                                      f2_pack(cs, cs), f2_pack(-lq[0], -lq[1]));
+                                      f2_pack(cs, cs), f2_pack(nl[0], nl[1]));
           const uint64_t x23 = f2_fma(f2_pack(__uint_as_float(u[4 * c4 + 2]), __uint_as_float(u[4 * c4 + 3])),
-                                      f2_pack(cs, cs), f2_pack(-lq[2], -lq[3]));
+                                      f2_pack(cs, cs), f2_pack(nl[2], nl[3]));
           const bool poly = (c4 & 3) < NPOLY;
           const uint64_t p01 = poly ? exp2_poly_f2<3>(x01) : exp2_sfu_f2(x01);
           const uint64_t p23 = poly ? exp2_poly_f2<3>(x23) : exp2_sfu_f2(x23);

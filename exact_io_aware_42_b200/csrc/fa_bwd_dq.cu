@@ -245,6 +245,8 @@ __global__ void __launch_bounds__(320, 1) bwd_dq_kernel(const __grid_constant__ 
     const float l2 = q < p.N ? p.lse[grow] * 1.4426950408889634f : INFINITY;   // rows past N: P = 0
     const float dlt = q < p.N ? p.delta[grow] : 0.f;
     const float cs = p.scale_log2;
+    // ALiBi: -slope log2(e) |key - query| for this query head
+    const float sl2 = p.alibi ? p.alibi[bh % p.H] * 1.4426950408889634f : 0.f;
     bool ok = true;
     for (int j = 0; j < n_j && ok; ++j) {
       const int t = j & 1;
@@ -258,10 +260,16 @@ __global__ void __launch_bounds__(320, 1) bwd_dq_kernel(const __grid_constant__ 
       tc_fence_after();
       uint32_t u[64];
       tmem_ld64(tS, u);
+      const float dk0 = static_cast<float>(kbase - q);
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
+        float n0 = -l2, n1 = -l2;
+        if (p.alibi) {
+          n0 -= sl2 * fabsf(dk0 + static_cast<float>(c));
+          n1 -= sl2 * fabsf(dk0 + static_cast<float>(c + 1));
+        }
         const uint64_t x = f2_fma(f2_pack(__uint_as_float(u[c]), __uint_as_float(u[c + 1])), f2_pack(cs, cs),
-                                  f2_pack(-l2, -l2));
+                                  f2_pack(n0, n1));
         float p0, p1;
         f2_unpack(exp2_sfu_f2(x), p0, p1);
         u[c] = __float_as_uint(p0);

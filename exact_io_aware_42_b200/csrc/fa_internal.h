@@ -44,6 +44,8 @@ struct FwdParams {
   int kv_group;         // G = H / H_kv query heads per K/V head (1: no grouping)
   int window;           // causal sliding window: key j visible to query i iff i - window <= j <= i
                         // (no window: kNoWindow)
+  const float* alibi;   // ALiBi slopes [H] (natural-log units) or nullptr
+  int H;                // query heads per batch: head of flattened index bh is bh % H
   float scale_log2;     // scale * log2(e)
   float scale;
   int poly_pairs;       // of every 8 column pairs, how many use the FMA-pipe exp2
@@ -96,6 +98,8 @@ struct BwdParams {
   int n_q;              // ceil(N / 128): query blocks
   int kv_group;         // G = H / H_kv query heads per K/V head (1: no grouping)
   int window;           // as in FwdParams
+  const float* alibi;   // as in FwdParams
+  int H;
   float scale_log2;     // scale * log2(e)
   float scale;
   int poly_groups;      // of every 4 groups of 4 columns, how many use the FMA-pipe exp2

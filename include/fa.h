@@ -174,7 +174,7 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float
                      int d, float scale, int causal, void* stream);
 
 /*
- * Extended entry points: grouped K/V heads and a causal sliding window.
+ * Extended entry points: grouped K/V heads, a causal sliding window, ALiBi.
  *
  * Grouped K/V heads (GQA; MQA when H_kv = 1).  The librarian page lists
  * GQA/MQA as natively supported ("Cases where FlashAttention does not
@@ -195,8 +195,14 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float
  * without causal, or window_left < -1, is FA_ERR_INVALID_ARG.  Key blocks
  * wholly outside every row's window are skipped, not masked.
  *
- * H_kv = H with window_left = -1 is exactly fa_fwd / fa_bwd /
- * fa_bwd_deterministic / fa_fwd_fp8.  fa_bwd_ex takes the workspace of
+ * ALiBi (the same list names it; no formula).  Reading: the scaled score of
+ * query i and key j gets -slope_h * |i - j| added before the softmax (natural
+ * log units, one slope per query head h).  alibi_slopes: NULL for none, else
+ * a device array of H fp32 slopes (finite, >= 0; 4-byte aligned, else
+ * FA_ERR_MISALIGNED), read by the kernels.  The returned L includes the bias.
+ *
+ * H_kv = H with window_left = -1 and alibi_slopes = NULL is exactly fa_fwd /
+ * fa_bwd / fa_bwd_deterministic / fa_fwd_fp8.  fa_bwd_ex takes the workspace of
  * fa_bwd_workspace_size(B, H, N, d) (deterministic = 0) or
  * fa_bwd_deterministic_workspace_size(B, H, N, d) (deterministic != 0),
  * sized by the query heads.  In the backward one thread block per (K/V
@@ -204,15 +210,16 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float
  * so dK and dV are summed on chip, in a fixed order.
  */
 fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                    int H_kv, int N, int d, float scale, int causal, int window_left, void* stream);
+                    int H_kv, int N, int d, float scale, int causal, int window_left,
+                    const float* alibi_slopes, void* stream);
 fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* o, const void* dout,
                     const float* lse, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N,
-                    int d, float scale, int causal, int window_left, int deterministic,
-                    void* workspace, size_t workspace_bytes, void* stream);
+                    int d, float scale, int causal, int window_left, const float* alibi_slopes,
+                    int deterministic, void* workspace, size_t workspace_bytes, void* stream);
 fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v8, const float* sq,
                         const float* sk, const float* sv, void* o, float* lse, int B, int H,
                         int H_kv, int N, int d, float scale, int causal, int window_left,
-                        void* stream);
+                        const float* alibi_slopes, void* stream);
 
 /*
  * Device status word of the current device: FA_OK, or the first in-kernel

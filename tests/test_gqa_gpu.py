@@ -131,8 +131,8 @@ def test_gqa_bad_head_counts():
     lse = torch.zeros((1, 4, 128), dtype=torch.float32, device="cuda")
     from exact_io_aware_42_b200._lib import lib
     code = lib().fa_fwd_ex(q.data_ptr(), k.data_ptr(), k.data_ptr(), q.data_ptr(), lse.data_ptr(),
-                           1, 4, 3, 128, 64, 0.125, 0, -1, None)
+                           1, 4, 3, 128, 64, 0.125, 0, -1, None, None)
     assert code == 1
     code = lib().fa_fwd_ex(q.data_ptr(), k.data_ptr(), k.data_ptr(), q.data_ptr(), lse.data_ptr(),
-                           1, 4, 0, 128, 64, 0.125, 0, -1, None)
+                           1, 4, 0, 128, 64, 0.125, 0, -1, None, None)
     assert code == 1

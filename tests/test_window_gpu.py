@@ -89,9 +89,9 @@ def test_window_argument_errors():
     q = torch.zeros((1, 2, 128, 64), dtype=torch.bfloat16, device="cuda")
     lse = torch.zeros((1, 2, 128), dtype=torch.float32, device="cuda")
     args = (q.data_ptr(), q.data_ptr(), q.data_ptr(), q.data_ptr(), lse.data_ptr(), 1, 2, 2, 128, 64, 0.125)
-    assert lib().fa_fwd_ex(*args, 0, 5, None) == 1       # window without causal
-    assert lib().fa_fwd_ex(*args, 1, -2, None) == 1      # window_left < -1
-    assert lib().fa_fwd_ex(*args, 1, -1, None) == 0      # no window
+    assert lib().fa_fwd_ex(*args, 0, 5, None, None) == 1       # window without causal
+    assert lib().fa_fwd_ex(*args, 1, -2, None, None) == 1      # window_left < -1
+    assert lib().fa_fwd_ex(*args, 1, -1, None, None) == 0      # no window
     torch.cuda.synchronize()
     with pytest.raises(ValueError):
         fa.fwd(q, q, q, causal=False, window=3)
