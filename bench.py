@@ -63,11 +63,19 @@ def workloads():
     out["mqa_B4_H16_Hkv1_N4096_d128_causal"] = dict(B=4, H=16, H_kv=1, N=4096, d=128, causal=True, seed=6)
     # causal sliding window of 1024 keys at N = 16384: FLOPs counted over the visible pairs only
     out["window1024_B1_H16_N16384_d128"] = dict(B=1, H=16, N=16384, d=128, causal=True, seed=7, window=1024)
+    # ALiBi with the geometric slopes 2^(-8 (h + 1) / H)
+    out["alibi_B4_H16_N4096_d128_causal"] = dict(B=4, H=16, N=4096, d=128, causal=True, seed=8, alibi=True)
     for name, w in out.items():
         w["name"] = name
         w.setdefault("H_kv", w["H"])
         w.setdefault("window", None)
+        w.setdefault("alibi", False)
     return out
+
+
+def alibi_slopes(H):
+    """Geometric ALiBi slopes 2^(-8 (h + 1) / H), one per query head."""
+    return [2.0 ** (-8.0 * (h + 1) / H) for h in range(H)]
 
 
 WORKLOAD = None   # set in main()
@@ -194,7 +202,8 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs, deterministic=False, window=None):
+def build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs, deterministic=False, window=None,
+               alibi=None):
     """The hot path as a list of (stage name, callable, FLOPs, kernel launches)."""
     state = {}
 
@@ -205,12 +214,13 @@ def build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs, deterministic=
 
     def s_fwd():
         state["o"], state["lse"] = fa.fwd(q, k, v, causal=causal, out=bufs["o"], lse=bufs["lse"],
-                                          window=window)
+                                          window=window, alibi=alibi)
 
     def s_bwd():
         state["dq"], state["dk"], state["dv"] = fa.bwd(
             q, k, v, bufs["o"], do, bufs["lse"], causal=causal, workspace=ws,
-            dq=bufs["dq"], dk=bufs["dk"], dv=bufs["dv"], deterministic=deterministic, window=window)
+            dq=bufs["dq"], dk=bufs["dk"], dv=bufs["dv"], deterministic=deterministic, window=window,
+            alibi=alibi)
 
     src = {"q": q, "k": k, "v": v}
     q8 = {n: torch.empty(t.shape, dtype=torch.uint8, device=q.device) for n, t in src.items()}
@@ -227,7 +237,7 @@ def build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs, deterministic=
     def s_fwd8():
         state["o_fp8"], state["lse_fp8"] = fa.fwd_fp8(q8["q"], q8["k"], q8["v"], sc8["q"], sc8["k"],
                                                       sc8["v"], causal=causal, out=o8, lse=lse8,
-                                                      window=window)
+                                                      window=window, alibi=alibi)
 
     f = fwd_flops(B, H, N, d, causal, window)
     # backward launches: preprocess, main, and postprocess (atomic) or dQ (deterministic)
@@ -298,17 +308,18 @@ def oracle_sample(budget_s: float, B, H, N, d, causal, with_bwd: bool):
         kh = h // (H // H_kv)           # the K/V head of query head h
         kl = (slice(b, b + 1), slice(kh, kh + 1))
         win = WORKLOAD.get("window")
-        oracle.attn_fwd_gqa_ref(q[sl], k[kl], v[kl], sc, causal, window=win)
+        sl_ = [alibi_slopes(H)[h]] if WORKLOAD.get("alibi") else None
+        oracle.attn_fwd_gqa_ref(q[sl], k[kl], v[kl], sc, causal, window=win, alibi=sl_)
         flops += fwd_flops(1, 1, N, d, causal, win)
         if with_bwd:
-            oracle.attn_bwd_gqa_ref(q[sl], k[kl], v[kl], do[sl], sc, causal, window=win)
+            oracle.attn_bwd_gqa_ref(q[sl], k[kl], v[kl], do[sl], sc, causal, window=win, alibi=sl_)
             flops += 2.5 * fwd_flops(1, 1, N, d, causal, win)
             # FP8 rows: block quantisation (Q, K rotated; V) and attention on the
             # dequantised values
             sg = inputs.signs(d).numpy()
             deq = [oracle.dequant_fp8_ref(*oracle.quant_fp8_ref(x[s_].double().numpy(), rot, sg))
                    for x, s_, rot in ((q, sl, True), (k, kl, True), (v, kl, False))]
-            oracle.attn_fwd_gqa_ref(deq[0], deq[1], deq[2], sc, causal, window=win)
+            oracle.attn_fwd_gqa_ref(deq[0], deq[1], deq[2], sc, causal, window=win, alibi=sl_)
             flops += fwd_flops(1, 1, N, d, causal, win)
         heads += 1
         if time.perf_counter() - t0 >= budget_s:
@@ -353,7 +364,7 @@ def config_block():
     w = WORKLOAD
     in_bytes = 2 * (w["H"] + w["H_kv"]) * w["B"] * w["N"] * w["d"] * 2
     return {"workload": w["name"], "B": w["B"], "H": w["H"], "H_kv": w["H_kv"], "N": w["N"], "d": w["d"],
-            "bwd": BWD_MODE, "window": w["window"],
+            "bwd": BWD_MODE, "window": w["window"], "alibi": "slopes 2^(-8(h+1)/H)" if w["alibi"] else None,
             "causal": w["causal"], "global_batch": w["B"], "seq_len": w["N"],
             "parallelism": "independent replicas per GPU (heads), no collective",
             "l2": (f"inputs (Q, K, V, dO) {in_bytes / 2**20:.0f} MiB > 126 MB L2, no flush"
@@ -385,7 +396,9 @@ def run_ours(args):
     signs = inputs.signs(d).to(dev)
     q, k, v, do = (t.to(dev) for t in (hq, hk, hv, hdo))
     stages, state = build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs,
-                               deterministic=BWD_MODE == "deterministic", window=w["window"])
+                               deterministic=BWD_MODE == "deterministic", window=w["window"],
+                               alibi=torch.tensor(alibi_slopes(H), dtype=torch.float32, device=dev)
+                               if w["alibi"] else None)
     step_flops = sum(s[2] for s in stages)
     launches_per_step = sum(s[3] for s in stages)
 

@@ -39,6 +39,15 @@ def max_abs(x, ref) -> float:
     return float(np.max(np.abs(f64(x) - f64(ref)))) if np.size(ref) else 0.0
 
 
+def max_scaled_err(o, o_ref) -> float:
+    """max |err| / max(1, |ref|) elementwise: the forward bound for masks
+    (sliding window, ALiBi) that average few keys per row, where |O| grows
+    past 1 and one bf16 half-ulp of O alone approaches 1e-2 (the same
+    reading as the large-magnitude forward test)."""
+    o, o_ref = f64(o), f64(o_ref)
+    return float(np.max(np.abs(o - o_ref) / np.maximum(1.0, np.abs(o_ref)))) if o_ref.size else 0.0
+
+
 def assert_fwd_close(o, lse, o_ref, lse_ref, tag=""):
     o, lse = f64(o), f64(lse)
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse)), f"{tag}: non-finite output"

@@ -14,7 +14,8 @@ import torch
 
 import oracle
 from exact_io_aware_42_b200 import inputs
-from tests.helpers import GRAD_REL_RMS, GRAD_RMS_FLOOR, LSE_MAX_ABS, O_MAX_ABS, O_REL_RMS, f64, rel_rms
+from tests.helpers import (GRAD_REL_RMS, GRAD_RMS_FLOOR, LSE_MAX_ABS, O_MAX_ABS, O_REL_RMS, f64,
+                           max_scaled_err, rel_rms)
 
 pytestmark = pytest.mark.gpu
 
@@ -39,7 +40,7 @@ def test_window_fwd_bwd_parity(N, d, w):
     torch.cuda.synchronize()
     o_ref, lse_ref = oracle.attn_fwd_gqa_ref(q, k, v, scale, True, window=w)
     og, lg = f64(o.cpu()), f64(lse.cpu())
-    assert np.max(np.abs(og - o_ref)) <= O_MAX_ABS
+    assert max_scaled_err(og, o_ref) <= O_MAX_ABS
     assert rel_rms(og, o_ref) <= O_REL_RMS
     assert np.max(np.abs(lg - lse_ref)) <= LSE_MAX_ABS
     ref = oracle.attn_bwd_gqa_ref(q, k, v, do, scale, True, window=w)
@@ -63,7 +64,7 @@ def test_window_full_size_sampled_rows():
     rows = [0, 127, 128, 1023, 1024, 1025, 2047, 3000, 4095]
     for b, h in ((0, 0), (1, 7)):
         o_ref, l_ref = oracle.attn_fwd_rows_ref(q[b, h], k[b, h], v[b, h], 1 / math.sqrt(d), True, rows, window=w)
-        assert np.max(np.abs(f64(o[b, h, rows]) - o_ref)) <= O_MAX_ABS
+        assert max_scaled_err(o[b, h, rows], o_ref) <= O_MAX_ABS
         assert np.max(np.abs(f64(lse[b, h, rows]) - l_ref)) <= LSE_MAX_ABS
 
 
