@@ -34,6 +34,8 @@
 // dQ reduction (thread = query row); warp 12 TMA producer (also stages L and
 // D of each query block in shared memory); warp 13 TMEM owner and the single
 // MMA-issuing thread.  Every wait is bounded (fa_ptx.cuh).
+#include <type_traits>
+
 #include "fa_exp2.cuh"
 #include "fa_internal.h"
 #include "fa_ptx.cuh"
@@ -407,13 +409,15 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
       {
         uint32_t u[64];
         tmem_ld64(tS, u);
+        // one uniform branch on ALiBi outside the unrolled loop
+        auto p_rows = [&](auto alibi_on) {
 #pragma unroll
         for (int c4 = 0; c4 < 16; ++c4) {
           const float4 l4 = L4[c4];
           const float lq[4] = {l4.x, l4.y, l4.z, l4.w};
           float pv[4];
           float nl[4] = {-lq[0], -lq[1], -lq[2], -lq[3]};
-          if (p.alibi) {
+          if constexpr (decltype(alibi_on)::value) {
 #pragma unroll
             for (int t = 0; t < 4; ++t) nl[t] -= sl2 * fabsf(dq0 + static_cast<float>(4 * c4 + t));
           }
@@ -434,6 +438,11 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
           u[2 * c4] = pack_bf16x2(pv[0], pv[1]);
           u[2 * c4 + 1] = pack_bf16x2(pv[2], pv[3]);
         }
+        };
+        if (p.alibi)
+          p_rows(std::true_type{});
+        else
+          p_rows(std::false_type{});
 #pragma unroll
         for (int c = 0; c < 32; ++c) pp[c] = u[c];
         tmem_st32(tS, pp);

@@ -21,6 +21,8 @@
 // TMA producer, warp 9 TMEM owner and the single MMA-issuing thread.  K and V
 // have separate rings so that K_j, which the dQ product reads last, does not
 // hold back the next V.  Every wait is bounded (fa_ptx.cuh).
+#include <type_traits>
+
 #include "fa_exp2.cuh"
 #include "fa_internal.h"
 #include "fa_ptx.cuh"
@@ -261,10 +263,12 @@ __global__ void __launch_bounds__(320, 1) bwd_dq_kernel(const __grid_constant__ 
       uint32_t u[64];
       tmem_ld64(tS, u);
       const float dk0 = static_cast<float>(kbase - q);
+      // one uniform branch on ALiBi outside the unrolled loop
+      auto p_row = [&](auto alibi_on) {
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
         float n0 = -l2, n1 = -l2;
-        if (p.alibi) {
+        if constexpr (decltype(alibi_on)::value) {
           n0 -= sl2 * fabsf(dk0 + static_cast<float>(c));
           n1 -= sl2 * fabsf(dk0 + static_cast<float>(c + 1));
         }
@@ -275,6 +279,11 @@ __global__ void __launch_bounds__(320, 1) bwd_dq_kernel(const __grid_constant__ 
         u[c] = __float_as_uint(p0);
         u[c + 1] = __float_as_uint(p1);
       }
+      };
+      if (p.alibi)
+        p_row(std::true_type{});
+      else
+        p_row(std::false_type{});
       if (edge) {   // keys past N, and (diagonal tile) keys after the query
 #pragma unroll
         for (int c = 0; c < 64; ++c) {

@@ -316,9 +316,6 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
       sv_next = p.sv[kv_base + j_start];
     }
     constexpr float kTau = FP8 ? 0.f : kRescaleTau;
-    // ALiBi: this query head's slope in log2 units
-    const bool alibi = p.alibi != nullptr;
-    const float sl2 = alibi ? p.alibi[bh % p.H] * 1.4426950408889634f : 0.f;
     float m_use = -INFINITY;
     float l = 0.f;
     bool ok = true;
@@ -339,14 +336,15 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
       // ALiBi sends every block through this path: the bias is added to the
       // scaled scores before the row maximum is taken.
       const bool masked = (CAUSAL && (jb == qi || jb * kBlockN < qi * kBlockM + kBlockM - 1 - p.window)) ||
-                          ((jb + 1) * kBlockN > p.N) || alibi;
+                          ((jb + 1) * kBlockN > p.N) || p.alibi != nullptr;
       if (masked) {
         // scaled scores with -inf where the key is hidden or past N: column i
         // is visible iff lo <= i < hi
         const int key0 = jb * kBlockN;
         const int hi = (CAUSAL ? min(row + 1, p.N) : p.N) - key0;
         const int lo = CAUSAL ? row - p.window - key0 : 0;
-        if (alibi) {   // + slope log2(e) * -|key - row|
+        if (p.alibi != nullptr) {   // + this query head's slope log2(e) * -|key - row|
+          const float sl2 = p.alibi[bh % p.H] * 1.4426950408889634f;
           const float dk = static_cast<float>(key0 - row);
 #pragma unroll
           for (int i = 0; i < 128; ++i) {
