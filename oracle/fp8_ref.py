@@ -8,7 +8,7 @@ instead of a whole-tensor scale; pre-multiplication by a random orthogonal
 Hadamard-based matrix before quantising), and [Lineage] "FA3 (2024)", idea 3
 (E4M3 inputs, block quantisation, random rotation via Hadamard).
 
-Readings where the pages are silent (each listed in the design doc):
+Readings where the pages are silent:
 
 * Block: 128 consecutive rows of one (b, h) times all d columns, one fp32
   scale per block.  (The Librarian page says 64 x d tiles; the workload under
