@@ -207,7 +207,8 @@ def build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs, deterministic=
     """The hot path as a list of (stage name, callable, FLOPs, kernel launches)."""
     state = {}
 
-    ws = torch.empty(fa.bwd_workspace_size(B, H, N, d, deterministic), dtype=torch.uint8, device=q.device)
+    ws = torch.empty(fa.bwd_workspace_size(B, H, N, d, deterministic, k.shape[1]), dtype=torch.uint8,
+                     device=q.device)
     bufs = {n: torch.empty_like(q) for n in ("o", "dq")}
     bufs.update({n: torch.empty_like(k) for n in ("dk", "dv")})
     bufs["lse"] = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
@@ -295,7 +296,10 @@ def oracle_sample(budget_s: float, B, H, N, d, causal, with_bwd: bool):
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
     except Exception:  # noqa: BLE001
         cores = os.cpu_count()
-    H_kv = WORKLOAD.get("H_kv", H)
+    g = WORKLOAD["H"] // WORKLOAD.get("H_kv", WORKLOAD["H"])   # query heads per K/V head
+    if H % g:
+        g = 1                       # a smaller warm-up shape than the workload's
+    H_kv = H // g
     key = (B, H, H_kv, N, d)
     if key not in _ORACLE_INPUTS:
         _ORACLE_INPUTS[key] = inputs.make_gqa(B, H, H_kv, N, d, WORKLOAD["seed"], with_do=True)

@@ -26,6 +26,7 @@ SIGNATURES = {
     "fa_bwd_deterministic_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int]),
     "fa_bwd_deterministic": (c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, c_int, c_int, c_int, c_int,
                                      c_float, c_int, _P, c_size_t, _P]),
+    "fa_bwd_ex_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int, c_int, c_int]),
     "fa_fwd_ex": (c_int, [_P, _P, _P, _P, _P, c_int, c_int, c_int, c_int, c_int, c_float, c_int, c_int,
                           _P, _P]),
     "fa_bwd_ex": (c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, c_int, c_int, c_int, c_int, c_int,

@@ -100,7 +100,10 @@ def fwd(q, k, v, causal: bool = False, scale: Optional[float] = None, out=None, 
     return o, lse_t
 
 
-def bwd_workspace_size(B: int, H: int, N: int, d: int, deterministic: bool = False) -> int:
+def bwd_workspace_size(B: int, H: int, N: int, d: int, deterministic: bool = False,
+                       H_kv: Optional[int] = None) -> int:
+    if H_kv is not None and H_kv != H:
+        return int(lib().fa_bwd_ex_workspace_size(B, H, H_kv, N, d, int(bool(deterministic))))
     if deterministic:
         return int(lib().fa_bwd_deterministic_workspace_size(B, H, N, d))
     return int(lib().fa_bwd_workspace_size(B, H, N, d))
@@ -126,7 +129,7 @@ def bwd(q, k, v, o, do, lse, causal: bool = False, scale: Optional[float] = None
         raise ValueError("lse must be a contiguous fp32 [B, H, N] tensor")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    ws_bytes = bwd_workspace_size(B, H, N, d, deterministic)
+    ws_bytes = bwd_workspace_size(B, H, N, d, deterministic, h_kv)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
     dq = torch.empty_like(q) if dq is None else dq

@@ -133,6 +133,24 @@ fa_status check_kv_heads(int H, int H_kv) {
   return FA_OK;
 }
 
+// CTAs sharing one (K/V head, key block) in the backward: the smallest
+// divisor S of G = H / H_kv that gives the grid about three CTAs per SM of
+// the B200 (148 SMs), so that few K/V heads (MQA) still fill the GPU; 1 when
+// the grid is large enough already.
+int kv_split_for(int B, int H, int H_kv, int N) {
+  const int G = H / H_kv;
+  const long long ctas = static_cast<long long>(B) * H_kv * ((N + 127) / 128);
+  int S = 1;
+  while (S < G && ctas * S < 3 * 148) {
+    int next = S + 1;
+    while (G % next) ++next;
+    S = next;
+  }
+  return S;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
 // Sliding window: -1 (none) or >= 0 with causal; returns the kernels' value.
 fa_status check_window(int window_left, int causal, int* window) {
   if (window_left < -1 || (window_left >= 0 && !causal)) return FA_ERR_INVALID_ARG;
@@ -211,6 +229,15 @@ extern "C" size_t fa_bwd_deterministic_workspace_size(int B, int H, int N, int d
   return (rows * sizeof(float) + 255) & ~static_cast<size_t>(255);
 }
 
+extern "C" size_t fa_bwd_ex_workspace_size(int B, int H, int H_kv, int N, int d, int deterministic) {
+  if (B < 0 || H < 0 || N < 0 || (d != 64 && d != 128) || H_kv < 1 || (H > 0 && H % H_kv)) return 0;
+  const size_t base = deterministic ? fa_bwd_deterministic_workspace_size(B, H, N, d)
+                                    : fa_bwd_workspace_size(B, H, N, d);
+  const int S = H > 0 ? kv_split_for(B, H, H_kv, N) : 1;
+  const size_t part = S > 1 ? static_cast<size_t>(S) * 2 * B * H_kv * N * d * sizeof(float) : 0;
+  return base + round256(part);
+}
+
 namespace {
 
 // Both backward variants: shared argument checks and tensor maps; the
@@ -231,8 +258,7 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))
     return FA_ERR_MISALIGNED;
-  const size_t need = deterministic ? fa_bwd_deterministic_workspace_size(B, H, N, d)
-                                    : fa_bwd_workspace_size(B, H, N, d);
+  const size_t need = fa_bwd_ex_workspace_size(B, H, H_kv, N, d, deterministic ? 1 : 0);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return FA_ERR_WORKSPACE;
   DeviceInfo* di = nullptr;
@@ -270,6 +296,12 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   p.window = window;
   p.alibi = alibi_slopes;
   p.H = H;
+  p.kv_split = kv_split_for(B, H, H_kv, N);
+  p.kv_part = p.kv_split > 1
+                  ? reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                             (deterministic ? fa_bwd_deterministic_workspace_size(B, H, N, d)
+                                                            : fa_bwd_workspace_size(B, H, N, d)))
+                  : nullptr;
   p.scale = scale;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.poly_groups = bwd_poly_groups();
@@ -277,6 +309,8 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   cudaError_t e = launch_bwd_preprocess(static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout),
                                         delta, dq_acc, rows, d, s);
   if (e == cudaSuccess) e = launch_bwd_main(p, d, causal != 0, !deterministic, s);
+  if (e == cudaSuccess && p.kv_split > 1)
+    e = launch_bwd_kv_reduce(p.kv_part, p.dv, p.dk, static_cast<long long>(B) * H_kv * N * d, p.kv_split, s);
   if (e == cudaSuccess) {
     if (deterministic)
       e = launch_bwd_dq(p, d, causal != 0, s);

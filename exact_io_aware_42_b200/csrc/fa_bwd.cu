@@ -140,6 +140,27 @@ __global__ void __launch_bounds__(256) bwd_postprocess_kernel(const float4* __re
   }
 }
 
+// ------------------------------------------------------------------ split reduction
+// dV, dK = bf16(sum over splits s = 0..S-1, in that order, of the fp32
+// partials [s][dV, dK][n]); n counts the elements of one of dV, dK.
+__global__ void __launch_bounds__(256) bwd_kv_reduce_kernel(const float4* __restrict__ part,
+                                                            uint2* __restrict__ dv, uint2* __restrict__ dk,
+                                                            long long n4, int splits) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < 2 * n4; i += stride) {
+    const long long which = i / n4, e = i % n4;
+    float4 a = part[which * n4 + e];
+    for (int s = 1; s < splits; ++s) {
+      const float4 b = part[(static_cast<long long>(s) * 2 + which) * n4 + e];
+      a.x += b.x;
+      a.y += b.y;
+      a.z += b.z;
+      a.w += b.w;
+    }
+    (which ? dk : dv)[e] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+  }
+}
+
 // ------------------------------------------------------------------ main
 __device__ __forceinline__ void st_shared_v4b(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                               uint32_t d) {
@@ -194,15 +215,20 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
   // kvh is the K/V head (flattened [B * H_kv]); with grouped K/V heads the
   // CTA visits the query blocks of its G query heads one head after the
   // other, so dK and dV sum over the group in TMEM.
-  const int kvh = blockIdx.x / p.n_kv;
+  // With kv_split = S > 1 (few K/V heads) the G query heads of a group are
+  // shared out over S CTAs per key block, G / S heads each; their dK, dV go
+  // to fp32 partials that a reduction kernel sums in split order.
+  const int kvh = blockIdx.x / (p.n_kv * p.kv_split);
+  const int split = (blockIdx.x / p.n_kv) % p.kv_split;
   const int j = blockIdx.x % p.n_kv;
+  const int g_per = p.kv_group / p.kv_split;   // query heads of this CTA
   const int i0 = CAUSAL ? j : 0;
   // Sliding window (causal): the last query block that sees a key of block j.
   const int i_last = CAUSAL ? min(p.n_q - 1, (j * 128 + 127 + p.window) / 128) : p.n_q - 1;
   const int n_i = i_last - i0 + 1;          // query blocks per query head (>= 1)
-  const int n_it = n_i * p.kv_group;
+  const int n_it = n_i * g_per;
   auto q_block = [&](int idx) { return i0 + idx % n_i; };
-  auto q_head = [&](int idx) { return kvh * p.kv_group + idx / n_i; };
+  auto q_head = [&](int idx) { return kvh * p.kv_group + split * g_per + idx / n_i; };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_KV), 1);
@@ -496,16 +522,30 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
       // writes head-dim columns [0, d/2), wg 1 [d/2, d).
       tc_fence_after();
       const size_t g = (static_cast<size_t>(kvh) * p.N + (key_ok ? key : 0)) * D;
+      const size_t kv_elems = static_cast<size_t>(p.BH / p.kv_group) * p.N * D;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {      // 0: dV, 1: dK (times scale)
         const uint32_t src = tmem + (which ? C::kColDK : C::kColDV) + lane_off;
         uint16_t* dst = (which ? p.dk : p.dv) + g;
         const float mul = which ? p.scale : 1.f;
+        // split partials: [split][dV, dK][B * H_kv, N, d] fp32
+        float* part = p.kv_part + (static_cast<size_t>(split) * 2 + which) * kv_elems + g;
 #pragma unroll
         for (int cc = 0; cc < D / 64; ++cc) {
           const int ch = wg * (D / 64) + cc;
           uint32_t u[32];
           tmem_ld32(src + 32 * ch, u);
+          if (p.kv_split > 1) {
+            if (key_ok) {
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                st_global_v4(part + 32 * ch + 4 * q, __float_as_uint(__uint_as_float(u[4 * q]) * mul),
+                             __float_as_uint(__uint_as_float(u[4 * q + 1]) * mul),
+                             __float_as_uint(__uint_as_float(u[4 * q + 2]) * mul),
+                             __float_as_uint(__uint_as_float(u[4 * q + 3]) * mul));
+            }
+            continue;
+          }
           uint32_t pk[16];
 #pragma unroll
           for (int t = 0; t < 16; ++t)
@@ -600,7 +640,8 @@ cudaError_t launch_main_impl(const BwdParams& p, cudaStream_t stream) {
   auto kern = bwd_main_kernel<D, CAUSAL, NPOLY, DQ>;
   cudaError_t e = set_smem_once<bwd_main_kernel<D, CAUSAL, NPOLY, DQ>>(C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>(p.n_kv) * static_cast<unsigned>(p.BH / p.kv_group);
+  const unsigned grid = static_cast<unsigned>(p.n_kv) * static_cast<unsigned>(p.BH / p.kv_group) *
+                        static_cast<unsigned>(p.kv_split);
   kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(p);
   return cudaGetLastError();
 }
@@ -640,6 +681,15 @@ cudaError_t launch_bwd_main(const BwdParams& p, int d, bool causal, bool with_dq
   if (d == 64)
     return causal ? launch_main_np<64, true>(p, with_dq, stream) : launch_main_np<64, false>(p, with_dq, stream);
   return causal ? launch_main_np<128, true>(p, with_dq, stream) : launch_main_np<128, false>(p, with_dq, stream);
+}
+
+cudaError_t launch_bwd_kv_reduce(const float* part, uint16_t* dv, uint16_t* dk, long long n, int splits,
+                                 cudaStream_t stream) {
+  const long long n4 = n / 4;
+  bwd_kv_reduce_kernel<<<elementwise_grid(2 * n4), 256, 0, stream>>>(
+      reinterpret_cast<const float4*>(part), reinterpret_cast<uint2*>(dv), reinterpret_cast<uint2*>(dk), n4,
+      splits);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_postprocess(const float* dq_acc, uint16_t* dq, long long n, float scale,

@@ -100,6 +100,8 @@ struct BwdParams {
   int window;           // as in FwdParams
   const float* alibi;   // as in FwdParams
   int H;
+  int kv_split;         // S: CTAs sharing one (K/V head, key block); 1 = dK, dV stored directly
+  float* kv_part;       // S > 1: fp32 partials [S][dV, dK][B * H_kv, N, d]
   float scale_log2;     // scale * log2(e)
   float scale;
   int poly_groups;      // of every 4 groups of 4 columns, how many use the FMA-pipe exp2
@@ -114,6 +116,9 @@ cudaError_t launch_bwd_preprocess(const uint16_t* o, const uint16_t* dout, float
 cudaError_t launch_bwd_main(const BwdParams& p, int d, bool causal, bool with_dq, cudaStream_t stream);
 // Deterministic dQ: one CTA per query block, key blocks in ascending order.
 cudaError_t launch_bwd_dq(const BwdParams& p, int d, bool causal, cudaStream_t stream);
+// dv, dk <- bf16(sum over the S splits of the fp32 partials); n = elements of one of dv, dk
+cudaError_t launch_bwd_kv_reduce(const float* part, uint16_t* dv, uint16_t* dk, long long n, int splits,
+                                 cudaStream_t stream);
 // dq <- bf16(scale * dq_acc)
 cudaError_t launch_bwd_postprocess(const float* dq_acc, uint16_t* dq, long long n, float scale,
                                    cudaStream_t stream);

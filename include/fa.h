@@ -202,13 +202,17 @@ fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float
  * FA_ERR_MISALIGNED), read by the kernels.  The returned L includes the bias.
  *
  * H_kv = H with window_left = -1 and alibi_slopes = NULL is exactly fa_fwd /
- * fa_bwd / fa_bwd_deterministic / fa_fwd_fp8.  fa_bwd_ex takes the workspace of
- * fa_bwd_workspace_size(B, H, N, d) (deterministic = 0) or
- * fa_bwd_deterministic_workspace_size(B, H, N, d) (deterministic != 0),
- * sized by the query heads.  In the backward one thread block per (K/V
- * head, key block) visits the query blocks of all G query heads in turn,
- * so dK and dV are summed on chip, in a fixed order.
+ * fa_bwd / fa_bwd_deterministic / fa_fwd_fp8.  fa_bwd_ex takes a workspace of
+ * fa_bwd_ex_workspace_size(B, H, H_kv, N, d, deterministic) bytes (256-byte
+ * aligned).  In the backward a thread block per (K/V head, key block)
+ * visits the query blocks of the group's query heads in turn, so dK and dV
+ * are summed on chip in a fixed order.  When B * H_kv * ceil(N / 128) is too
+ * small to fill the GPU (few K/V heads), the group is shared out over S
+ * thread blocks (S the smallest divisor of G giving about three per SM);
+ * each writes fp32 partial dK, dV to the workspace and a reduction kernel
+ * adds them in split order, so the results stay reproducible.
  */
+size_t fa_bwd_ex_workspace_size(int B, int H, int H_kv, int N, int d, int deterministic);
 fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                     int H_kv, int N, int d, float scale, int causal, int window_left,
                     const float* alibi_slopes, void* stream);

@@ -74,8 +74,12 @@ def test_gqa_matches_repeated_heads_bitwise(causal):
     assert torch.equal(o, o2) and torch.equal(lse, lse2)
     dq, dk, dv = fa.bwd(q, k, v, o, do, lse, causal=causal, deterministic=True)
     dq2, dk2, dv2 = fa.bwd(q, k_rep, v_rep, o, do, lse, causal=causal, deterministic=True)
+    # B * H_kv * ceil(N / 128) = 24 thread blocks: the group is split over
+    # several, whose fp32 partials are reduced in a fixed order
+    dq3, dk3, dv3 = fa.bwd(q, k, v, o, do, lse, causal=causal, deterministic=True)
     torch.cuda.synchronize()
     assert torch.equal(dq, dq2)
+    assert torch.equal(dq, dq3) and torch.equal(dk, dk3) and torch.equal(dv, dv3)
     for a, b in ((dk, dk2), (dv, dv2)):
         summed = b.float().reshape(B, H_kv, g, N, d).sum(dim=2)
         assert rel_rms(a.cpu(), summed.cpu()) <= 5e-3
