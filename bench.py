@@ -344,8 +344,10 @@ def run_reference(args):
         oracle_sample(0.0, 1, 1, 256, w["d"], w["causal"], with_bwd)
     vals = []
     t_all = time.perf_counter()
+    # each step a bounded sample: about 150 s of oracle work for the whole run at most
+    per_step = min(args.ref_seconds, max(0.5, 150.0 / max(1, args.steps)))
     for _ in range(args.steps):
-        vals.append(oracle_sample(args.ref_seconds, w["B"], w["H"], w["N"], w["d"], w["causal"], with_bwd))
+        vals.append(oracle_sample(per_step, w["B"], w["H"], w["N"], w["d"], w["causal"], with_bwd))
     dt = time.perf_counter() - t_all
     v = sum(x["value"] for x in vals) / len(vals)
     cpu = dict(vals[-1])

@@ -88,3 +88,36 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(lb, "_LIB", None)
     with pytest.raises(RuntimeError, match="missing"):
         lb.lib()
+
+
+@pytest.mark.parametrize("hkv,causal,window,alibi,code", [
+    (3, 0, -1, None, 1),        # H = 4 not a multiple of H_kv = 3
+    (0, 0, -1, None, 1),        # H_kv < 1
+    (2, 0, 5, None, 1),         # window without causal
+    (2, 1, -2, None, 1),        # window_left < -1
+    (2, 1, 5, A + 2, 3),        # ALiBi slopes not 4-byte aligned
+])
+def test_fwd_ex_argument_errors(L, hkv, causal, window, alibi, code):
+    assert L.fa_fwd_ex(A, A, A, A, A, 1, 4, hkv, 128, 64, 0.1, causal, window, alibi, None) == code
+
+
+def test_bwd_ex_argument_errors(L):
+    args = (A,) * 9 + (1, 4, 2, 128, 64, 0.1)
+    assert L.fa_bwd_ex(*args, 0, 7, None, 0, A, 1 << 30, None) == 1      # window without causal
+    assert L.fa_bwd_ex(*args, 1, -1, None, 0, A, 16, None) == 4          # workspace too small
+    assert L.fa_bwd_ex(*(A,) * 9, 1, 4, 3, 128, 64, 0.1, 1, -1, None, 0, A, 1 << 30, None) == 1
+
+
+def test_ex_workspace_sizes(L):
+    # H_kv = H: the plain sizes
+    assert L.fa_bwd_ex_workspace_size(4, 16, 16, 4096, 128, 0) == L.fa_bwd_workspace_size(4, 16, 4096, 128)
+    assert L.fa_bwd_ex_workspace_size(4, 16, 16, 4096, 128, 1) == \
+        L.fa_bwd_deterministic_workspace_size(4, 16, 4096, 128)
+    # MQA B4 H16 N4096: 128 (K/V head, key block) pairs, split S = 4: fp32 partials 4 x 2 x 4 x 4096 x 128
+    part = 4 * 2 * 4 * 4096 * 128 * 4
+    assert L.fa_bwd_ex_workspace_size(4, 16, 1, 4096, 128, 1) == \
+        L.fa_bwd_deterministic_workspace_size(4, 16, 4096, 128) + part
+    # GQA 32:8 at B4 N4096 fills the GPU (1024 pairs): no partials
+    assert L.fa_bwd_ex_workspace_size(4, 32, 8, 4096, 128, 0) == L.fa_bwd_workspace_size(4, 32, 4096, 128)
+    assert L.fa_bwd_ex_workspace_size(1, 4, 3, 128, 64, 0) == 0
+    assert L.fa_bwd_deterministic_workspace_size(2, 3, 100, 64) == 2560
