@@ -65,7 +65,11 @@ __device__ __forceinline__ void st_global_v4_dq(void* dst, uint32_t a, uint32_t 
                : "memory");
 }
 
-template <int D, bool CAUSAL>
+// NPOLY of every 8 column pairs take the FMA-pipe exp2 (fa_exp2.cuh), the
+// rest the SFU (d = 64 only, FA_DQ_POLY; measured on B200 the SFU-only
+// variant was fastest: the phase is bound by instruction latency, not by
+// the SFU's throughput).
+template <int D, bool CAUSAL, int NPOLY>
 __global__ void __launch_bounds__(320, 1) bwd_dq_kernel(const __grid_constant__ BwdParams p) {
   using C = DqCfg<D>;
   constexpr int NK = C::kStagesK;
@@ -275,7 +279,7 @@ __global__ void __launch_bounds__(320, 1) bwd_dq_kernel(const __grid_constant__ 
         const uint64_t x = f2_fma(f2_pack(__uint_as_float(u[c]), __uint_as_float(u[c + 1])), f2_pack(cs, cs),
                                   f2_pack(n0, n1));
         float p0, p1;
-        f2_unpack(exp2_sfu_f2(x), p0, p1);
+        f2_unpack(((c / 2) % 8 < NPOLY) ? exp2_poly_f2<3>(x) : exp2_sfu_f2(x), p0, p1);
         u[c] = __float_as_uint(p0);
         u[c + 1] = __float_as_uint(p1);
       }
@@ -343,21 +347,27 @@ __global__ void __launch_bounds__(320, 1) bwd_dq_kernel(const __grid_constant__ 
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, int NPOLY>
 cudaError_t launch_dq_impl(const BwdParams& p, cudaStream_t stream) {
   using C = DqCfg<D>;
-  cudaError_t e = set_smem_once<bwd_dq_kernel<D, CAUSAL>>(C::kSmemBytes);
+  cudaError_t e = set_smem_once<bwd_dq_kernel<D, CAUSAL, NPOLY>>(C::kSmemBytes);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(p.n_q) * static_cast<unsigned>(p.BH);
-  bwd_dq_kernel<D, CAUSAL><<<grid, C::kThreads, C::kSmemBytes, stream>>>(p);
+  bwd_dq_kernel<D, CAUSAL, NPOLY><<<grid, C::kThreads, C::kSmemBytes, stream>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_bwd_dq(const BwdParams& p, int d, bool causal, cudaStream_t stream) {
-  if (d == 64) return causal ? launch_dq_impl<64, true>(p, stream) : launch_dq_impl<64, false>(p, stream);
-  return causal ? launch_dq_impl<128, true>(p, stream) : launch_dq_impl<128, false>(p, stream);
+  // d = 64: poly_groups (FA_BWD_POLY) of 4 selects 0, 2 or 4 of 8 pairs on the polynomial
+  if (d == 64) {
+    const int np = p.dq_poly;
+    if (np == 4) return causal ? launch_dq_impl<64, true, 4>(p, stream) : launch_dq_impl<64, false, 4>(p, stream);
+    if (np == 2) return causal ? launch_dq_impl<64, true, 2>(p, stream) : launch_dq_impl<64, false, 2>(p, stream);
+    return causal ? launch_dq_impl<64, true, 0>(p, stream) : launch_dq_impl<64, false, 0>(p, stream);
+  }
+  return causal ? launch_dq_impl<128, true, 0>(p, stream) : launch_dq_impl<128, false, 0>(p, stream);
 }
 
 }  // namespace fa

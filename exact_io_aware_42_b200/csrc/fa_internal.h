@@ -101,6 +101,7 @@ struct BwdParams {
   const float* alibi;   // as in FwdParams
   int H;
   int kv_split;         // S: CTAs sharing one (K/V head, key block); 1 = dK, dV stored directly
+  int dq_poly;          // deterministic dQ kernel, d = 64: of every 8 column pairs, how many use the FMA-pipe exp2
   float* kv_part;       // S > 1: fp32 partials [S][dV, dK][B * H_kv, N, d]
   float scale_log2;     // scale * log2(e)
   float scale;
@@ -108,6 +109,7 @@ struct BwdParams {
 };
 
 constexpr int kDefaultBwdPolyGroups = 0;
+constexpr int kDefaultDqPolyPairsD64 = 0;   // measured: the polynomial share did not help (latency-bound)
 
 // D = rowsum(dO o O) per row, and dq_acc <- 0 (dq_acc == nullptr: D only).
 cudaError_t launch_bwd_preprocess(const uint16_t* o, const uint16_t* dout, float* delta,
