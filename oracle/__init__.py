@@ -41,4 +41,6 @@ from .fp8_ref import (  # noqa: F401
     quant_fp8_ref,
     dequant_fp8_ref,
     quant_fp8_per_tensor_ref,
+    quant_fp8_per_tensor_codes_ref,
+    MIN_SCALE,
 )

@@ -14,7 +14,11 @@ Readings where the pages are silent:
   scale per block.  (The Librarian page says 64 x d tiles; the workload under
   test asks for 128-row blocks.)
 * Scale: ``scale = fp32(amax) / 448`` in IEEE fp32, 448 being the largest
-  finite E4M3 magnitude; a block whose amax is 0 gets scale 1.
+  finite E4M3 magnitude; a block whose amax is 0 gets scale 1.  The scale
+  is floored at 2^-126, the smallest normal fp32: below that amax / 448 is
+  subnormal and has no finite fp32 reciprocal, which a kernel that divides
+  by multiplying with the reciprocal cannot use.  With the floor every
+  quotient still lies within [-448, 448].
 * Code: ``e4m3(fp32(x) / scale)`` -- the quotient is rounded to fp32 first
   (the kernel's precision), then to E4M3 with round-to-nearest-even and
   saturation to +-448 (OCP e4m3fn: no infinities, 0x7F/0xFF are NaN).
@@ -28,6 +32,7 @@ from __future__ import annotations
 import numpy as np
 
 E4M3_MAX = 448.0
+MIN_SCALE = np.float32(2.0 ** -126)   # smallest normal fp32
 QBLOCK_ROWS = 128
 
 
@@ -127,7 +132,7 @@ def quant_fp8_ref(x, rotate: bool, signs=None, block_rows: int = QBLOCK_ROWS):
             for j in range(nblk):
                 blk = xr[b, h, j * block_rows:(j + 1) * block_rows]
                 amax = np.float32(np.max(np.abs(blk))) if blk.size else np.float32(0)
-                sc = np.float32(1.0) if amax == 0 else np.float32(amax / np.float32(E4M3_MAX))
+                sc = np.float32(1.0) if amax == 0 else max(np.float32(amax / np.float32(E4M3_MAX)), MIN_SCALE)
                 scales[b, h, j] = sc
                 q = (blk / sc).astype(np.float32)      # IEEE fp32 quotient
                 codes[b, h, j * block_rows:(j + 1) * block_rows] = e4m3_encode_ref(q)
@@ -141,11 +146,17 @@ def dequant_fp8_ref(codes, scales, block_rows: int = QBLOCK_ROWS) -> np.ndarray:
     return vals * sc[:, :, :vals.shape[2], None]
 
 
-def quant_fp8_per_tensor_ref(x):
+def quant_fp8_per_tensor_codes_ref(x):
     """Whole-tensor E4M3 quantisation without rotation (the baseline the FA3
-    pillar improves on).  Returns fp64 dequantised values."""
+    pillar improves on): one scale for the whole tensor, the same rules as a
+    block otherwise.  Returns (codes uint8, scale fp32)."""
     x = np.asarray(x, dtype=np.float64).astype(np.float32)
-    amax = np.float32(np.max(np.abs(x)))
-    sc = np.float32(1.0) if amax == 0 else np.float32(amax / np.float32(E4M3_MAX))
-    codes = e4m3_encode_ref((x / sc).astype(np.float32))
+    amax = np.float32(np.max(np.abs(x))) if x.size else np.float32(0)
+    sc = np.float32(1.0) if amax == 0 else max(np.float32(amax / np.float32(E4M3_MAX)), MIN_SCALE)
+    return e4m3_encode_ref((x / sc).astype(np.float32)), sc
+
+
+def quant_fp8_per_tensor_ref(x):
+    """Whole-tensor E4M3 quantisation, dequantised: fp64 values code * scale."""
+    codes, sc = quant_fp8_per_tensor_codes_ref(x)
     return e4m3_decode_ref(codes) * np.float64(sc)

@@ -130,3 +130,75 @@ def test_planted_mistake_ties_away_is_caught():
     away = np.searchsorted(pos, mids, side="left").astype(np.uint8)   # always round up
     theirs = torch.tensor(mids, dtype=torch.float32).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     assert np.array_equal(ours, theirs) and not np.array_equal(away, theirs)
+
+
+def test_tiny_block_scale_is_floored_at_smallest_normal():
+    """A block whose amax / 448 would be subnormal takes the scale 2^-126
+    (the smallest normal fp32); its codes are finite, exact multiples and
+    decode back within the E4M3 bound.  The per-tensor quantiser follows the
+    same rule."""
+    x = np.zeros((1, 1, 128, 8))
+    x[0, 0, 0, :4] = [1e-37, -3e-38, 2.0 ** -130, 0.0]     # amax / 448 ~ 2.2e-40: subnormal
+    codes, scales = oracle.quant_fp8_ref(x, False)
+    assert scales[0, 0, 0] == np.float32(2.0 ** -126) == oracle.MIN_SCALE
+    vals = oracle.e4m3_decode_ref(codes)
+    assert np.all(np.isfinite(vals)) and np.all(np.abs(vals) <= 448.0)
+    deq = oracle.dequant_fp8_ref(codes, scales)
+    xf = x.astype(np.float32).astype(np.float64)
+    bound = np.maximum(np.abs(xf) * 2.0 ** -4, 2.0 ** -126 * 2.0 ** -10) * (1 + 1e-6)
+    assert np.all(np.abs(deq - xf) <= bound)
+    assert codes[0, 0, 0, 3] == 0 and np.all(codes[0, 0, 1:] == 0)
+    c1, s1 = oracle.quant_fp8_per_tensor_codes_ref(x)
+    assert s1 == oracle.MIN_SCALE and np.array_equal(c1, codes)
+    # just above the floor the plain rule applies
+    x2 = x.copy()
+    x2[0, 0, 0, 0] = 448.0 * 2.0 ** -120
+    _, s2 = oracle.quant_fp8_ref(x2, False)
+    assert s2[0, 0, 0] == np.float32(2.0 ** -120)
+
+
+def test_fp8_target_is_below_what_e4m3_can_reach_on_the_fp8_workload(record_property):
+    """The FP8 forward's 5e-2 relative-RMS target against the unquantised
+    truth is not reachable by any E4M3 kernel on the FP8 workload (N(0, 1)
+    with 0.1 % of entries x20, B2 H16 N8192 d128, non-causal): exact fp64
+    attention on the quantised values alone, with no kernel rounding at all,
+    already exceeds it.  Computed with the oracle only, on two heads and
+    every 8th query row (rows of a non-causal head are independent).
+
+    * Q, K, V block-quantised with the rotation (the kernel's inputs);
+    * only Q, K quantised, V exact (the reading that keeps P V in bf16);
+    both are above 5e-2.  The baselines: block scales without the rotation,
+    and one scale per tensor without the rotation (the FA3 pages' "baseline
+    FP8"), both worse than the rotated block format."""
+    from exact_io_aware_42_b200 import inputs
+    q, k, v = inputs.make_workload(inputs.FP8)
+    d = q.shape[-1]
+    sc = 1 / math.sqrt(d)
+    s = inputs.signs(d).numpy()
+    rows = np.arange(0, q.shape[2], 8)
+    out = {}
+    for b, h in ((0, 0), (1, 11)):
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        qf, kf, vf = (t[sl].double().numpy() for t in (q, k, v))
+
+        def deq(x, rot):
+            return oracle.dequant_fp8_ref(*oracle.quant_fp8_ref(x, rot, s))[0, 0]
+
+        def err(qq, kk, vv):
+            o, _ = oracle.attn_fwd_rows_ref(qq, kk, vv, sc, False, rows)
+            den = np.sqrt(np.mean(o_t ** 2))
+            return float(np.sqrt(np.mean((o - o_t) ** 2)) / den)
+
+        o_t, _ = oracle.attn_fwd_rows_ref(qf[0, 0], kf[0, 0], vf[0, 0], sc, False, rows)
+        qr, kr, vb = deq(qf, True), deq(kf, True), deq(vf, False)
+        pt = [oracle.quant_fp8_per_tensor_ref(x)[0, 0] for x in (qf, kf, vf)]
+        e = {"qkv_rotated": err(qr, kr, vb), "qk_rotated_v_exact": err(qr, kr, vf[0, 0]),
+             "qkv_block_naive": err(deq(qf, False), deq(kf, False), vb),
+             "qkv_tensor_naive": err(*pt)}
+        out[(b, h)] = e
+        assert e["qkv_rotated"] > 5e-2 and e["qk_rotated_v_exact"] > 5e-2, e
+        assert e["qkv_tensor_naive"] > e["qkv_rotated"] and e["qkv_block_naive"] > e["qkv_rotated"], e
+        # the rotated block format itself stays within 1.5x of the target
+        assert e["qkv_rotated"] < 7.5e-2, e
+    record_property("fp8_format_errors", {f"{b},{h}": v_ for (b, h), v_ in out.items()})
+    print({f"{b},{h}": {k_: round(x, 4) for k_, x in v_.items()} for (b, h), v_ in out.items()})
