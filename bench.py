@@ -2,22 +2,27 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step is one pass of the whole path over the workload "B4 H16 N4096 d128
-causal" (4 x 16 heads, 4096 tokens, head dim 128, bf16, synthetic N(0, 1)
-inputs from exact_io_aware_42_b200.inputs):
+The default workload is "B4 H16 N4096 d128 causal" (4 x 16 heads, 4096
+tokens, head dim 128, bf16, synthetic N(0, 1) inputs from
+exact_io_aware_42_b200.inputs).  Every row of the hot path runs in each timed
+iteration of one of two loops of K steps:
 
-  bf16 forward (O, LSE) -> bf16 backward (dQ, dK, dV) -> FP8 block
-  quantisation of Q, K (rotated) and V -> FP8 forward.
+  step (the metric's path): bf16 forward (O, LSE) -> bf16 backward (dQ, dK, dV)
+  FP8 loop:                 E4M3 block quantisation of Q, K (rotated) and V
+                            -> FP8 forward (key ``fp8`` of the JSON line)
 
-``value`` is the whole job's attention TFLOPS: algorithmic FLOPs of every
-stage (forward 4 B H N^2 d, halved when causal; backward 2.5 x forward; the
-FP8 forward counted like a forward) over the device time of the K timed steps,
-max over ranks.  Inputs (4 x 64 MiB) exceed the 126 MB L2, so no flush is
-needed between steps.  ``e2e`` is the same metric through the public API with
-the inputs copied from pinned host memory and every output copied back inside
-the timed region.  Under torchrun every rank runs its own copy of the
-workload on its own GPU (independent heads, no collective on the data path):
-weak scaling.
+``value`` is the whole job's BF16 attention TFLOPS: algorithmic FLOPs of the
+step (forward 4 B H N^2 d, halved when causal; backward 2.5 x forward) over
+the device time of the K timed steps, max over ranks; ``dtype`` is bf16.  The
+FP8 forward has its own line and its own roofline against an FP8 peak.  Inputs
+(4 x 64 MiB) exceed the 126 MB L2, so no flush is needed between steps.
+Workloads whose inputs fit in L2 are latency-bound; their steps are submitted
+as one CUDA graph (``config.submission``) so that the device time is the
+kernels', not the host's launch rate.  ``e2e`` is the step through the public
+API, eagerly, with the inputs copied from pinned host memory and every output
+copied back inside the timed region.  Under torchrun every rank runs its own
+copy of the workload on its own GPU (independent heads, no collective on the
+data path): weak scaling.
 
 ``--impl reference`` times the fp64 CPU oracle (the only other code this
 script may run) on a bounded sample of the same workload on the host cores.
@@ -25,6 +30,8 @@ script may run) on a bounded sample of the same workload on the host cores.
 ``--bwd deterministic`` times the reproducible backward (dK, dV kernel plus
 the query-block-major dQ kernel) in place of the atomic one; the ``gqa_`` /
 ``mqa_`` workloads have fewer K/V heads than query heads (grouped K/V).
+``--fwd-poly-pairs`` / ``--fwd-poly-degree`` set the forward's exp2 split for
+a measurement (fa_set_tuning); the default is the library's.
 """
 from __future__ import annotations
 
@@ -33,7 +40,6 @@ import hashlib
 import json
 import math
 import os
-import re
 import subprocess
 import sys
 import threading
@@ -63,6 +69,9 @@ def workloads():
     out["mqa_B4_H16_Hkv1_N4096_d128_causal"] = dict(B=4, H=16, H_kv=1, N=4096, d=128, causal=True, seed=6)
     # causal sliding window of 1024 keys at N = 16384: FLOPs counted over the visible pairs only
     out["window1024_B1_H16_N16384_d128"] = dict(B=1, H=16, N=16384, d=128, causal=True, seed=7, window=1024)
+    # head dim 256 (forward only: the backward is not built for d = 256)
+    out["attn_B4_H8_N4096_d256_causal"] = dict(B=4, H=8, N=4096, d=256, causal=True, seed=9, fwd_only=True)
+    out["attn_B4_H8_N4096_d256_noncausal"] = dict(B=4, H=8, N=4096, d=256, causal=False, seed=9, fwd_only=True)
     # ALiBi with the geometric slopes 2^(-8 (h + 1) / H)
     out["alibi_B4_H16_N4096_d128_causal"] = dict(B=4, H=16, N=4096, d=128, causal=True, seed=8, alibi=True)
     for name, w in out.items():
@@ -70,6 +79,7 @@ def workloads():
         w.setdefault("H_kv", w["H"])
         w.setdefault("window", None)
         w.setdefault("alibi", False)
+        w.setdefault("fwd_only", False)
     return out
 
 
@@ -119,28 +129,40 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+KERNEL_SOURCES = {
+    "fwd": ("fa_fwd.cu",),
+    "fwd256": ("fa_fwd_d256.cu",),
+    "bwd": ("fa_bwd.cu",),
+    "bwd_dq": ("fa_bwd_dq.cu",),
+    "fp8": ("fa_fp8.cu",),
+}
+
+
 def kernel_source_hash(which: str):
+    """Hash of the sources a kernel is built from (its own file and the shared
+    headers), to tell whether a stored profile was taken on this code."""
     h = hashlib.sha256()
-    main = "fa_fwd.cu" if which == "fwd" else "fa_bwd.cu"
-    for name in (main, "fa_ptx.cuh", "fa_exp2.cuh", "fa_exp2_poly.h", "fa_internal.h"):
+    for name in KERNEL_SOURCES[which] + ("fa_ptx.cuh", "fa_exp2.cuh", "fa_exp2_poly.h", "fa_internal.h"):
         with open(os.path.join(ROOT, "exact_io_aware_42_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(which: str):
-    """DRAM bytes per launch of the forward ("fwd") or backward main ("bwd")
-    kernel from the committed ncu summary, if that capture was taken on the
-    current kernel source (else None)."""
-    name = "fwd_bf16" if which == "fwd" else "bwd_main_bf16"
-    path = os.path.join(ROOT, "profiles", f"{name}_B4_H16_N4096_d128_causal.md")
+def profiled_traffic(kernel: str, workload: str, which: str):
+    """DRAM bytes (read + write) per launch of ``kernel`` on ``workload`` from
+    profiles/traffic.json, written from an ncu capture; None unless that
+    capture was taken on the current source of the kernel (``which``)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
-    text = open(path).read()
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)\s+source_sha:\s*([0-9a-f]+)", text)
-    if not m or m.group(2) != kernel_source_hash(which):
-        return None
-    return float(m.group(1))
+    with open(path) as f:
+        table = json.load(f)
+    for e in table.get("entries", []):
+        if e.get("kernel") == kernel and e.get("workload") == workload:
+            if e.get("source_sha") != kernel_source_hash(which):
+                return None
+            return float(e["dram_bytes_per_launch"])
+    return None
 
 
 class ClockSampler:
@@ -203,11 +225,12 @@ class ClockSampler:
 
 
 def build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs, deterministic=False, window=None,
-               alibi=None):
-    """The hot path as a list of (stage name, callable, FLOPs, kernel launches)."""
+               alibi=None, fwd_only=False):
+    """The hot path as two lists of (stage name, callable, FLOPs, kernel
+    launches): the bf16 step the metric is quoted on, and the FP8 rows."""
     state = {}
 
-    ws = torch.empty(fa.bwd_workspace_size(B, H, N, d, deterministic, k.shape[1]), dtype=torch.uint8,
+    ws = torch.empty(max(1, fa.bwd_workspace_size(B, H, N, d, deterministic, k.shape[1])), dtype=torch.uint8,
                      device=q.device)
     bufs = {n: torch.empty_like(q) for n in ("o", "dq")}
     bufs.update({n: torch.empty_like(k) for n in ("dk", "dv")})
@@ -236,20 +259,50 @@ def build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs, deterministic=
         fa.quant_fp8(v, None, out=q8["v"], scales=sc8["v"])
 
     def s_fwd8():
-        state["o_fp8"], state["lse_fp8"] = fa.fwd_fp8(q8["q"], q8["k"], q8["v"], sc8["q"], sc8["k"],
-                                                      sc8["v"], causal=causal, out=o8, lse=lse8,
-                                                      window=window, alibi=alibi)
+        fa.fwd_fp8(q8["q"], q8["k"], q8["v"], sc8["q"], sc8["k"], sc8["v"], causal=causal, out=o8, lse=lse8,
+                   window=window, alibi=alibi)
 
     f = fwd_flops(B, H, N, d, causal, window)
-    # backward launches: preprocess, main, and postprocess (atomic) or dQ (deterministic)
-    stages = [("fwd_bf16", s_fwd, f, 1), ("bwd_bf16", s_bwd, 2.5 * f, 3)]
-    if d == 128:   # the FP8 forward exists for d = 128 only
-        stages += [("quant_fp8", s_quant, 0.0, 3), ("fwd_fp8", s_fwd8, f, 1)]
-    return stages, state
+    # backward launches: preprocess, main, and postprocess (atomic) or dQ
+    # (deterministic), plus the split reduction when few K/V heads share out a group
+    bwd_launches = 3 + (1 if fa.bwd_workspace_size(B, H, N, d, deterministic, k.shape[1]) >
+                        fa.bwd_workspace_size(B, H, N, d, deterministic) else 0)
+    step = [("fwd_bf16", s_fwd, f, 1)]
+    if not fwd_only:
+        step.append(("bwd_bf16", s_bwd, 2.5 * f, bwd_launches))
+    fp8 = [("quant_fp8", s_quant, 0.0, 3), ("fwd_fp8", s_fwd8, f, 1)] if d == 128 else []
+    return step, fp8, state
 
 
-def time_stages(torch, stages, steps, stream):
-    """Device time of ``steps`` passes over the stages, plus per-stage event times."""
+def time_stages(torch, stages, steps, stream, graph=False):
+    """Device time of ``steps`` passes over the stages, plus per-stage event
+    times.  With ``graph`` each stage's ``steps`` calls are captured into one
+    CUDA graph first; the graphs are then replayed in stage order inside the
+    timed region, each bracketed by events on the launching stream."""
+    if graph:
+        graphs = []
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        for _, fn, _, _ in stages:
+            with torch.cuda.stream(side):
+                fn()                   # one eager call on the capture stream first
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                for _ in range(steps):
+                    fn()
+            graphs.append(g)
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in stages]
+        for (e0, e1), g in zip(ev, graphs):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        per_stage = [e0.elapsed_time(e1) / steps for e0, e1 in ev]
+        total_ms = ev[0][0].elapsed_time(ev[-1][1])
+        del graphs
+        return total_ms, per_stage
     ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in stages] for _ in range(steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -318,20 +371,13 @@ def oracle_sample(budget_s: float, B, H, N, d, causal, with_bwd: bool):
         if with_bwd:
             oracle.attn_bwd_gqa_ref(q[sl], k[kl], v[kl], do[sl], sc, causal, window=win, alibi=sl_)
             flops += 2.5 * fwd_flops(1, 1, N, d, causal, win)
-            # FP8 rows: block quantisation (Q, K rotated; V) and attention on the
-            # dequantised values
-            sg = inputs.signs(d).numpy()
-            deq = [oracle.dequant_fp8_ref(*oracle.quant_fp8_ref(x[s_].double().numpy(), rot, sg))
-                   for x, s_, rot in ((q, sl, True), (k, kl, True), (v, kl, False))]
-            oracle.attn_fwd_gqa_ref(deq[0], deq[1], deq[2], sc, causal, window=win, alibi=sl_)
-            flops += fwd_flops(1, 1, N, d, causal, win)
         heads += 1
         if time.perf_counter() - t0 >= budget_s:
             break
     dt = time.perf_counter() - t0
     return {"value": flops / dt / 1e12, "unit": "TFLOPS", "cores": int(cores), "kind": "oracle",
             "sample": f"{heads} of {B * H} heads of {WORKLOAD['name']}, fwd"
-                      + ("+bwd+fp8 quant/fwd" if with_bwd else "") + f", fp64 numpy, {dt:.1f} s"}
+                      + ("+bwd" if with_bwd else "") + f", fp64 numpy, {dt:.1f} s"}
 
 
 def run_reference(args):
@@ -339,7 +385,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     w = WORKLOAD
-    with_bwd = STAGES_WITH_BWD
+    with_bwd = not w["fwd_only"]
     for _ in range(args.warmup):
         oracle_sample(0.0, 1, 1, 256, w["d"], w["causal"], with_bwd)
     vals = []
@@ -355,18 +401,22 @@ def run_reference(args):
     line = {"metric": METRIC, "value": v, "unit": "TFLOPS", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "impl": "reference", "config": config_block(), "cpu_baseline": cpu,
+            "impl": "reference", "config": config_block(False), "cpu_baseline": cpu,
             "e2e": {"value": v, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
 METRIC = "attention fwd/bwd TFLOPS (BF16 causal+non-causal) and % of B200 tensor peak"
-STAGES_WITH_BWD = True
 BWD_MODE = "atomic"   # set in main()
 
 
-def config_block():
+def latency_bound(w) -> bool:
+    """Inputs (Q, K, V, dO) small enough to stay in the 126 MB L2."""
+    return 2 * (w["H"] + w["H_kv"]) * w["B"] * w["N"] * w["d"] * 2 <= 126e6
+
+
+def config_block(graph: bool):
     w = WORKLOAD
     in_bytes = 2 * (w["H"] + w["H_kv"]) * w["B"] * w["N"] * w["d"] * 2
     return {"workload": w["name"], "B": w["B"], "H": w["H"], "H_kv": w["H_kv"], "N": w["N"], "d": w["d"],
@@ -376,8 +426,18 @@ def config_block():
             "l2": (f"inputs (Q, K, V, dO) {in_bytes / 2**20:.0f} MiB > 126 MB L2, no flush"
                    if in_bytes > 126e6 else
                    "inputs smaller than L2: timed warm in L2 (latency-bound workload)"),
-            "step": "fwd_bf16 + bwd_bf16" + (" + quant_fp8 (Q, K rotated; V) + fwd_fp8" if w["d"] == 128 else ""),
-            "fp8": "quantisation and forward in E4M3 (kind::f8f6f4), counted at forward FLOPs"}
+            "submission": ("one CUDA graph per stage of K calls (latency-bound: device time, not host launch rate)"
+                           if graph else "eager launches through the public API"),
+            "step": ("fwd_bf16 (head dim 256: forward only)" if w["fwd_only"] else "fwd_bf16 + bwd_bf16")
+                    + " (value, ms_per_step, e2e)",
+            "fp8_loop": ("quant_fp8 (Q, K rotated; V) + fwd_fp8 in a second loop of K steps, key fp8"
+                         if w["d"] == 128 else "none (the FP8 forward is built for d = 128)"),
+            "exp2_split": {"fwd_poly_pairs": TUNING.get("fwd_poly_pairs"),
+                           "fwd_poly_degree": TUNING.get("fwd_poly_degree"),
+                           "fp8_poly_pairs": TUNING.get("fp8_poly_pairs")}}
+
+
+TUNING = {}   # effective measurement controls, filled in run_ours
 
 
 def run_ours(args):
@@ -398,13 +458,22 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
     w = WORKLOAD
     B, H, N, d, causal, H_kv = w["B"], w["H"], w["N"], w["d"], w["causal"], w["H_kv"]
+    if args.fwd_poly_pairs is not None:
+        fa.set_tuning("fwd_poly_pairs", args.fwd_poly_pairs)
+    if args.fwd_poly_degree is not None:
+        fa.set_tuning("fwd_poly_degree", args.fwd_poly_degree)
+    if args.fp8_poly_pairs is not None:
+        fa.set_tuning("fp8_poly_pairs", args.fp8_poly_pairs)
+    TUNING.update({k_: fa.get_tuning(k_, d) for k_ in ("fwd_poly_pairs", "fwd_poly_degree", "fp8_poly_pairs")})
+    graph = {"auto": latency_bound(w), "on": True, "off": False}[args.graph]
     hq, hk, hv, hdo = inputs.make_gqa(B, H, H_kv, N, d, w["seed"] + rank, with_do=True)
     signs = inputs.signs(d).to(dev)
     q, k, v, do = (t.to(dev) for t in (hq, hk, hv, hdo))
-    stages, state = build_step(fa, torch, B, H, N, d, causal, q, k, v, do, signs,
-                               deterministic=BWD_MODE == "deterministic", window=w["window"],
-                               alibi=torch.tensor(alibi_slopes(H), dtype=torch.float32, device=dev)
-                               if w["alibi"] else None)
+    stages, fp8_stages, state = build_step(
+        fa, torch, B, H, N, d, causal, q, k, v, do, signs, deterministic=BWD_MODE == "deterministic",
+        window=w["window"],
+        alibi=torch.tensor(alibi_slopes(H), dtype=torch.float32, device=dev) if w["alibi"] else None,
+        fwd_only=w["fwd_only"])
     step_flops = sum(s[2] for s in stages)
     launches_per_step = sum(s[3] for s in stages)
 
@@ -418,19 +487,24 @@ def run_ours(args):
         return reduce_max(x, dist, dev, world)
 
     for _ in range(args.warmup):
-        for s in stages:
+        for s in stages + fp8_stages:
             s[1]()
     barrier()
     with ClockSampler(local) as clk:
-        total_ms, per_stage = time_stages(torch, stages, args.steps, stream)
+        total_ms, per_stage = time_stages(torch, stages, args.steps, stream, graph)
+        barrier()
+        fp8_total_ms, fp8_per_stage = (time_stages(torch, fp8_stages, args.steps, stream, graph)
+                                       if fp8_stages else (0.0, []))
     barrier()
     fa_status = fa.get_status()
     total_ms = max_over_ranks(total_ms)
     per_stage = [max_over_ranks(x) for x in per_stage]
+    fp8_total_ms = max_over_ranks(fp8_total_ms)
+    fp8_per_stage = [max_over_ranks(x) for x in fp8_per_stage]
     ms_step = total_ms / args.steps
     value = whole_job_tflops(world, step_flops, ms_step)
 
-    # end to end through the public API, host buffers in and out
+    # end to end through the public API (eager), host buffers in and out
     pin = {n: t.pin_memory() for n, t in (("q", hq), ("k", hk), ("v", hv), ("do", hdo))}
     dev_in = {"q": q, "k": k, "v": v, "do": do}
     h2d = sum(t.numel() * t.element_size() for t in pin.values())
@@ -460,41 +534,74 @@ def run_ours(args):
     barrier()
 
     peaks, peak_src = measured_peaks()
-    idx = {st[0]: i for i, st in enumerate(stages)}
-    peak = float(peaks["bf16_tflops_sustained"])
+    burst = float(peaks["bf16_tflops"])
+    sustained = float(peaks["bf16_tflops_sustained"])
+    clocks = clk.summary()
 
-    def roof(name, kernel, nbytes):
-        ms = per_stage[idx[name]]
-        ach = stages[idx[name]][2] / (ms * 1e-3) / 1e12
-        return {"kernel": kernel, "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                "frac": ach / peak,
-                "peak_source": f"{peak_src} bf16_tflops_sustained (timed inside the step loop)",
-                "algorithmic_bytes": nbytes}
+    def roof(stage_list, times, name, kernel, nbytes, peak, peak_note, traffic):
+        i = [st[0] for st in stage_list].index(name)
+        ms = times[i]
+        ach = stage_list[i][2] / (ms * 1e-3) / 1e12
+        out = {"kernel": kernel, "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+               "frac": ach / peak, "peak_source": peak_note, "algorithmic_bytes": nbytes,
+               "ms_per_launch": ms, "traffic": traffic}
+        return out
+
+    burst_note = (f"{peak_src} bf16_tflops (burst: the timed region is short and the SM clock "
+                  f"sampled during it is {clocks.get('sm_mhz')} of {clocks.get('sm_max_mhz')} MHz)")
+    cz = "causal" if causal else "non-causal"
+    if BWD_MODE == "atomic":
+        bwd_kernel = f"bwd_main_kernel<{d}, {cz}> (+ preprocess and dQ postprocess launches in the timed call)"
+    else:
+        bwd_kernel = (f"bwd_main_kernel<{d}, {cz}, no dQ> + bwd_dq_kernel (+ preprocess) in the timed call")
+    roof_bwd = None
+    if not w["fwd_only"]:
+        roof_bwd = roof(stages, per_stage, "bwd_bf16", bwd_kernel, bwd_bytes(B, H, N, d, H_kv), burst, burst_note,
+                        profiled_traffic("bwd_main_kernel", w["name"], "bwd") if BWD_MODE == "atomic" else None)
+        roof_bwd["frac_sustained"] = roof_bwd["achieved"] / sustained
+        roof_bwd["frac_nominal_2250"] = roof_bwd["achieved"] / 2250.0
+    fwd_name = "fwd256_kernel" if d == 256 else "fwd_kernel"
+    roof_fwd = roof(stages, per_stage, "fwd_bf16", f"{fwd_name}<{d}, {cz}, bf16> (persistent)",
+                    fwd_bytes(B, H, N, d, H_kv), burst, burst_note,
+                    profiled_traffic(fwd_name, w["name"], "fwd256" if d == 256 else "fwd"))
+    roof_fwd["frac_sustained"] = roof_fwd["achieved"] / sustained
+    roof_fwd["frac_nominal_2250"] = roof_fwd["achieved"] / 2250.0
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_block(),
-        "pct_of_peak": {"measured_bf16_burst": value / world / float(peaks["bf16_tflops"]),
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_block(graph),
+        "pct_of_peak": {"measured_bf16_burst": value / world / burst,
+                        "measured_bf16_sustained": value / world / sustained,
                         "nominal_2250": value / world / 2250.0},
         "stages": {s[0]: {"ms": per_stage[i], "tflops": s[2] / (per_stage[i] * 1e-3) / 1e12}
                    for i, s in enumerate(stages)},
-        "roofline": dict(roof("bwd_bf16", (f"bwd_main_kernel<{d}, {'causal' if causal else 'non-causal'}> "
-                              "(+ pre/post kernels in the timed call)") if BWD_MODE == "atomic" else
-                              (f"bwd_main_kernel<{d}, {'causal' if causal else 'non-causal'}, no dQ> + "
-                               "bwd_dq_kernel (+ preprocess) in the timed call"), bwd_bytes(B, H, N, d, H_kv)),
-                         traffic=profiled_traffic("bwd") if (w["name"] == DEFAULT_WORKLOAD and BWD_MODE == "atomic")
-                         else None),
-        "roofline_fwd": dict(roof("fwd_bf16", f"fwd_kernel<{d}, {'causal' if causal else 'non-causal'}, bf16>",
-                                  fwd_bytes(B, H, N, d, H_kv)),
-                             traffic=profiled_traffic("fwd") if w["name"] == DEFAULT_WORKLOAD else None),
+        # the dominant kernel: the backward where the step has one, else the forward
+        "roofline": roof_bwd if roof_bwd is not None else roof_fwd,
+        "roofline_fwd": roof_fwd,
         "e2e": {"value": whole_job_tflops(world, step_flops, e2e_ms), "unit": "TFLOPS",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk.summary(),
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "submission": "eager"},
+        "gpu_launches": launches_per_step * args.steps + sum(s[3] for s in fp8_stages) * args.steps,
+        "clocks": clocks,
         "device_status": fa_status,
     }
+    if fp8_stages:
+        fp8_peak = 2.0 * burst
+        fp8_flops = sum(s[2] for s in fp8_stages)
+        rf = roof(fp8_stages, fp8_per_stage, "fwd_fp8", f"fwd_kernel<128, {cz}, e4m3>", None, fp8_peak,
+                  f"2 x {peak_src} bf16_tflops burst (nominal 2:1 ratio of dense E4M3 to bf16; no measured "
+                  "FP8 peak)", None)
+        rf["algorithmic_bytes"] = fwd_bytes(B, H, N, d, H_kv) - (B * H + 2 * B * H_kv) * N * d
+        line["fp8"] = {
+            "dtype": "e4m3 (Q, K, V, P) with fp32 accumulation", "ms_per_step": fp8_total_ms / args.steps,
+            "tflops": world * fp8_flops / (fp8_total_ms / args.steps * 1e-3) / 1e12,
+            "stages": {s[0]: {"ms": fp8_per_stage[i],
+                              "tflops": (s[2] / (fp8_per_stage[i] * 1e-3) / 1e12) if s[2] else None}
+                       for i, s in enumerate(fp8_stages)},
+            "roofline_fp8": rf,
+        }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = oracle_sample(args.ref_seconds, B, H, N, d, causal, STAGES_WITH_BWD)
+        line["cpu_baseline"] = oracle_sample(args.ref_seconds, B, H, N, d, causal, not w["fwd_only"])
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -516,6 +623,13 @@ def main():
                     help="configuration to time (default: the one the headline metric is quoted on)")
     ap.add_argument("--bwd", choices=["atomic", "deterministic"], default="atomic",
                     help="backward variant timed in the step (default: atomic dQ accumulation)")
+    ap.add_argument("--graph", choices=["auto", "on", "off"], default="auto",
+                    help="submit the timed calls as CUDA graphs (auto: for workloads whose inputs fit in L2)")
+    ap.add_argument("--fwd-poly-pairs", type=int, choices=[0, 2, 4], default=None,
+                    help="forward exp2 split for a measurement (default: the library's)")
+    ap.add_argument("--fwd-poly-degree", type=int, choices=[3, 4], default=None)
+    ap.add_argument("--fp8-poly-pairs", type=int, choices=[0, 2, 4], default=None,
+                    help="FP8 forward exp2 split for a measurement (default: the library's)")
     args = ap.parse_args()
     global WORKLOAD, BWD_MODE
     WORKLOAD = workloads()[args.workload]

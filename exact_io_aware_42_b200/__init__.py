@@ -14,5 +14,7 @@ from .api import (  # noqa: F401
     get_status,
     n_blocks,
     quant_fp8,
+    set_tuning,
+    get_tuning,
 )
 from ._lib import FaError, library_path  # noqa: F401

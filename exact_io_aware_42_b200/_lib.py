@@ -39,6 +39,9 @@ SIGNATURES = {
     "fa_fwd_fp8": (c_int, [_P, _P, _P, _P, _P, _P, _P, _P, c_int, c_int, c_int, c_int, c_float,
                            c_int, _P]),
     "fa_selftest_wait_timeout": (c_int, [_P]),
+    "fa_selftest_exp2": (c_int, [_P, _P, ctypes.c_longlong, c_int, _P]),
+    "fa_set_tuning": (c_int, [c_int, c_int]),
+    "fa_get_tuning": (c_int, [c_int, c_int]),
     "fa_get_status": (c_uint, []),
     "fa_clear_status": (None, []),
     "fa_status_string": (ctypes.c_char_p, [c_int]),
@@ -47,6 +50,10 @@ SIGNATURES = {
 STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_MISALIGNED",
           4: "FA_ERR_WORKSPACE", 5: "FA_ERR_LAUNCH", 6: "FA_ERR_PIPELINE_TIMEOUT",
           7: "FA_ERR_NO_DEVICE", 8: "FA_ERR_SCRATCH_LIMIT"}
+
+
+# fa_tune_knob values (include/fa.h)
+TUNE_FWD_POLY_PAIRS, TUNE_FWD_POLY_DEGREE, TUNE_BWD_POLY_GROUPS, TUNE_DQ_POLY_PAIRS, TUNE_FP8_POLY_PAIRS = 1, 2, 3, 4, 5
 
 
 class FaError(RuntimeError):

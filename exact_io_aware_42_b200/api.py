@@ -18,10 +18,11 @@ from typing import Optional
 
 import torch
 
-from ._lib import check, lib
+from ._lib import (TUNE_BWD_POLY_GROUPS, TUNE_DQ_POLY_PAIRS, TUNE_FP8_POLY_PAIRS, TUNE_FWD_POLY_DEGREE,
+                   TUNE_FWD_POLY_PAIRS, check, lib)
 
 __all__ = ["fwd", "bwd", "bwd_workspace_size", "bwd_noalloc", "quant_fp8", "fwd_fp8", "get_status",
-           "clear_status", "n_blocks"]
+           "clear_status", "n_blocks", "set_tuning", "get_tuning", "TUNING_KNOBS"]
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
@@ -100,6 +101,23 @@ def fwd(q, k, v, causal: bool = False, scale: Optional[float] = None, out=None, 
     return o, lse_t
 
 
+def _check_bwd_args(q, k, v, o, do, lse, dq=None, dk=None, dv=None):
+    """Shapes, dtypes and layout of the backward's tensors; returns (B, H, N, d, H_kv)."""
+    _check_bhnd("q", q, torch.bfloat16)
+    B, H, N, d = q.shape
+    h_kv = _kv_shape("k", q.shape, k)
+    for name, t in (("k", k), ("v", v), ("dk", dk), ("dv", dv)):
+        if t is not None:
+            _check_bhnd(name, t, torch.bfloat16, (B, h_kv, N, d))
+    for name, t in (("o", o), ("do", do), ("dq", dq)):
+        if t is not None:
+            _check_bhnd(name, t, torch.bfloat16, q.shape)
+    if (not lse.is_cuda or lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N)
+            or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous CUDA fp32 [B, H, N] tensor")
+    return B, H, N, d, h_kv
+
+
 def bwd_workspace_size(B: int, H: int, N: int, d: int, deterministic: bool = False,
                        H_kv: Optional[int] = None) -> int:
     if H_kv is not None and H_kv != H:
@@ -118,15 +136,7 @@ def bwd(q, k, v, o, do, lse, causal: bool = False, scale: Optional[float] = None
     ``deterministic=True`` calls fa_bwd_deterministic: bitwise reproducible
     gradients (dQ by a separate query-block-major kernel).  ``window``, ``alibi`` as in fwd."""
     wl = _window(window, causal)
-    _check_bhnd("q", q, torch.bfloat16)
-    B, H, N, d = q.shape
-    h_kv = _kv_shape("k", q.shape, k)
-    for name, t in (("k", k), ("v", v)):
-        _check_bhnd(name, t, torch.bfloat16, (B, h_kv, N, d))
-    for name, t in (("o", o), ("do", do)):
-        _check_bhnd(name, t, torch.bfloat16, q.shape)
-    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous fp32 [B, H, N] tensor")
+    B, H, N, d, h_kv = _check_bwd_args(q, k, v, o, do, lse)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     ws_bytes = bwd_workspace_size(B, H, N, d, deterministic, h_kv)
@@ -200,9 +210,11 @@ def clear_status() -> None:
 def bwd_noalloc(q, k, v, o, do, lse, causal: bool = False, scale: Optional[float] = None,
                 dq=None, dk=None, dv=None):
     """Backward with the library's built-in scratch instead of a workspace
-    (for callers that cannot allocate device memory; see fa_bwd_noalloc)."""
-    _check_bhnd("q", q, torch.bfloat16)
-    B, H, N, d = q.shape
+    (for callers that cannot allocate device memory; see fa_bwd_noalloc).
+    Every tensor is checked as in ``bwd``; K/V heads must equal H here."""
+    B, H, N, d, h_kv = _check_bwd_args(q, k, v, o, do, lse, dq, dk, dv)
+    if h_kv != H:
+        raise ValueError("bwd_noalloc takes K/V with H heads (no grouped K/V heads)")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     dq = torch.empty_like(q) if dq is None else dq
@@ -213,3 +225,19 @@ def bwd_noalloc(q, k, v, o, do, lse, causal: bool = False, scale: Optional[float
                                 _stream())
     check("fa_bwd_noalloc", code)
     return dq, dk, dv
+
+
+TUNING_KNOBS = {"fwd_poly_pairs": TUNE_FWD_POLY_PAIRS, "fwd_poly_degree": TUNE_FWD_POLY_DEGREE,
+                "bwd_poly_groups": TUNE_BWD_POLY_GROUPS, "dq_poly_pairs": TUNE_DQ_POLY_PAIRS,
+                "fp8_poly_pairs": TUNE_FP8_POLY_PAIRS}
+
+
+def set_tuning(knob: str, value: int) -> None:
+    """Measurement control (fa_set_tuning): the share of the softmax exp2 on
+    the FMA-pipe polynomial, or its degree; -1 restores the default."""
+    check("fa_set_tuning", lib().fa_set_tuning(TUNING_KNOBS[knob], int(value)))
+
+
+def get_tuning(knob: str, d: int = 128) -> int:
+    """The value of a measurement control that a call with head dim d uses now."""
+    return int(lib().fa_get_tuning(TUNING_KNOBS[knob], int(d)))

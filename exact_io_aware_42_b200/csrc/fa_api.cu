@@ -5,8 +5,8 @@
 
 #include <cmath>
 #include <cstdint>
-#include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "fa.h"
@@ -22,92 +22,106 @@ namespace {
 constexpr int kMaxN = 1 << 20;
 constexpr int kMaxBH = 1 << 20;
 constexpr int kMaxDevices = 64;
+// Work items (query-tile pairs x heads) of one forward launch: kept within int range.
+constexpr long long kMaxWorkItems = (1LL << 31) - 4096;
 
 struct DeviceInfo {
-  bool probed = false;
-  bool ok = false;
+  std::atomic<int> state{0};   // 0 not probed, 1 usable, 2 unusable (sm_100 absent)
   unsigned int* status = nullptr;
+  int sms = 0;                 // multiprocessor count
 };
 
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
-// Current device checked once: sm_100 present, status-word address, driver
-// entry point for tensor-map encoding.
+// Current device, probed once (under the lock): sm_100 present, SM count,
+// status-word address, driver entry point for tensor-map encoding.  Later
+// calls read the probed state without taking the lock.
 fa_status current_device(DeviceInfo** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     cudaGetLastError();
     return FA_ERR_NO_DEVICE;
   }
-  std::lock_guard<std::mutex> lock(g_mu);
   DeviceInfo& di = g_dev[dev];
-  if (!di.probed) {
-    di.probed = true;
-    int major = 0, minor = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
-      cudaGetLastError();
-      return FA_ERR_NO_DEVICE;
-    }
-    if (major != 10 || minor != 0) return FA_ERR_UNSUPPORTED;
-    void* addr = nullptr;
-    if (cudaGetSymbolAddress(&addr, g_status) != cudaSuccess) {
-      cudaGetLastError();
-      return FA_ERR_NO_DEVICE;
-    }
-    di.status = static_cast<unsigned int*>(addr);
-    if (!g_encode) {
-      void* fn = nullptr;
-      cudaDriverEntryPointQueryResult q;
-      if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
-                                           &q) != cudaSuccess ||
-          q != cudaDriverEntryPointSuccess || fn == nullptr) {
+  int s = di.state.load(std::memory_order_acquire);
+  if (s == 0) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    s = di.state.load(std::memory_order_relaxed);
+    if (s == 0) {
+      int major = 0, minor = 0, sms = 0;
+      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return FA_ERR_NO_DEVICE;   // not marked probed: a later call may try again
+      }
+      if (major != 10 || minor != 0) {
+        di.state.store(2, std::memory_order_release);
+        return FA_ERR_UNSUPPORTED;
+      }
+      void* addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, g_status) != cudaSuccess) {
         cudaGetLastError();
         return FA_ERR_NO_DEVICE;
       }
-      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+      if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                             &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr) {
+          cudaGetLastError();
+          return FA_ERR_NO_DEVICE;
+        }
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+      }
+      di.status = static_cast<unsigned int*>(addr);
+      di.sms = sms;
+      s = 1;
+      di.state.store(1, std::memory_order_release);
     }
-    di.ok = true;
   }
-  if (!di.ok) return FA_ERR_UNSUPPORTED;
+  if (s != 1) return FA_ERR_UNSUPPORTED;
   *out = &di;
   return FA_OK;
 }
 
-// Share of the exp2 work on the FMA pipe (pairs of 8); FA_POLY_PAIRS in the
-// environment overrides the per-d default for measurement (0, 2 or 4).
+// Measurement controls (fa_set_tuning), stored as value + 1 so that the
+// zero-initialised 0 means "the built-in default".
+std::atomic<int> g_tune[FA_TUNE_COUNT];
+
+int tune_raw(int knob) { return g_tune[knob].load(std::memory_order_relaxed) - 1; }
+
+// Share of the forward's exp2 work on the FMA pipe (pairs of 8) and the
+// polynomial's degree.
 int poly_pairs(int d) {
-  static int env = [] {
-    const char* e = std::getenv("FA_POLY_PAIRS");
-    if (!e) return -1;
-    const int x = std::atoi(e);
-    return (x == 0 || x == 2 || x == 4) ? x : -1;
-  }();
-  if (env >= 0) return env;
-  return d == 64 ? kDefaultPolyPairsD64 : kDefaultPolyPairsD128;
+  const int v = tune_raw(FA_TUNE_FWD_POLY_PAIRS);
+  if (v >= 0) return v;
+  return d == 64 ? kDefaultPolyPairsD64 : d == 256 ? kDefaultPolyPairsD256 : kDefaultPolyPairsD128;
 }
 
-// Backward P-phase exp2 share on the FMA pipe (groups of 4); FA_BWD_POLY
-// overrides the default for measurement (0, 1 or 2).
+int fp8_poly_pairs() {
+  const int v = tune_raw(FA_TUNE_FP8_POLY_PAIRS);
+  return v >= 0 ? v : kDefaultPolyPairsFp8;
+}
+
+int poly_degree() {
+  const int v = tune_raw(FA_TUNE_FWD_POLY_DEGREE);
+  return v >= 0 ? v : kDefaultPolyDegree;
+}
+
+// Backward P-phase exp2 share on the FMA pipe (groups of 4 of 16 column quads).
 int bwd_poly_groups() {
-  static int v = [] {
-    const char* e = std::getenv("FA_BWD_POLY");
-    const int x = e ? std::atoi(e) : -1;
-    return (x == 0 || x == 1 || x == 2) ? x : kDefaultBwdPolyGroups;
-  }();
-  return v;
+  const int v = tune_raw(FA_TUNE_BWD_POLY_GROUPS);
+  return v >= 0 ? v : kDefaultBwdPolyGroups;
 }
 
-// Deterministic dQ kernel at d = 64: FA_DQ_POLY in {0, 2, 4} overrides the default share.
+// Deterministic dQ kernel at d = 64: pairs of 8 on the polynomial.
 int dq_poly_pairs() {
-  const char* s = std::getenv("FA_DQ_POLY");
-  if (s && *s) {
-    const int x = std::atoi(s);
-    if (x == 0 || x == 2 || x == 4) return x;
-  }
-  return kDefaultDqPolyPairsD64;
+  const int v = tune_raw(FA_TUNE_DQ_POLY_PAIRS);
+  return v >= 0 ? v : kDefaultDqPolyPairsD64;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -115,8 +129,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // 3-D view [BH, N, d] of a contiguous [B, H, N, d] tensor, 128-byte swizzle,
 // box {box_inner elements, box_rows, 1}; out-of-range elements read as zero
 // and are skipped on store.
-bool encode_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, int d, int N,
-               int BH, int box_inner, int box_rows) {
+bool encode_3d_uncached(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, int d,
+                        int N, int BH, int box_inner, int box_rows) {
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                         static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * esize,
@@ -129,10 +143,50 @@ bool encode_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esi
   return r == CUDA_SUCCESS;
 }
 
-fa_status check_shape(int B, int H, int N, int d, float scale) {
+// A tensor map is a pure function of its arguments (address, type, extents,
+// box), so encoded maps are kept in a small per-thread cache: a repeated call
+// on the same buffers and shape copies 128 bytes instead of encoding again.
+// Nothing can go stale -- a different buffer or shape is a different key.
+struct MapKey {
+  const void* base;
+  int dt, d, N, BH, box_inner, box_rows;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && dt == o.dt && d == o.d && N == o.N && BH == o.BH &&
+           box_inner == o.box_inner && box_rows == o.box_rows;
+  }
+};
+struct MapEntry {
+  MapKey key;
+  CUtensorMap map;
+  bool valid;
+};
+constexpr int kMapCacheSlots = 64;
+thread_local MapEntry t_maps[kMapCacheSlots];
+
+bool encode_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, int d, int N,
+               int BH, int box_inner, int box_rows) {
+  const MapKey key{base, static_cast<int>(dt), d, N, BH, box_inner, box_rows};
+  uint64_t h = reinterpret_cast<uintptr_t>(base) >> 8;
+  h = h * 0x9E3779B97F4A7C15ull ^ (static_cast<uint64_t>(N) << 20) ^ (static_cast<uint64_t>(BH) << 3) ^
+      static_cast<uint64_t>(dt * 131 + d * 7 + box_inner + box_rows);
+  h *= 0xBF58476D1CE4E5B9ull;
+  MapEntry& e = t_maps[(h >> 58) & (kMapCacheSlots - 1)];
+  if (e.valid && e.key == key) {
+    *m = e.map;
+    return true;
+  }
+  if (!encode_3d_uncached(m, base, dt, esize, d, N, BH, box_inner, box_rows)) return false;
+  e.key = key;
+  e.map = *m;
+  e.valid = true;
+  return true;
+}
+
+// allow256: the bf16 forward also serves head dim 256.
+fa_status check_shape(int B, int H, int N, int d, float scale, bool allow256 = false) {
   if (B < 0 || H < 0 || N < 0) return FA_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || scale < 0.f) return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && !(allow256 && d == 256)) return FA_ERR_UNSUPPORTED;
   if (N > kMaxN || static_cast<long long>(B) * H > kMaxBH) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
@@ -144,19 +198,28 @@ fa_status check_kv_heads(int H, int H_kv) {
 }
 
 // CTAs sharing one (K/V head, key block) in the backward: the smallest
-// divisor S of G = H / H_kv that gives the grid about three CTAs per SM of
-// the B200 (148 SMs), so that few K/V heads (MQA) still fill the GPU; 1 when
-// the grid is large enough already.
-int kv_split_for(int B, int H, int H_kv, int N) {
+// divisor S of G = H / H_kv that gives the grid about three CTAs per SM, so
+// that few K/V heads (MQA) still fill the GPU; 1 when the grid is large
+// enough already.  ``sms`` is the device's multiprocessor count.
+int kv_split_for(int B, int H, int H_kv, int N, int sms) {
   const int G = H / H_kv;
   const long long ctas = static_cast<long long>(B) * H_kv * ((N + 127) / 128);
   int S = 1;
-  while (S < G && ctas * S < 3 * 148) {
+  while (S < G && ctas * S < 3LL * sms) {
     int next = S + 1;
     while (G % next) ++next;
     S = next;
   }
   return S;
+}
+
+// Multiprocessor count of the current device for sizing decisions made
+// before any launch (the workspace size query): the probed value, or 148
+// (B200) when no usable device is current.
+int current_sms() {
+  DeviceInfo* di = nullptr;
+  if (current_device(&di) == FA_OK && di->sms > 0) return di->sms;
+  return 148;
 }
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -176,7 +239,7 @@ using namespace fa;
 extern "C" fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
                                int B, int H, int H_kv, int N, int d, float scale, int causal,
                                int window_left, const float* alibi_slopes, void* stream) {
-  fa_status st = check_shape(B, H, N, d, scale);
+  fa_status st = check_shape(B, H, N, d, scale, true);
   if (reinterpret_cast<uintptr_t>(alibi_slopes) & 3u) return FA_ERR_MISALIGNED;
   if (st != FA_OK) return st;
   if (H > 0 && (st = check_kv_heads(H, H_kv)) != FA_OK) return st;
@@ -197,9 +260,10 @@ extern "C" fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void
   const int BHkv = B * H_kv;
   if (!encode_3d(&p.tm_q, q, bf, 2, d, N, BH, 64, kBlockM) ||
       !encode_3d(&p.tm_k, k, bf, 2, d, N, BHkv, 64, kBlockN) ||
-      !encode_3d(&p.tm_v, v, bf, 2, d, N, BHkv, 64, kBlockN) ||
-      !encode_3d(&p.tm_o, o, bf, 2, d, N, BH, 64, kBlockM))
+      !encode_3d(&p.tm_v, v, bf, 2, d, N, BHkv, 64, kBlockN))
     return FA_ERR_INVALID_ARG;
+  p.o = static_cast<uint16_t*>(o);
+  p.sms = di->sms;
   p.lse = lse;
   p.status = di->status;
   p.N = N;
@@ -210,10 +274,14 @@ extern "C" fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void
   p.H = H;
   p.n_kv = (N + kBlockN - 1) / kBlockN;
   p.n_pairs = ((N + kBlockM - 1) / kBlockM + 1) / 2;
+  if (static_cast<long long>(p.n_pairs) * BH > kMaxWorkItems) return FA_ERR_UNSUPPORTED;
   p.scale = scale;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.poly_pairs = poly_pairs(d);
-  cudaError_t e = launch_fwd_bf16(p, d, causal != 0, static_cast<cudaStream_t>(stream));
+  p.poly_deg = poly_degree();
+  if (d == 256 && static_cast<long long>(p.n_kv) * BH > kMaxWorkItems) return FA_ERR_UNSUPPORTED;
+  cudaError_t e = d == 256 ? launch_fwd_d256(p, causal != 0, static_cast<cudaStream_t>(stream))
+                           : launch_fwd_bf16(p, d, causal != 0, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     cudaGetLastError();
     return FA_ERR_LAUNCH;
@@ -243,7 +311,7 @@ extern "C" size_t fa_bwd_ex_workspace_size(int B, int H, int H_kv, int N, int d,
   if (B < 0 || H < 0 || N < 0 || (d != 64 && d != 128) || H_kv < 1 || (H > 0 && H % H_kv)) return 0;
   const size_t base = deterministic ? fa_bwd_deterministic_workspace_size(B, H, N, d)
                                     : fa_bwd_workspace_size(B, H, N, d);
-  const int S = H > 0 ? kv_split_for(B, H, H_kv, N) : 1;
+  const int S = H > 0 ? kv_split_for(B, H, H_kv, N, current_sms()) : 1;
   const size_t part = S > 1 ? static_cast<size_t>(S) * 2 * B * H_kv * N * d * sizeof(float) : 0;
   return base + round256(part);
 }
@@ -306,7 +374,7 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   p.window = window;
   p.alibi = alibi_slopes;
   p.H = H;
-  p.kv_split = kv_split_for(B, H, H_kv, N);
+  p.kv_split = kv_split_for(B, H, H_kv, N, di->sms);
   p.kv_part = p.kv_split > 1
                   ? reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                              (deterministic ? fa_bwd_deterministic_workspace_size(B, H, N, d)
@@ -426,9 +494,10 @@ extern "C" fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v
   const int BHkv = B * H_kv;
   if (!encode_3d(&p.tm_q, q8, u8, 1, d, N, BH, 128, kBlockM) ||
       !encode_3d(&p.tm_k, k8, u8, 1, d, N, BHkv, 128, kBlockN) ||
-      !encode_3d(&p.tm_v, v8, u8, 1, d, N, BHkv, 128, kBlockN) ||
-      !encode_3d(&p.tm_o, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, BH, 64, kBlockM))
+      !encode_3d(&p.tm_v, v8, u8, 1, d, N, BHkv, 128, kBlockN))
     return FA_ERR_INVALID_ARG;
+  p.o = static_cast<uint16_t*>(o);
+  p.sms = di->sms;
   p.lse = lse;
   p.status = di->status;
   p.sq = sq;
@@ -442,8 +511,11 @@ extern "C" fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v
   p.H = H;
   p.n_kv = (N + kBlockN - 1) / kBlockN;
   p.n_pairs = ((N + kBlockM - 1) / kBlockM + 1) / 2;
+  if (static_cast<long long>(p.n_pairs) * BH > kMaxWorkItems) return FA_ERR_UNSUPPORTED;
   p.scale = scale;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.poly_pairs = fp8_poly_pairs();
+  p.poly_deg = poly_degree();
   cudaError_t e = launch_fwd_fp8(p, causal != 0, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -457,6 +529,55 @@ extern "C" fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, 
                                 int N, int d, float scale, int causal, void* stream) {
   return fa_fwd_fp8_ex(q8, k8, v8, sq, sk, sv, o, lse, B, H, H, N, d, scale, causal, -1, nullptr,
                        stream);
+}
+
+namespace {
+
+bool tuning_value_ok(int knob, int value) {
+  if (value == -1) return true;
+  switch (knob) {
+    case FA_TUNE_FWD_POLY_PAIRS: return value == 0 || value == 2 || value == 4;
+    case FA_TUNE_FWD_POLY_DEGREE: return value == 3 || value == 4;
+    case FA_TUNE_BWD_POLY_GROUPS: return value == 0 || value == 1 || value == 2;
+    case FA_TUNE_DQ_POLY_PAIRS: return value == 0 || value == 2 || value == 4;
+    case FA_TUNE_FP8_POLY_PAIRS: return value == 0 || value == 2 || value == 4;
+    default: return false;
+  }
+}
+
+}  // namespace
+
+extern "C" fa_status fa_set_tuning(int knob, int value) {
+  if (knob <= 0 || knob >= FA_TUNE_COUNT || !tuning_value_ok(knob, value)) return FA_ERR_INVALID_ARG;
+  g_tune[knob].store(value + 1, std::memory_order_relaxed);
+  return FA_OK;
+}
+
+extern "C" int fa_get_tuning(int knob, int d) {
+  switch (knob) {
+    case FA_TUNE_FWD_POLY_PAIRS: return poly_pairs(d);
+    case FA_TUNE_FWD_POLY_DEGREE: return poly_degree();
+    case FA_TUNE_BWD_POLY_GROUPS: return bwd_poly_groups();
+    case FA_TUNE_DQ_POLY_PAIRS: return d == 64 ? dq_poly_pairs() : 0;
+    case FA_TUNE_FP8_POLY_PAIRS: return fp8_poly_pairs();
+    default: return -1;
+  }
+}
+
+extern "C" fa_status fa_selftest_exp2(const float* x, float* y, long long n, int degree, void* stream) {
+  if (n < 0 || (n & 1) || (degree != 0 && degree != 3 && degree != 4 && degree != 5))
+    return FA_ERR_INVALID_ARG;
+  if (n == 0) return FA_OK;
+  if (!x || !y) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) & 7u) return FA_ERR_MISALIGNED;
+  DeviceInfo* di = nullptr;
+  fa_status st = current_device(&di);
+  if (st != FA_OK) return st;
+  if (launch_selftest_exp2(x, y, n, degree, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+  }
+  return FA_OK;
 }
 
 extern "C" fa_status fa_selftest_wait_timeout(void* stream) {

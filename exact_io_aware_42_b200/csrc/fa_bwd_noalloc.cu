@@ -14,7 +14,10 @@
 // is only a stand-in object, not a device address.  The device address is
 // therefore looked up once per device, with that device current, through
 // cudaGetSymbolAddress, the first time this entry point runs on it; that
-// first call should come before any stream capture.
+// first call should come before any stream capture.  The address is kept
+// together with the unique id of the CUDA context it was found in: after a
+// device reset the module is loaded again into a new context, possibly at
+// another address, so a changed context id triggers a new lookup.
 //
 // All calls share the one array and it keeps the previous call's contents;
 // the part that must start at zero (the dQ accumulator) is cleared by the
@@ -22,6 +25,7 @@
 // overlap on the GPU (different streams, or different host threads without
 // ordering between them) race on the array and give wrong gradients:
 // serialise them.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -34,27 +38,67 @@ constexpr int kMaxDevicesNoAlloc = 64;
 
 static __device__ __align__(256) unsigned char g_bwd_scratch[FA_BWD_NOALLOC_SCRATCH_BYTES];
 
-std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevicesNoAlloc] = {};
+struct ScratchSlot {
+  void* addr = nullptr;
+  unsigned long long ctx_id = 0;
+};
 
-// Device address of g_bwd_scratch on the current device (looked up once).
+std::mutex g_scratch_mu;
+ScratchSlot g_scratch[kMaxDevicesNoAlloc];
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id of the current CUDA context (driver entry points looked up once;
+// 0 if unavailable, which then only disables the reset check).
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &fn, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &fn, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(fn);
+    cudaGetLastError();
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx != nullptr &&
+      get_id(ctx, &id) == CUDA_SUCCESS)
+    return id;
+  return 0;
+}
+
+// Device address of g_bwd_scratch on the current device (looked up once per
+// device and context).
 fa_status scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevicesNoAlloc) {
     cudaGetLastError();
     return FA_ERR_NO_DEVICE;
   }
+  // (Before the first runtime call on this device there may be no context
+  // yet: cudaGetSymbolAddress creates it, and the id is read after it.)
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  ScratchSlot& slot = g_scratch[dev];
+  unsigned long long id = current_context_id();
+  if (slot.addr == nullptr || (id != 0 && id != slot.ctx_id)) {
     void* ptr = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&ptr, g_bwd_scratch);
     if (e != cudaSuccess || ptr == nullptr) {
       cudaGetLastError();
       return FA_ERR_NO_DEVICE;
     }
-    g_scratch_addr[dev] = ptr;
+    slot.addr = ptr;
+    slot.ctx_id = current_context_id();
   }
-  *out = g_scratch_addr[dev];
+  *out = slot.addr;
   return FA_OK;
 }
 

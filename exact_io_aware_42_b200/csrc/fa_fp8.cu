@@ -6,7 +6,7 @@
 //
 // Per (b, h) and 128-row block of a [B, H, N, d] bf16 tensor:
 //   x <- x diag(s) H_d / sqrt(d)       (optional; H_d Sylvester, s given)
-//   scale = amax(|x| over the block) / 448   (1 if the block is all zero)
+//   scale = max(amax(|x| over the block) / 448, 2^-126)   (1 if the block is all zero)
 //   code  = e4m3_rn_satfinite(fp32(x) / scale)
 // One CTA of 128 threads per block, thread = row (d = 128: the block moves
 // through shared memory by TMA both ways; d = 64: direct loads).  The rotation is the fast
@@ -26,6 +26,12 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
+
+// Smallest block scale: the smallest normal fp32, 2^-126.  A block whose
+// amax / 448 would be subnormal takes this scale instead, so that 1 / scale
+// stays finite (a subnormal scale has no finite fp32 reciprocal and would
+// turn 0 / scale into NaN).  Every quotient is then still at most 448.
+constexpr float kMinScale = 1.17549435082228751e-38f;
 
 // x / s rounded to nearest, by Markstein's correction step (P. Markstein,
 // "Computation of elementary functions on the IBM RISC System/6000
@@ -93,7 +99,7 @@ __global__ void __launch_bounds__(128) quant_fp8_kernel(const uint4* __restrict_
   if ((r & 31) == 0) warp_max[r >> 5] = am;
   __syncthreads();
   am = fmaxf(fmaxf(warp_max[0], warp_max[1]), fmaxf(warp_max[2], warp_max[3]));
-  const float scale = am > 0.f ? __fdiv_rn(am, 448.f) : 1.f;
+  const float scale = am > 0.f ? fmaxf(__fdiv_rn(am, 448.f), kMinScale) : 1.f;
   const float inv = __frcp_rn(scale);
   if (r == 0) scales[static_cast<size_t>(bh) * nblk + blk] = scale;
   if (valid) {
@@ -190,7 +196,7 @@ __global__ void __launch_bounds__(128) quant_fp8_tma_kernel(const __grid_constan
   if ((r & 31) == 0) warp_max[r >> 5] = am;
   __syncthreads();
   am = fmaxf(fmaxf(warp_max[0], warp_max[1]), fmaxf(warp_max[2], warp_max[3]));
-  const float scale = am > 0.f ? __fdiv_rn(am, 448.f) : 1.f;
+  const float scale = am > 0.f ? fmaxf(__fdiv_rn(am, 448.f), kMinScale) : 1.f;
   const float inv = __frcp_rn(scale);
   if (r == 0) p.scales[static_cast<size_t>(bh) * p.nblk + blk] = scale;
 #pragma unroll

@@ -31,7 +31,7 @@ struct FwdParams {
   CUtensorMap tm_q;     // [BH, N, d] bf16 or e4m3, box {64 or 128 elems, 128, 1}
   CUtensorMap tm_k;
   CUtensorMap tm_v;
-  CUtensorMap tm_o;     // bf16 output, box {64, 128, 1}
+  uint16_t* o;          // bf16 output [BH, N, d]
   float* lse;           // [BH, N]
   unsigned int* status;
   const float* sq;      // fp8 only: block scales [BH, n_qblk]
@@ -49,6 +49,8 @@ struct FwdParams {
   float scale_log2;     // scale * log2(e)
   float scale;
   int poly_pairs;       // of every 8 column pairs, how many use the FMA-pipe exp2
+  int poly_deg;         // degree of that polynomial (3 or 4)
+  int sms;              // multiprocessor count: persistent grid size
 };
 
 // Default share of the softmax exp2 taken by the polynomial (of 8 column
@@ -58,10 +60,18 @@ struct FwdParams {
 // pairs on the polynomial was fastest.
 constexpr int kDefaultPolyPairsD128 = 0;
 constexpr int kDefaultPolyPairsD64 = 4;
+constexpr int kDefaultPolyPairsD256 = 0;
+constexpr int kDefaultPolyDegree = 4;
+// FP8 forward: share of the exp2 on the polynomial (pairs of 8)
+constexpr int kDefaultPolyPairsFp8 = 0;
 
 cudaError_t launch_fwd_bf16(const FwdParams& p, int d, bool causal, cudaStream_t stream);
+// Head dim 256 (one query tile per work item, K/V streamed as 64-column panels).
+cudaError_t launch_fwd_d256(const FwdParams& p, bool causal, cudaStream_t stream);
 // One CTA waiting on an mbarrier nothing arrives on (failure-path self-test).
 cudaError_t launch_selftest_wait(unsigned int* status, cudaStream_t stream);
+// y[i] = 2^x[i] by the softmax's exp2 (degree 0: the SFU; 3, 4, 5: the polynomial).
+cudaError_t launch_selftest_exp2(const float* x, float* y, long long n, int degree, cudaStream_t stream);
 // E4M3 forward (d = 128): tm_q/tm_k/tm_v are uint8 maps, sq/sk/sv block scales.
 cudaError_t launch_fwd_fp8(const FwdParams& p, bool causal, cudaStream_t stream);
 // Block quantisation of one bf16 tensor to E4M3 (signs == nullptr: no rotation).

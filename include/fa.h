@@ -133,7 +133,9 @@ fa_status fa_bwd_deterministic(const void* q, const void* k, const void* v, cons
  *    B * H * N above 65,027 rows; at d = 64, above 129,055).
  *  - The first call on a device looks up the array's device address on that
  *    device (cudaGetSymbolAddress); make that first call before any stream
- *    capture.
+ *    capture.  The address is remembered per device together with the
+ *    CUDA context it was looked up in; after a device reset (a new primary
+ *    context) the next call looks it up again.
  *  - All calls share the one array, which keeps the previous call's
  *    contents (the part that must start at zero is cleared on every call).
  *    Calls that can overlap on the GPU race on it: serialise them.
@@ -150,12 +152,20 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
  *  x8     : e4m3 [B, H, N, d] output codes.
  *  scales : fp32 [B, H, ceil(N / 128)] output, one per 128-row block:
  *           scale = amax / 448 (1 for an all-zero block).
- *  signs  : NULL for no rotation, else d fp32 values in {+1, -1}: each row
- *           is first multiplied by diag(signs) H_d / sqrt(d) (H_d the
- *           Sylvester Hadamard matrix), which leaves Q K^T unchanged when
+ *  signs  : NULL for no rotation, else d fp32 device values in {+1, -1}:
+ *           each row is first multiplied by diag(signs) H_d / sqrt(d) (H_d
+ *           the Sylvester Hadamard matrix), which leaves Q K^T unchanged when
  *           applied to both Q and K with the same signs.  V is quantised
  *           with signs = NULL.
- * code = round_to_nearest_even_satfinite(fp32(x) / scale).
+ * code = round_to_nearest_even_satfinite(fp32(x) / scale), with
+ * scale = max(amax / 448, 2^-126) for a block with a nonzero entry (the
+ * floor keeps the scale a normal fp32 number, so its reciprocal is finite).
+ * Contract note: the random signs are an argument, not drawn from a seed
+ * inside the library.  The pages ask for a random-sign Hadamard rotation but
+ * name no generator; taking the signs as data lets the caller choose the
+ * generator and lets a checker apply exactly the same rotation, and it keeps
+ * the library free of hidden random state.  (A (rotate, seed) form is this
+ * call with signs drawn by the caller from that seed.)
  */
 fa_status fa_quant_fp8(const void* x, void* x8, float* scales, int B, int H, int N, int d,
                        const float* signs, void* stream);
@@ -226,6 +236,35 @@ fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v8, const fl
                         const float* alibi_slopes, void* stream);
 
 /*
+ * Measurement controls (not part of the attention contract).  The softmax's
+ * exp2 can run on the SFU (ex2.approx) or, for a share of the elements, as a
+ * polynomial on the FMA pipe (the librarian page, "FA4 -- Blackwell's
+ * asymmetry", idea 1).  Which share is fastest was chosen by measurement per
+ * kernel and head dim; these knobs let a caller (the benchmark, the tests)
+ * re-run that measurement.  Settings are process-wide, apply to calls made
+ * after them, and are not meant to be changed while other threads launch.
+ *  FA_TUNE_FWD_POLY_PAIRS   forward bf16, of every 8 score pairs: 0, 2 or 4
+ *  FA_TUNE_FWD_POLY_DEGREE  forward polynomial degree: 3 or 4
+ *  FA_TUNE_BWD_POLY_GROUPS  backward P phase, of every 4 column groups: 0, 1 or 2
+ *  FA_TUNE_DQ_POLY_PAIRS    deterministic dQ kernel at d = 64: 0, 2 or 4
+ *  FA_TUNE_FP8_POLY_PAIRS   FP8 forward, of every 8 score pairs: 0, 2 or 4
+ *                           (same polynomial degree as the bf16 forward)
+ * value -1 restores the built-in default.  Any other value, or an unknown
+ * knob, is FA_ERR_INVALID_ARG.  fa_get_tuning returns the value a call with
+ * head dim d would use now.
+ */
+typedef enum fa_tune_knob {
+  FA_TUNE_FWD_POLY_PAIRS = 1,
+  FA_TUNE_FWD_POLY_DEGREE = 2,
+  FA_TUNE_BWD_POLY_GROUPS = 3,
+  FA_TUNE_DQ_POLY_PAIRS = 4,
+  FA_TUNE_FP8_POLY_PAIRS = 5,
+  FA_TUNE_COUNT = 6
+} fa_tune_knob;
+fa_status fa_set_tuning(int knob, int value);
+int fa_get_tuning(int knob, int d);
+
+/*
  * Device status word of the current device: FA_OK, or the first in-kernel
  * failure (FA_ERR_PIPELINE_TIMEOUT, with the failing wait's site in bits
  * 8..15) since the last fa_clear_status().  Synchronises with the device
@@ -242,6 +281,17 @@ void fa_clear_status(void);
  * usable.  Synchronise, then read fa_get_status() and fa_clear_status().
  */
 fa_status fa_selftest_wait_timeout(void* stream);
+
+/*
+ * Self-test of the softmax's exp2 (not part of the attention computation):
+ * y[i] = 2^x[i] for n (even) fp32 device values, evaluated in pairs exactly
+ * as the attention kernels evaluate it.  degree 0 is the SFU instruction;
+ * 3, 4 or 5 the FMA-pipe polynomial of that degree (Cody-Waite reduction and
+ * a minimax polynomial on [-1/2, 1/2]; inputs below -126 are clamped).  x and
+ * y are 8-byte aligned.  Lets a test measure the approximation's relative
+ * error against fp64 on a dense grid.
+ */
+fa_status fa_selftest_exp2(const float* x, float* y, long long n, int degree, void* stream);
 
 /* Static, human-readable name of a status code. */
 const char* fa_status_string(int status);

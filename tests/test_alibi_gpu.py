@@ -87,3 +87,23 @@ def test_alibi_fp8_forward():
     deq = [oracle.dequant_fp8_ref(c.cpu().numpy(), x.cpu().numpy()) for c, x in ((q8, sq), (k8, sk), (v8, sv))]
     o_ref, _ = oracle.attn_fwd_gqa_ref(deq[0], deq[1], deq[2], 1 / math.sqrt(d), True, alibi=sl.numpy())
     assert rel_rms(o.cpu(), o_ref) <= 3e-2
+
+
+@pytest.mark.parametrize("N,causal,w,H,H_kv,alibi", [(300, True, None, 4, 2, True), (513, False, None, 4, 1, True),
+                                                     (700, True, 200, 4, 2, False), (700, True, 150, 2, 2, True)])
+def test_masks_and_grouped_heads_forward_d256(N, causal, w, H, H_kv, alibi):
+    """The head-dim-256 forward takes grouped K/V heads, the sliding window
+    and ALiBi exactly like the d <= 128 kernel."""
+    fa = _fa()
+    q, k, v = inputs.make_gqa(1, H, H_kv, N, 256, seed=1400 + N)
+    sl = slopes(H) if alibi else None
+    o, lse = fa.fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, window=w,
+                    alibi=sl.cuda() if alibi else None)
+    torch.cuda.synchronize()
+    assert fa.get_status() == 0
+    o_ref, lse_ref = oracle.attn_fwd_gqa_ref(q, k, v, 1 / math.sqrt(256), causal, window=w,
+                                             alibi=sl.numpy() if alibi else None)
+    og, lg = f64(o.cpu()), f64(lse.cpu())
+    assert max_scaled_err(og, o_ref) <= O_MAX_ABS
+    assert rel_rms(og, o_ref) <= O_REL_RMS
+    assert np.max(np.abs(lg - lse_ref)) <= LSE_MAX_ABS

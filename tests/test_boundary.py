@@ -52,7 +52,8 @@ A = 4096  # a 16-byte aligned fake device address; never dereferenced on these p
 
 @pytest.mark.parametrize("args,code", [
     ((A, A, A, A, A, 1, 1, 128, 96, 0.1, 0), 2),         # d unsupported
-    ((A, A, A, A, A, 1, 1, 128, 256, 0.1, 0), 2),
+    ((A, A, A, A, A, 1, 1, 128, 192, 0.1, 0), 2),
+    ((A, A, A, A, A, 1, 1, 128, 512, 0.1, 0), 2),
     ((A, A, A, A, A, -1, 1, 128, 64, 0.1, 0), 1),        # negative size
     ((A, A, A, A, A, 1, 1, -5, 64, 0.1, 0), 1),
     ((A, A, A, A, A, 1, 1, 128, 64, -0.5, 0), 1),        # negative scale
@@ -121,3 +122,42 @@ def test_ex_workspace_sizes(L):
     assert L.fa_bwd_ex_workspace_size(4, 32, 8, 4096, 128, 0) == L.fa_bwd_workspace_size(4, 32, 4096, 128)
     assert L.fa_bwd_ex_workspace_size(1, 4, 3, 128, 64, 0) == 0
     assert L.fa_bwd_deterministic_workspace_size(2, 3, 100, 64) == 2560
+
+
+def test_tuning_controls(L):
+    """fa_set_tuning accepts only the documented values, -1 restores the
+    default, and fa_get_tuning reports what a call would use (no device
+    needed)."""
+    from exact_io_aware_42_b200._lib import (TUNE_BWD_POLY_GROUPS, TUNE_DQ_POLY_PAIRS, TUNE_FWD_POLY_DEGREE,
+                                             TUNE_FWD_POLY_PAIRS)
+    d128 = L.fa_get_tuning(TUNE_FWD_POLY_PAIRS, 128)
+    d64 = L.fa_get_tuning(TUNE_FWD_POLY_PAIRS, 64)
+    assert d128 in (0, 2, 4) and d64 in (0, 2, 4)
+    assert L.fa_set_tuning(TUNE_FWD_POLY_PAIRS, 2) == 0
+    assert L.fa_get_tuning(TUNE_FWD_POLY_PAIRS, 128) == 2 and L.fa_get_tuning(TUNE_FWD_POLY_PAIRS, 64) == 2
+    assert L.fa_set_tuning(TUNE_FWD_POLY_PAIRS, -1) == 0
+    assert L.fa_get_tuning(TUNE_FWD_POLY_PAIRS, 128) == d128
+    for knob, bad in ((TUNE_FWD_POLY_PAIRS, 3), (TUNE_FWD_POLY_DEGREE, 5), (TUNE_BWD_POLY_GROUPS, 4),
+                      (TUNE_DQ_POLY_PAIRS, 1), (0, 0), (99, 0)):
+        assert L.fa_set_tuning(knob, bad) == 1
+    assert L.fa_get_tuning(TUNE_FWD_POLY_DEGREE, 64) in (3, 4)
+    assert L.fa_get_tuning(TUNE_DQ_POLY_PAIRS, 128) == 0
+    assert L.fa_get_tuning(99, 64) == -1
+
+
+def test_exp2_selftest_argument_errors(L):
+    assert L.fa_selftest_exp2(A, A, 3, 3, None) == 1          # odd count
+    assert L.fa_selftest_exp2(A, A, 4, 6, None) == 1          # no such degree
+    assert L.fa_selftest_exp2(None, A, 4, 3, None) == 1
+    assert L.fa_selftest_exp2(A + 4, A, 4, 3, None) == 3      # not 8-byte aligned
+    assert L.fa_selftest_exp2(None, None, 0, 3, None) == 0    # empty
+
+
+def test_head_dim_256_is_forward_only(L):
+    """d = 256 is served by the bf16 forward; the backward, the quantiser and
+    the FP8 forward reject it before touching the device."""
+    assert L.fa_bwd_workspace_size(1, 1, 128, 256) == 0
+    assert L.fa_bwd(*(A,) * 9, 1, 1, 128, 256, 0.1, 0, A, 1 << 30, None) == 2
+    assert L.fa_bwd_noalloc(*(A,) * 9, 1, 1, 128, 256, 0.1, 0, None) == 2
+    assert L.fa_quant_fp8(A, A, A, 1, 1, 128, 256, None, None) == 2
+    assert L.fa_fwd_fp8(*(A,) * 8, 1, 1, 128, 256, 0.1, 0, None) == 2

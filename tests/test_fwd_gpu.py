@@ -140,3 +140,72 @@ def test_fwd_empty_and_errors():
     assert e.value.code == 2
     torch.cuda.synchronize()
     assert fa.get_status() == 0
+
+
+@pytest.fixture
+def restore_tuning():
+    yield
+    fa = _fa()
+    for knob in fa.api.TUNING_KNOBS:
+        fa.set_tuning(knob, -1)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("pairs,deg", [(0, 3), (2, 3), (4, 3), (2, 4), (4, 4)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fwd_exp2_split_variants(d, pairs, deg, causal, restore_tuning):
+    """Every exp2 split the forward can run (0, 2 or 4 of 8 score pairs on the
+    FMA-pipe polynomial, degree 3 or 4) meets the same tolerances, with
+    several tiles and a ragged tail."""
+    fa = _fa()
+    fa.set_tuning("fwd_poly_pairs", pairs)
+    fa.set_tuning("fwd_poly_degree", deg)
+    assert fa.get_tuning("fwd_poly_pairs", d) == pairs and fa.get_tuning("fwd_poly_degree", d) == deg
+    q, k, v = inputs.make_qkv(2, 2, 1000, d, seed=300 + d + pairs)
+    o, lse = run_fwd(q, k, v, causal)
+    o_ref, l_ref = oracle.attn_fwd_ref(q, k, v, 1 / math.sqrt(d), causal)
+    assert_fwd_close(o, lse, o_ref, l_ref, f"d={d} pairs={pairs} deg={deg} causal={causal}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 7, 127, 128, 129, 255, 257, 383, 513, 1000])
+def test_fwd_d256_ragged(N, causal):
+    """Head dim 256 (its own kernel: one query tile per work item, K/V in
+    64-column panels) over several tiles and ragged tails."""
+    q, k, v = inputs.make_qkv(1, 2, N, 256, seed=500 + N)
+    o, lse = run_fwd(q, k, v, causal)
+    o_ref, l_ref = oracle.attn_fwd_ref(q, k, v, 1 / math.sqrt(256), causal)
+    assert_fwd_close(o, lse, o_ref, l_ref, f"d=256 N={N} causal={causal}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fwd_d256_many_items_sampled_heads(causal):
+    """More work items than SMs (several rounds of the persistent grid)."""
+    q, k, v = inputs.make_qkv(4, 16, 2048, 256, seed=521)
+    o, lse = run_fwd(q, k, v, causal)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    for b, h in ((0, 0), (2, 9), (3, 15)):
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        o_ref, l_ref = oracle.attn_fwd_ref(q[sl], k[sl], v[sl], 1 / math.sqrt(256), causal)
+        assert_fwd_close(o[sl], lse[sl], o_ref, l_ref, f"d=256 b={b} h={h}")
+
+
+@pytest.mark.parametrize("pairs,deg", [(2, 3), (4, 4)])
+def test_fwd_d256_exp2_split(pairs, deg, restore_tuning):
+    fa = _fa()
+    fa.set_tuning("fwd_poly_pairs", pairs)
+    fa.set_tuning("fwd_poly_degree", deg)
+    q, k, v = inputs.make_qkv(1, 3, 700, 256, seed=530 + pairs)
+    for causal in (False, True):
+        o, lse = run_fwd(q, k, v, causal)
+        o_ref, l_ref = oracle.attn_fwd_ref(q, k, v, 1 / math.sqrt(256), causal)
+        assert_fwd_close(o, lse, o_ref, l_ref, f"d=256 pairs={pairs} deg={deg} causal={causal}")
+
+
+def test_fwd_d256_backward_rejected():
+    fa = _fa()
+    q, k, v = (t.cuda() for t in inputs.make_qkv(1, 1, 128, 256, seed=1))
+    o, lse = fa.fwd(q, k, v)
+    with pytest.raises(fa.FaError) as e:
+        fa.bwd(q, k, v, o, o, lse)
+    assert e.value.code == 2
