@@ -432,6 +432,7 @@ def config_block(graph: bool):
                     + " (value, ms_per_step, e2e)",
             "fp8_loop": ("quant_fp8 (Q, K rotated; V) + fwd_fp8 in a second loop of K steps, key fp8"
                          if w["d"] == 128 else "none (the FP8 forward is built for d = 128)"),
+            "bwd_pair": TUNING.get("bwd_pair"),
             "exp2_split": {"fwd_poly_pairs": TUNING.get("fwd_poly_pairs"),
                            "fwd_poly_degree": TUNING.get("fwd_poly_degree"),
                            "fp8_poly_pairs": TUNING.get("fp8_poly_pairs")}}
@@ -464,7 +465,10 @@ def run_ours(args):
         fa.set_tuning("fwd_poly_degree", args.fwd_poly_degree)
     if args.fp8_poly_pairs is not None:
         fa.set_tuning("fp8_poly_pairs", args.fp8_poly_pairs)
-    TUNING.update({k_: fa.get_tuning(k_, d) for k_ in ("fwd_poly_pairs", "fwd_poly_degree", "fp8_poly_pairs")})
+    if args.bwd_pair is not None:
+        fa.set_tuning("bwd_pair", args.bwd_pair)
+    TUNING.update({k_: fa.get_tuning(k_, d) for k_ in ("fwd_poly_pairs", "fwd_poly_degree", "fp8_poly_pairs",
+                                                       "bwd_pair")})
     graph = {"auto": latency_bound(w), "on": True, "off": False}[args.graph]
     hq, hk, hv, hdo = inputs.make_gqa(B, H, H_kv, N, d, w["seed"] + rank, with_do=True)
     signs = inputs.signs(d).to(dev)
@@ -553,7 +557,8 @@ def run_ours(args):
     if BWD_MODE == "atomic":
         bwd_kernel = f"bwd_main_kernel<{d}, {cz}> (+ preprocess and dQ postprocess launches in the timed call)"
     else:
-        bwd_kernel = (f"bwd_main_kernel<{d}, {cz}, no dQ> + bwd_dq_kernel (+ preprocess) in the timed call")
+        main = "bwd_pair_kernel (CTA pairs)" if TUNING.get("bwd_pair") == 1 else f"bwd_main_kernel<{d}, {cz}, no dQ>"
+        bwd_kernel = f"{main} + bwd_dq_kernel (+ preprocess) in the timed call"
     roof_bwd = None
     if not w["fwd_only"]:
         roof_bwd = roof(stages, per_stage, "bwd_bf16", bwd_kernel, bwd_bytes(B, H, N, d, H_kv), burst, burst_note,
@@ -628,6 +633,8 @@ def main():
     ap.add_argument("--fwd-poly-pairs", type=int, choices=[0, 2, 4], default=None,
                     help="forward exp2 split for a measurement (default: the library's)")
     ap.add_argument("--fwd-poly-degree", type=int, choices=[3, 4], default=None)
+    ap.add_argument("--bwd-pair", type=int, choices=[0, 1], default=None,
+                    help="deterministic backward at d = 128: dK, dV on CTA pairs (1) or single CTAs (0)")
     ap.add_argument("--fp8-poly-pairs", type=int, choices=[0, 2, 4], default=None,
                     help="FP8 forward exp2 split for a measurement (default: the library's)")
     args = ap.parse_args()

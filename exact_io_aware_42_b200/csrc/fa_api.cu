@@ -118,6 +118,11 @@ int bwd_poly_groups() {
   return v >= 0 ? v : kDefaultBwdPolyGroups;
 }
 
+int bwd_pair() {
+  const int v = tune_raw(FA_TUNE_BWD_PAIR);
+  return v >= 0 ? v : kDefaultBwdPair;
+}
+
 // Deterministic dQ kernel at d = 64: pairs of 8 on the polynomial.
 int dq_poly_pairs() {
   const int v = tune_raw(FA_TUNE_DQ_POLY_PAIRS);
@@ -359,6 +364,10 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   if (!deterministic &&
       !encode_3d(&p.tm_dqacc, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, N, BH, 32, 128))
     return FA_ERR_INVALID_ARG;
+  const bool pair = deterministic && d == 128 && bwd_pair() == 1;
+  if (pair && (!encode_3d(&p.tm_q64, q, bf, 2, d, N, BH, 64, 64) ||
+               !encode_3d(&p.tm_do64, dout, bf, 2, d, N, BH, 64, 64)))
+    return FA_ERR_INVALID_ARG;
   p.lse = lse;
   p.delta = delta;
   p.dq_acc = dq_acc;
@@ -387,7 +396,8 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = launch_bwd_preprocess(static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout),
                                         delta, dq_acc, rows, d, s);
-  if (e == cudaSuccess) e = launch_bwd_main(p, d, causal != 0, !deterministic, s);
+  if (e == cudaSuccess)
+    e = pair ? launch_bwd_pair(p, causal != 0, s) : launch_bwd_main(p, d, causal != 0, !deterministic, s);
   if (e == cudaSuccess && p.kv_split > 1)
     e = launch_bwd_kv_reduce(p.kv_part, p.dv, p.dk, static_cast<long long>(B) * H_kv * N * d, p.kv_split, s);
   if (e == cudaSuccess) {
@@ -541,6 +551,7 @@ bool tuning_value_ok(int knob, int value) {
     case FA_TUNE_BWD_POLY_GROUPS: return value == 0 || value == 1 || value == 2;
     case FA_TUNE_DQ_POLY_PAIRS: return value == 0 || value == 2 || value == 4;
     case FA_TUNE_FP8_POLY_PAIRS: return value == 0 || value == 2 || value == 4;
+    case FA_TUNE_BWD_PAIR: return value == 0 || value == 1;
     default: return false;
   }
 }
@@ -560,6 +571,7 @@ extern "C" int fa_get_tuning(int knob, int d) {
     case FA_TUNE_BWD_POLY_GROUPS: return bwd_poly_groups();
     case FA_TUNE_DQ_POLY_PAIRS: return d == 64 ? dq_poly_pairs() : 0;
     case FA_TUNE_FP8_POLY_PAIRS: return fp8_poly_pairs();
+    case FA_TUNE_BWD_PAIR: return d == 128 ? bwd_pair() : 0;
     default: return -1;
   }
 }

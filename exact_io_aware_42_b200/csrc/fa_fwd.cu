@@ -144,7 +144,7 @@ __device__ __forceinline__ int my_item(int k) {
 // SFU.  FP8: Q, K, V are E4M3 with per-128-row block scales and both products
 // run as kind::f8f6f4 (see the FP8 notes at the softmax).
 template <int D, bool CAUSAL, int NPOLY, int DEG, bool FP8>
-__global__ void __maxnreg__(200) fwd_kernel(const __grid_constant__ FwdParams p) {
+__global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ FwdParams p) {
   using C = FwdCfg<D, FP8>;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];

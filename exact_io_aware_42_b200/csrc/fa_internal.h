@@ -95,6 +95,8 @@ struct BwdParams {
   CUtensorMap tm_v;
   CUtensorMap tm_do;
   CUtensorMap tm_dqacc; // fp32 [BH, N, d] accumulator, box {32, 128, 1}, for TMA reduce-add
+  CUtensorMap tm_q64;   // bf16 [BH, N, d], box {64, 64, 1}: half query blocks (CTA-pair kernel)
+  CUtensorMap tm_do64;
   const float* lse;     // [BH, N], natural log
   const float* delta;   // [BH, N], D = rowsum(dO o O)
   float* dq_acc;        // [BH, N, d] fp32, zeroed by the preprocess kernel
@@ -119,6 +121,8 @@ struct BwdParams {
 };
 
 constexpr int kDefaultBwdPolyGroups = 0;
+// dK, dV of the deterministic backward at d = 128 on CTA pairs (1) or single CTAs (0)
+constexpr int kDefaultBwdPair = 0;
 constexpr int kDefaultDqPolyPairsD64 = 0;   // measured: the polynomial share did not help (latency-bound)
 
 // D = rowsum(dO o O) per row, and dq_acc <- 0 (dq_acc == nullptr: D only).
@@ -126,6 +130,8 @@ cudaError_t launch_bwd_preprocess(const uint16_t* o, const uint16_t* dout, float
                                   float* dq_acc, long long rows, int d, cudaStream_t stream);
 // with_dq: also accumulate dQ into dq_acc (atomic order); without: dK, dV only.
 cudaError_t launch_bwd_main(const BwdParams& p, int d, bool causal, bool with_dq, cudaStream_t stream);
+// dK, dV on CTA pairs (cta_group::2, d = 128; no dQ: pair with launch_bwd_dq).
+cudaError_t launch_bwd_pair(const BwdParams& p, bool causal, cudaStream_t stream);
 // Deterministic dQ: one CTA per query block, key blocks in ascending order.
 cudaError_t launch_bwd_dq(const BwdParams& p, int d, bool causal, cudaStream_t stream);
 // dv, dk <- bf16(sum over the S splits of the fp32 partials); n = elements of one of dv, dk

@@ -249,6 +249,9 @@ fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v8, const fl
  *  FA_TUNE_DQ_POLY_PAIRS    deterministic dQ kernel at d = 64: 0, 2 or 4
  *  FA_TUNE_FP8_POLY_PAIRS   FP8 forward, of every 8 score pairs: 0, 2 or 4
  *                           (same polynomial degree as the bf16 forward)
+ *  FA_TUNE_BWD_PAIR         deterministic backward at d = 128: dK, dV from
+ *                           CTA pairs sharing each product (1) or from single
+ *                           CTAs (0); same results either way
  * value -1 restores the built-in default.  Any other value, or an unknown
  * knob, is FA_ERR_INVALID_ARG.  fa_get_tuning returns the value a call with
  * head dim d would use now.
@@ -259,7 +262,8 @@ typedef enum fa_tune_knob {
   FA_TUNE_BWD_POLY_GROUPS = 3,
   FA_TUNE_DQ_POLY_PAIRS = 4,
   FA_TUNE_FP8_POLY_PAIRS = 5,
-  FA_TUNE_COUNT = 6
+  FA_TUNE_BWD_PAIR = 6,
+  FA_TUNE_COUNT = 7
 } fa_tune_knob;
 fa_status fa_set_tuning(int knob, int value);
 int fa_get_tuning(int knob, int d);
