@@ -69,9 +69,9 @@ def workloads():
     out["mqa_B4_H16_Hkv1_N4096_d128_causal"] = dict(B=4, H=16, H_kv=1, N=4096, d=128, causal=True, seed=6)
     # causal sliding window of 1024 keys at N = 16384: FLOPs counted over the visible pairs only
     out["window1024_B1_H16_N16384_d128"] = dict(B=1, H=16, N=16384, d=128, causal=True, seed=7, window=1024)
-    # head dim 256 (forward only: the backward is not built for d = 256)
-    out["attn_B4_H8_N4096_d256_causal"] = dict(B=4, H=8, N=4096, d=256, causal=True, seed=9, fwd_only=True)
-    out["attn_B4_H8_N4096_d256_noncausal"] = dict(B=4, H=8, N=4096, d=256, causal=False, seed=9, fwd_only=True)
+    # head dim 256 (its own forward kernel; backward by the d = 256 dK, dV and dQ kernels)
+    out["attn_B4_H8_N4096_d256_causal"] = dict(B=4, H=8, N=4096, d=256, causal=True, seed=9)
+    out["attn_B4_H8_N4096_d256_noncausal"] = dict(B=4, H=8, N=4096, d=256, causal=False, seed=9)
     # ALiBi with the geometric slopes 2^(-8 (h + 1) / H)
     out["alibi_B4_H16_N4096_d128_causal"] = dict(B=4, H=16, N=4096, d=128, causal=True, seed=8, alibi=True)
     for name, w in out.items():

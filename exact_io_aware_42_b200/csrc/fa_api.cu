@@ -299,21 +299,24 @@ extern "C" fa_status fa_fwd(const void* q, const void* k, const void* v, void* o
   return fa_fwd_ex(q, k, v, o, lse, B, H, H, N, d, scale, causal, -1, nullptr, stream);
 }
 
+extern "C" size_t fa_bwd_deterministic_workspace_size(int B, int H, int N, int d) {
+  if (B < 0 || H < 0 || N < 0 || (d != 64 && d != 128 && d != 256)) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  return (rows * sizeof(float) + 255) & ~static_cast<size_t>(255);
+}
+
+// d = 256 has one backward (no dQ accumulator): the same workspace as the
+// deterministic call.
 extern "C" size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (d == 256) return fa_bwd_deterministic_workspace_size(B, H, N, d);
   if (B < 0 || H < 0 || N < 0 || (d != 64 && d != 128)) return 0;
   const size_t rows = static_cast<size_t>(B) * H * N;
   auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   return up(rows * d * sizeof(float)) + up(rows * sizeof(float));
 }
 
-extern "C" size_t fa_bwd_deterministic_workspace_size(int B, int H, int N, int d) {
-  if (B < 0 || H < 0 || N < 0 || (d != 64 && d != 128)) return 0;
-  const size_t rows = static_cast<size_t>(B) * H * N;
-  return (rows * sizeof(float) + 255) & ~static_cast<size_t>(255);
-}
-
 extern "C" size_t fa_bwd_ex_workspace_size(int B, int H, int H_kv, int N, int d, int deterministic) {
-  if (B < 0 || H < 0 || N < 0 || (d != 64 && d != 128) || H_kv < 1 || (H > 0 && H % H_kv)) return 0;
+  if (B < 0 || H < 0 || N < 0 || (d != 64 && d != 128 && d != 256) || H_kv < 1 || (H > 0 && H % H_kv)) return 0;
   const size_t base = deterministic ? fa_bwd_deterministic_workspace_size(B, H, N, d)
                                     : fa_bwd_workspace_size(B, H, N, d);
   const int S = H > 0 ? kv_split_for(B, H, H_kv, N, current_sms()) : 1;
@@ -330,7 +333,7 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
                      const float* lse, void* dq, void* dk, void* dv, int B, int H, int H_kv, int N,
                      int d, float scale, int causal, int window_left, const float* alibi_slopes,
                      void* workspace, size_t workspace_bytes, void* stream, bool deterministic) {
-  fa_status st = check_shape(B, H, N, d, scale);
+  fa_status st = check_shape(B, H, N, d, scale, true);
   if (reinterpret_cast<uintptr_t>(alibi_slopes) & 3u) return FA_ERR_MISALIGNED;
   if (st != FA_OK) return st;
   if (H > 0 && (st = check_kv_heads(H, H_kv)) != FA_OK) return st;
@@ -338,6 +341,8 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   if ((st = check_window(window_left, causal, &window)) != FA_OK) return st;
   if (static_cast<long long>(B) * H * N == 0) return FA_OK;
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  // d = 256 has a single, reproducible backward (no dQ accumulator)
+  if (d == 256) deterministic = true;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))
     return FA_ERR_MISALIGNED;
@@ -365,8 +370,11 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
       !encode_3d(&p.tm_dqacc, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, N, BH, 32, 128))
     return FA_ERR_INVALID_ARG;
   const bool pair = deterministic && d == 128 && bwd_pair() == 1;
-  if (pair && (!encode_3d(&p.tm_q64, q, bf, 2, d, N, BH, 64, 64) ||
-               !encode_3d(&p.tm_do64, dout, bf, 2, d, N, BH, 64, 64)))
+  if ((pair || d == 256) && (!encode_3d(&p.tm_q64, q, bf, 2, d, N, BH, 64, 64) ||
+                             !encode_3d(&p.tm_do64, dout, bf, 2, d, N, BH, 64, 64)))
+    return FA_ERR_INVALID_ARG;
+  if (d == 256 && (!encode_3d(&p.tm_k64, k, bf, 2, d, N, BHkv, 64, 64) ||
+                   !encode_3d(&p.tm_v64, v, bf, 2, d, N, BHkv, 64, 64)))
     return FA_ERR_INVALID_ARG;
   p.lse = lse;
   p.delta = delta;
@@ -397,11 +405,15 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   cudaError_t e = launch_bwd_preprocess(static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout),
                                         delta, dq_acc, rows, d, s);
   if (e == cudaSuccess)
-    e = pair ? launch_bwd_pair(p, causal != 0, s) : launch_bwd_main(p, d, causal != 0, !deterministic, s);
+    e = d == 256 ? launch_bwd_kv256(p, causal != 0, s)
+        : pair   ? launch_bwd_pair(p, causal != 0, s)
+                 : launch_bwd_main(p, d, causal != 0, !deterministic, s);
   if (e == cudaSuccess && p.kv_split > 1)
     e = launch_bwd_kv_reduce(p.kv_part, p.dv, p.dk, static_cast<long long>(B) * H_kv * N * d, p.kv_split, s);
   if (e == cudaSuccess) {
-    if (deterministic)
+    if (d == 256)
+      e = launch_bwd_dq256(p, causal != 0, s);
+    else if (deterministic)
       e = launch_bwd_dq(p, d, causal != 0, s);
     else
       e = launch_bwd_postprocess(dq_acc, static_cast<uint16_t*>(dq), rows * d, scale, s);

@@ -86,8 +86,9 @@ enum : unsigned int { kSiteBProd = 16, kSiteBMmaKV, kSiteBMmaQ, kSiteBMmaFree, k
                       kSiteBSmS, kSiteBSmDP, kSiteBSmDQ, kSiteBDq, kSiteBEpi, kSiteBDrain, kSiteBAlign };
 
 // ------------------------------------------------------------------ preprocess
-// One group of d/8 threads per row: 16-byte loads of O and dO, fp32 dot
-// product reduced by shuffles; the same threads zero that row of dQ_acc.
+// One group of d/8 threads per row (d = 256: a whole warp): 16-byte loads of
+// O and dO, fp32 dot product reduced by shuffles; the same threads zero that
+// row of dQ_acc.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const uint4* __restrict__ o,
                                                              const uint4* __restrict__ dout,
@@ -660,6 +661,10 @@ cudaError_t launch_bwd_preprocess(const uint16_t* o, const uint16_t* dout, float
     bwd_preprocess_kernel<64><<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(o),
                                                         reinterpret_cast<const uint4*>(dout), delta,
                                                         reinterpret_cast<float4*>(dq_acc), rows);
+  else if (d == 256)
+    bwd_preprocess_kernel<256><<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(o),
+                                                         reinterpret_cast<const uint4*>(dout), delta,
+                                                         reinterpret_cast<float4*>(dq_acc), rows);
   else
     bwd_preprocess_kernel<128><<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(o),
                                                          reinterpret_cast<const uint4*>(dout), delta,

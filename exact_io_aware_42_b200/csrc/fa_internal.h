@@ -95,8 +95,10 @@ struct BwdParams {
   CUtensorMap tm_v;
   CUtensorMap tm_do;
   CUtensorMap tm_dqacc; // fp32 [BH, N, d] accumulator, box {32, 128, 1}, for TMA reduce-add
-  CUtensorMap tm_q64;   // bf16 [BH, N, d], box {64, 64, 1}: half query blocks (CTA-pair kernel)
+  CUtensorMap tm_q64;   // bf16 [BH, N, d], box {64, 64, 1}: 64-row blocks (CTA-pair and d = 256 kernels)
   CUtensorMap tm_do64;
+  CUtensorMap tm_k64;   // K, V with 64-row boxes (d = 256 dQ kernel)
+  CUtensorMap tm_v64;
   const float* lse;     // [BH, N], natural log
   const float* delta;   // [BH, N], D = rowsum(dO o O)
   float* dq_acc;        // [BH, N, d] fp32, zeroed by the preprocess kernel
@@ -132,6 +134,9 @@ cudaError_t launch_bwd_preprocess(const uint16_t* o, const uint16_t* dout, float
 cudaError_t launch_bwd_main(const BwdParams& p, int d, bool causal, bool with_dq, cudaStream_t stream);
 // dK, dV on CTA pairs (cta_group::2, d = 128; no dQ: pair with launch_bwd_dq).
 cudaError_t launch_bwd_pair(const BwdParams& p, bool causal, cudaStream_t stream);
+// Head dim 256: dK, dV per (key block, head-dim half) and dQ per query block.
+cudaError_t launch_bwd_kv256(const BwdParams& p, bool causal, cudaStream_t stream);
+cudaError_t launch_bwd_dq256(const BwdParams& p, bool causal, cudaStream_t stream);
 // Deterministic dQ: one CTA per query block, key blocks in ascending order.
 cudaError_t launch_bwd_dq(const BwdParams& p, int d, bool causal, cudaStream_t stream);
 // dv, dk <- bf16(sum over the S splits of the fp32 partials); n = elements of one of dv, dk

@@ -153,11 +153,16 @@ def test_exp2_selftest_argument_errors(L):
     assert L.fa_selftest_exp2(None, None, 0, 3, None) == 0    # empty
 
 
-def test_head_dim_256_is_forward_only(L):
-    """d = 256 is served by the bf16 forward; the backward, the quantiser and
-    the FP8 forward reject it before touching the device."""
-    assert L.fa_bwd_workspace_size(1, 1, 128, 256) == 0
-    assert L.fa_bwd(*(A,) * 9, 1, 1, 128, 256, 0.1, 0, A, 1 << 30, None) == 2
-    assert L.fa_bwd_noalloc(*(A,) * 9, 1, 1, 128, 256, 0.1, 0, None) == 2
+def test_head_dim_256_limits(L):
+    """d = 256: the forward and the backward take it (the backward is always
+    the reproducible one, with the D-only workspace); the quantiser and the
+    FP8 forward reject it before touching the device."""
+    rows = 2 * 3 * 100
+    ws = (rows * 4 + 255) // 256 * 256
+    assert L.fa_bwd_workspace_size(2, 3, 100, 256) == ws
+    assert L.fa_bwd_deterministic_workspace_size(2, 3, 100, 256) == ws
+    assert L.fa_bwd_ex_workspace_size(2, 3, 3, 100, 256, 0) == ws
+    assert L.fa_bwd(*(A,) * 9, 1, 1, 128, 256, 0.1, 0, A, 16, None) == 4      # workspace too small
     assert L.fa_quant_fp8(A, A, A, 1, 1, 128, 256, None, None) == 2
     assert L.fa_fwd_fp8(*(A,) * 8, 1, 1, 128, 256, 0.1, 0, None) == 2
+    assert L.fa_fwd(A, A, A, A, A, 1, 1, 128, 320, 0.1, 0, None) == 2
