@@ -7,9 +7,11 @@
 // gen_exp2_poly.py): Cody-Waite reduction x = n + f, n = round(x) via the
 // 1.5 * 2^23 rounding constant, f in [-1/2, 1/2]; 2^f by the Remez minimax
 // polynomial of fa_exp2_poly.h in Horner form with packed f32x2 FMAs; 2^n by
-// adding n to the exponent field.  Inputs are clamped to >= -126 so the
-// exponent never underflows; there the result is ~1e-38 instead of 0, which
-// is negligible next to the row sum (>= 1).
+// adding n to the exponent field.  Inputs are clamped to >= -125 so that
+// the result is always a normal number (at -126 the polynomial's value just
+// below 1 would land in the subnormal range, where adding n to the exponent
+// field no longer scales it); below the clamp the result is ~2.4e-38
+// instead of 0, negligible next to the row sum (>= 1).
 #pragma once
 
 #include "fa_exp2_poly.h"
@@ -24,13 +26,13 @@ __device__ __forceinline__ float exp2_coef(int k) {
   else return exp2_poly5_coef(k);
 }
 
-// 2^x for both halves of a packed pair, x <= 126.
+// 2^x for both halves of a packed pair, -125 <= x <= 126 (smaller x: 2^-125).
 template <int DEG>
 __device__ __forceinline__ uint64_t exp2_poly_f2(uint64_t x2) {
   float x0, x1;
   f2_unpack(x2, x0, x1);
-  x0 = fmaxf(x0, -126.f);
-  x1 = fmaxf(x1, -126.f);
+  x0 = fmaxf(x0, -125.f);
+  x1 = fmaxf(x1, -125.f);
   const uint64_t xc = f2_pack(x0, x1);
   const uint64_t magic = f2_pack(12582912.f, 12582912.f);    // 1.5 * 2^23
   const uint64_t t = f2_add(xc, magic);                      // round(x) in the low bits

@@ -20,7 +20,8 @@
  *  - ``stream`` is a cudaStream_t (NULL = the legacy default stream).  All
  *    calls are asynchronous on that stream.
  *  - Argument errors are returned synchronously, before any launch, and
- *    leave the outputs untouched.  Supported: d in {64, 128}; 0 <= N <=
+ *    leave the outputs untouched.  Supported: d in {64, 128, 256} for the
+ *    bf16 forward and backward, d = 128 for FP8; 0 <= N <=
  *    2^20; 0 <= B * H <= 2^20; scale finite and >= 0.  B * H * N == 0 is a
  *    valid empty problem: FA_OK, nothing launched.
  *  - Causal reading: with equal query and key lengths, key j is visible to
@@ -45,7 +46,7 @@ extern "C" {
 typedef enum fa_status {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1,      /* null pointer, negative size, bad scale     */
-  FA_ERR_UNSUPPORTED = 2,      /* d not in {64,128}, size limit, not sm_100  */
+  FA_ERR_UNSUPPORTED = 2,      /* unsupported d, size limit, not sm_100      */
   FA_ERR_MISALIGNED = 3,       /* a tensor base not 16-byte aligned          */
   FA_ERR_WORKSPACE = 4,        /* workspace null or smaller than required    */
   FA_ERR_LAUNCH = 5,           /* CUDA reported an error at launch           */
@@ -88,6 +89,9 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  * recomputation; lineage page "FA1 (2022)", idea 3).  The gradient itself is
  * the textbook one: dV = P^T dO, dP = dO V^T, D = rowsum(dO o O),
  * dS = P o (dP - D), dQ = scale dS K, dK = scale dS^T Q.
+ * At d = 256 there is one backward for both entry points: dK, dV per (key
+ * block, head-dim half) and dQ per query block, in a fixed order; its
+ * workspace is the D array only (fa_bwd_workspace_size reports that).
  */
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                  const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
@@ -130,7 +134,8 @@ fa_status fa_bwd_deterministic(const void* q, const void* k, const void* v, cons
  * library until the process exits.  Nothing is allocated or freed.
  *  - Problems whose fa_bwd_workspace_size() exceeds that size are rejected
  *    with FA_ERR_SCRATCH_LIMIT before any launch (at d = 128 that is
- *    B * H * N above 65,027 rows; at d = 64, above 129,055).
+ *    B * H * N above 65,027 rows; at d = 64, above 129,055; at d = 256,
+ *    whose backward needs only D, above 8,388,608).
  *  - The first call on a device looks up the array's device address on that
  *    device (cudaGetSymbolAddress); make that first call before any stream
  *    capture.  The address is remembered per device together with the

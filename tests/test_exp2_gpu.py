@@ -10,8 +10,10 @@ fp32, so the device error is that of the polynomial under fp32 Horner
 evaluation; the bound asserted is the stated one plus one fp32 ulp.
 
 Domain: the kernels evaluate 2^x for x <= 8 (scores minus a stale row max,
-at most the rescale threshold 8 above it); below -126 the input is clamped,
-so the grid is [-126, 8].  The default share of the forward at d = 64 uses
+at most the rescale threshold 8 above it); below -125 the polynomial's input
+is clamped (so that every result is a normal number), so the relative-error
+grid is [-125, 8] and the clamped range is checked for a negligible absolute
+value instead.  The default share of the forward at d = 64 uses
 the degree named by fa_get_tuning; its error must also meet the 1e-5 budget
 derived from the LSE tolerance (an error e on the p values that feed the
 row sum moves L by at most e).
@@ -31,13 +33,13 @@ ULP = 2.0 ** -23
 def _grid():
     # every fp32 value spacing matters near the reduction's integer seams, so
     # take a dense uniform grid plus the points just around every integer
-    g = np.linspace(-126.0, 8.0, 1 << 22, dtype=np.float64)
-    ints = np.arange(-126, 9, dtype=np.float64)
+    g = np.linspace(-125.0, 8.0, 1 << 22, dtype=np.float64)
+    ints = np.arange(-125, 9, dtype=np.float64)
     seams = np.concatenate([ints, ints + 0.5, ints - 0.5])
     seams = np.concatenate([seams, np.nextafter(seams.astype(np.float32), np.float32(-200)),
                             np.nextafter(seams.astype(np.float32), np.float32(200))])
     x = np.concatenate([g, seams]).astype(np.float32)
-    x = x[(x >= -126.0) & (x <= 8.0)]
+    x = x[(x >= -125.0) & (x <= 8.0)]
     if x.size % 2:
         x = x[:-1]
     return x
@@ -66,6 +68,15 @@ def test_poly_exp2_relative_error_on_dense_grid(degree, record_property):
     assert worst <= STATED[degree] + ULP, worst
     # it is a real approximation of that order, not an exact routine
     assert worst >= STATED[degree] * 0.5
+
+
+@pytest.mark.parametrize("degree", [3, 4, 5])
+def test_poly_exp2_below_the_clamp_is_negligible(degree):
+    """x < -125 returns about 2^-125 (~2.4e-38): no NaN, no infinity, nothing
+    that matters next to a softmax row sum of at least 1."""
+    x = np.concatenate([np.linspace(-400.0, -125.0, 4096), [-np.inf, -1e30]]).astype(np.float32)
+    y = _eval(x, degree)
+    assert np.all(np.isfinite(y)) and np.all(y >= 0) and np.all(y <= 2.0 ** -124)
 
 
 def test_sfu_exp2_relative_error():
