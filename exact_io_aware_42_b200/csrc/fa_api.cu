@@ -118,6 +118,16 @@ int bwd_poly_groups() {
   return v >= 0 ? v : kDefaultBwdPolyGroups;
 }
 
+int fwd_split_pv() {
+  const int v = tune_raw(FA_TUNE_FWD_SPLIT_PV);
+  return v >= 0 ? v : kDefaultFwdSplitPv;
+}
+
+int fwd_persistent() {
+  const int v = tune_raw(FA_TUNE_FWD_PERSISTENT);
+  return v >= 0 ? v : kDefaultFwdPersistent;
+}
+
 int bwd_pair() {
   const int v = tune_raw(FA_TUNE_BWD_PAIR);
   return v >= 0 ? v : kDefaultBwdPair;
@@ -269,6 +279,8 @@ extern "C" fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void
     return FA_ERR_INVALID_ARG;
   p.o = static_cast<uint16_t*>(o);
   p.sms = di->sms;
+  p.split_pv = fwd_split_pv();
+  p.persistent = fwd_persistent();
   p.lse = lse;
   p.status = di->status;
   p.N = N;
@@ -520,6 +532,8 @@ extern "C" fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v
     return FA_ERR_INVALID_ARG;
   p.o = static_cast<uint16_t*>(o);
   p.sms = di->sms;
+  p.split_pv = fwd_split_pv();
+  p.persistent = fwd_persistent();
   p.lse = lse;
   p.status = di->status;
   p.sq = sq;
@@ -564,6 +578,8 @@ bool tuning_value_ok(int knob, int value) {
     case FA_TUNE_DQ_POLY_PAIRS: return value == 0 || value == 2 || value == 4;
     case FA_TUNE_FP8_POLY_PAIRS: return value == 0 || value == 2 || value == 4;
     case FA_TUNE_BWD_PAIR: return value == 0 || value == 1;
+    case FA_TUNE_FWD_SPLIT_PV: return value == 0 || value == 1;
+    case FA_TUNE_FWD_PERSISTENT: return value == 0 || value == 1;
     default: return false;
   }
 }
@@ -584,6 +600,8 @@ extern "C" int fa_get_tuning(int knob, int d) {
     case FA_TUNE_DQ_POLY_PAIRS: return d == 64 ? dq_poly_pairs() : 0;
     case FA_TUNE_FP8_POLY_PAIRS: return fp8_poly_pairs();
     case FA_TUNE_BWD_PAIR: return d == 128 ? bwd_pair() : 0;
+    case FA_TUNE_FWD_SPLIT_PV: return fwd_split_pv();
+    case FA_TUNE_FWD_PERSISTENT: return fwd_persistent();
     default: return -1;
   }
 }

@@ -41,10 +41,12 @@ constexpr float kMinScale = 1.17549435082228751e-38f;
 // quotients here outside that range are below 2^-126 in magnitude, which
 // round to E4M3 zero either way.  Checked bit for bit against IEEE division
 // by the quantisation tests.
+// s > 0, so the quotient has the sign of x; copysignf restores it where the
+// correction step's sum of zeros would give +0 for x = -0.
 __device__ __forceinline__ float div_rn(float x, float s, float y) {
   const float q0 = x * y;
   const float r = fmaf(-q0, s, x);
-  return fmaf(r, y, q0);
+  return copysignf(fmaf(r, y, q0), x);
 }
 
 template <int D, bool ROT>

@@ -281,11 +281,16 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
       int g[2] = {0, 0};   // P V products issued per tile (all items): the P barriers' phase
       // returns false if a wait gave up
       auto issue_pv = [&](int t, uint32_t v_addr, bool acc) -> bool {
-        if (!mbar_wait(bar(bar_p<NS>(t)), g[t] & 1, ab, kSiteMmaP)) return false;
-        tc_fence_after();
-        issue_pv_half(t, v_addr, acc, 0);
+        // split: the first half as soon as it is in TMEM; otherwise both
+        // halves once all of P is (bar_ph completes after bar_p)
+        if (p.split_pv) {
+          if (!mbar_wait(bar(bar_p<NS>(t)), g[t] & 1, ab, kSiteMmaP)) return false;
+          tc_fence_after();
+          issue_pv_half(t, v_addr, acc, 0);
+        }
         if (!mbar_wait(bar(bar_ph<NS>(t)), g[t] & 1, ab, kSiteMmaP)) return false;
         tc_fence_after();
+        if (!p.split_pv) issue_pv_half(t, v_addr, acc, 0);
         issue_pv_half(t, v_addr, acc, 1);
         tc_commit(bar(bar_pv<NS>(t)));
         ++g[t];
@@ -596,9 +601,10 @@ cudaError_t launch_impl(const FwdParams& p, cudaStream_t stream) {
   auto kern = fwd_kernel<D, CAUSAL, NPOLY, DEG, FP8>;
   cudaError_t e = set_smem_once<fwd_kernel<D, CAUSAL, NPOLY, DEG, FP8>>(C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  // persistent: one CTA per SM (at most one per work item)
+  // persistent: one CTA per SM (at most one per work item); otherwise one
+  // CTA per work item, scheduled by the hardware in item order
   const long long items = static_cast<long long>(p.n_pairs) * p.BH;
-  const unsigned grid = static_cast<unsigned>(items < p.sms ? items : p.sms);
+  const unsigned grid = static_cast<unsigned>(p.persistent && items > p.sms ? p.sms : items);
   kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(p);
   return cudaGetLastError();
 }

@@ -444,7 +444,7 @@ cudaError_t launch256(const FwdParams& p, cudaStream_t stream) {
   cudaError_t e = set_smem_once<fwd256_kernel<CAUSAL, NPOLY, DEG>>(F256::kSmemBytes);
   if (e != cudaSuccess) return e;
   const long long items = static_cast<long long>(p.n_kv) * p.BH;
-  const unsigned grid = static_cast<unsigned>(items < p.sms ? items : p.sms);
+  const unsigned grid = static_cast<unsigned>(p.persistent && items > p.sms ? p.sms : items);
   fwd256_kernel<CAUSAL, NPOLY, DEG><<<grid, F256::kThreads, F256::kSmemBytes, stream>>>(p);
   return cudaGetLastError();
 }

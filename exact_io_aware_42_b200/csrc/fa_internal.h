@@ -51,6 +51,8 @@ struct FwdParams {
   int poly_pairs;       // of every 8 column pairs, how many use the FMA-pipe exp2
   int poly_deg;         // degree of that polynomial (3 or 4)
   int sms;              // multiprocessor count: persistent grid size
+  int split_pv;         // 1: P V issued in two 64-key halves as P arrives; 0: after all of P
+  int persistent;       // 1: grid of min(items, SMs) CTAs; 0: one CTA per work item
 };
 
 // Default share of the softmax exp2 taken by the polynomial (of 8 column
@@ -62,6 +64,8 @@ constexpr int kDefaultPolyPairsD128 = 0;
 constexpr int kDefaultPolyPairsD64 = 4;
 constexpr int kDefaultPolyPairsD256 = 0;
 constexpr int kDefaultPolyDegree = 4;
+constexpr int kDefaultFwdSplitPv = 1;
+constexpr int kDefaultFwdPersistent = 1;
 // FP8 forward: share of the exp2 on the polynomial (pairs of 8)
 constexpr int kDefaultPolyPairsFp8 = 0;
 

@@ -257,6 +257,10 @@ fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v8, const fl
  *  FA_TUNE_BWD_PAIR         deterministic backward at d = 128: dK, dV from
  *                           CTA pairs sharing each product (1) or from single
  *                           CTAs (0); same results either way
+ *  FA_TUNE_FWD_SPLIT_PV     forward: P V issued in two halves as P arrives (1)
+ *                           or after all of P (0)
+ *  FA_TUNE_FWD_PERSISTENT   forward: one CTA per SM walking the work items (1)
+ *                           or one CTA per work item (0)
  * value -1 restores the built-in default.  Any other value, or an unknown
  * knob, is FA_ERR_INVALID_ARG.  fa_get_tuning returns the value a call with
  * head dim d would use now.
@@ -268,7 +272,9 @@ typedef enum fa_tune_knob {
   FA_TUNE_DQ_POLY_PAIRS = 4,
   FA_TUNE_FP8_POLY_PAIRS = 5,
   FA_TUNE_BWD_PAIR = 6,
-  FA_TUNE_COUNT = 7
+  FA_TUNE_FWD_SPLIT_PV = 7,
+  FA_TUNE_FWD_PERSISTENT = 8,
+  FA_TUNE_COUNT = 9
 } fa_tune_knob;
 fa_status fa_set_tuning(int knob, int value);
 int fa_get_tuning(int knob, int d);

@@ -184,7 +184,14 @@ def test_quant_tiny_blocks_bit_exact(d):
     codes, scales = gpu_quant(x)
     rc, rs = oracle.quant_fp8_ref(f64(x), False)
     assert np.array_equal(scales, rs)
-    assert np.array_equal(codes, rc)
+    bad = np.argwhere(codes != rc)
+    detail = []
+    for idx in bad[:12]:
+        idx = tuple(idx)
+        xv = float(f64(x)[idx])
+        qv = np.float32(np.float32(xv) / rs[idx[0], idx[1], idx[2] // 128])
+        detail.append(f"{idx}: x={xv:.6e} q={float(qv):.9e} gpu=0x{codes[idx]:02x} oracle=0x{rc[idx]:02x}")
+    assert bad.size == 0, f"{len(bad)} codes differ:\n" + "\n".join(detail)
     assert scales[0, 0, 0] == oracle.MIN_SCALE and not np.any((codes & 0x7F) == 0x7F)
 
 
@@ -225,23 +232,33 @@ def test_fp8_fwd_rotated_block_vs_per_tensor_baseline(record_property):
     assert max(e_rot) <= 7.5e-2 + 1e-2
 
 
+# The FP8 kernel's own error against the oracle on the dequantised inputs is
+# that of P rounded to E4M3: a half-ulp of 2^-4 relative, 3.6e-2 RMS for a
+# uniformly distributed rounding error; O averages it over the row's keys,
+# so its relative RMS stays below that (measured ~3e-2).
+FP8_KERNEL_REL_RMS = 2.0 ** -4 / math.sqrt(3.0)
+
+
 @pytest.mark.parametrize("pairs", [2, 4])
 def test_fp8_fwd_exp2_split_variants(pairs):
-    """The FP8 forward with part of its exp2 on the FMA-pipe polynomial stays
-    within the same bound against the oracle on the dequantised inputs."""
+    """The FP8 forward with part of its exp2 on the FMA-pipe polynomial: within
+    the E4M3 rounding bound of P against the oracle on the dequantised inputs,
+    and within a few E4M3 code flips of the SFU-only kernel."""
     fa = _fa()
-    fa.set_tuning("fp8_poly_pairs", pairs)
-    try:
-        q, k, v = inputs.make_qkv(1, 2, 1000, 128, seed=93 + pairs, outliers=True)
-        q8, sq = fa.quant_fp8(q.cuda())
-        k8, sk = fa.quant_fp8(k.cuda())
-        v8, sv = fa.quant_fp8(v.cuda())
-        for causal in (False, True):
+    q, k, v = inputs.make_qkv(1, 2, 1000, 128, seed=93 + pairs, outliers=True)
+    q8, sq = fa.quant_fp8(q.cuda())
+    k8, sk = fa.quant_fp8(k.cuda())
+    v8, sv = fa.quant_fp8(v.cuda())
+    deq = [oracle.dequant_fp8_ref(c.cpu().numpy(), s_.cpu().numpy()) for c, s_ in ((q8, sq), (k8, sk), (v8, sv))]
+    for causal in (False, True):
+        o_sfu, _ = fa.fwd_fp8(q8, k8, v8, sq, sk, sv, causal=causal)
+        fa.set_tuning("fp8_poly_pairs", pairs)
+        try:
             o, _ = fa.fwd_fp8(q8, k8, v8, sq, sk, sv, causal=causal)
-            torch.cuda.synchronize()
-            assert fa.get_status() == 0
-            deq = [oracle.dequant_fp8_ref(c.cpu().numpy(), s_.cpu().numpy()) for c, s_ in ((q8, sq), (k8, sk), (v8, sv))]
-            o_ref, _ = oracle.attn_fwd_ref(deq[0], deq[1], deq[2], 1 / math.sqrt(128), causal)
-            assert rel_rms(o.cpu(), o_ref) <= 3e-2
-    finally:
-        fa.set_tuning("fp8_poly_pairs", -1)
+        finally:
+            fa.set_tuning("fp8_poly_pairs", -1)
+        torch.cuda.synchronize()
+        assert fa.get_status() == 0
+        o_ref, _ = oracle.attn_fwd_ref(deq[0], deq[1], deq[2], 1 / math.sqrt(128), causal)
+        assert rel_rms(o.cpu(), o_ref) <= FP8_KERNEL_REL_RMS
+        assert rel_rms(o.cpu(), o_sfu.cpu()) <= 1e-2
