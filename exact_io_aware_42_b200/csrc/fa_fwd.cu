@@ -30,8 +30,9 @@
 // softmax warpgroup works on its tile while the tensor core runs the other
 // tile's two products (the lineage page's "pingpong" idea, "FA3 (2024)",
 // carried by two TMEM-resident tiles instead of two register warpgroups).
-// Each P V runs in two halves of 64 keys, the first released while the
-// softmax still computes the second.
+// Optionally (FA_TUNE_FWD_SPLIT_PV) each P V runs in two halves of 64 keys,
+// the first released while the softmax still computes the second; measured
+// slower at d <= 128, so off by default.
 //
 // Conditional rescaling (librarian page, "FA4", idea 2): a row keeps its
 // stale max m until a new tile's max exceeds it by more than kRescaleTau
@@ -72,7 +73,6 @@ struct FwdCfg {
 };
 static_assert(FwdCfg<128, true>::kSmemBytes <= 232448, "fp8 forward shared memory");
 static_assert(FwdCfg<128, false>::kSmemBytes <= 232448, "bf16 forward shared memory");
-static_assert(FwdCfg<64, false>::kSmemBytes <= 232448, "bf16 forward shared memory");
 
 // barrier slots
 __device__ __forceinline__ int bar_q(int t) { return t; }                 // Q_t landed
@@ -146,6 +146,8 @@ __device__ __forceinline__ int my_item(int k) {
 template <int D, bool CAUSAL, int NPOLY, int DEG, bool FP8>
 __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ FwdParams p) {
   using C = FwdCfg<D, FP8>;
+  constexpr int kWarpProd = 8;
+  constexpr int kWarpMma = 9;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -177,7 +179,7 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == kWarpMma) {
     tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
     tmem_relinquish();
   }
@@ -186,8 +188,7 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Abort ab{abort_flag, p.status};
-
-  if (warp == 8) {
+  if (warp == kWarpProd) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_q);
@@ -236,7 +237,7 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
       }
     }
     __syncwarp();
-  } else if (warp == 9) {
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdescS =
@@ -269,28 +270,28 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
           const int kk = h * kHalf + kq;
           // V is MN-major (d contiguous); one K step is kK key rows of 128 bytes.
           // P in TMEM packs 32 bits per column: 2 bf16 or 4 E4M3 keys.
+          const uint32_t a_col = 8 * kk;
           const uint64_t b = smem_desc_sw128(v_addr + kk * kK * 128, C::kPanelBytes, 1024);
           if constexpr (FP8)
-            mma_f8_ts(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + kk * 8, b, kIdescO,
+            mma_f8_ts(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + a_col, b, kIdescO,
                       (acc || kk > 0) ? 1u : 0u);
           else
-            mma_f16_ts(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + kk * 8, b, kIdescO,
+            mma_f16_ts(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + a_col, b, kIdescO,
                        (acc || kk > 0) ? 1u : 0u);
         }
       };
       int g[2] = {0, 0};   // P V products issued per tile (all items): the P barriers' phase
       // returns false if a wait gave up
       auto issue_pv = [&](int t, uint32_t v_addr, bool acc) -> bool {
-        // split: the first half as soon as it is in TMEM; otherwise both
-        // halves once all of P is (bar_ph completes after bar_p)
-        if (p.split_pv) {
-          if (!mbar_wait(bar(bar_p<NS>(t)), g[t] & 1, ab, kSiteMmaP)) return false;
-          tc_fence_after();
-          issue_pv_half(t, v_addr, acc, 0);
-        }
-        if (!mbar_wait(bar(bar_ph<NS>(t)), g[t] & 1, ab, kSiteMmaP)) return false;
+        // split: the first half as soon as it is in TMEM (bar_p), the second
+        // after bar_ph; otherwise all of P behind the one release (bar_p)
+        if (!mbar_wait(bar(bar_p<NS>(t)), g[t] & 1, ab, kSiteMmaP)) return false;
         tc_fence_after();
-        if (!p.split_pv) issue_pv_half(t, v_addr, acc, 0);
+        issue_pv_half(t, v_addr, acc, 0);
+        if (p.split_pv) {
+          if (!mbar_wait(bar(bar_ph<NS>(t)), g[t] & 1, ab, kSiteMmaP)) return false;
+          tc_fence_after();
+        }
         issue_pv_half(t, v_addr, acc, 1);
         tc_commit(bar(bar_pv<NS>(t)));
         ++g[t];
@@ -510,40 +511,59 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
             }
           }
         };
-        // first half of P, then the O correction, then release that half to
-        // the P V product while the second half is computed
-        exp_half(std::integral_constant<int, 0>{});
-        if constexpr (FP8)
-          tmem_st16(tS, *reinterpret_cast<uint32_t(*)[16]>(&u[0]));
-        else
-          tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-        if (j > 0) {
-          // PV(j-1) must be done before O is touched or PV(j) is released;
-          // waiting every tile also keeps this waiter within one phase.
-          if (!(ok = mbar_wait_warp(bar(bar_pv<NS>(t)), (gj - 1) & 1, ab, kSiteSmPv))) break;
-          tc_fence_after();
-          if (__any_sync(0xffffffffu, need)) {
+        // split: the first half of P, the O correction, release of that half
+        // to the P V product, then the second half.  Otherwise all of P, the
+        // correction, and one release (measured faster at d <= 128: the extra
+        // wait for the first half's TMEM store lies on the softmax's path).
+        auto correct_o = [&]() -> bool {
+          if (j > 0) {
+            // PV(j-1) must be done before O is touched or PV(j) is released;
+            // waiting every tile also keeps this waiter within one phase.
+            if (!mbar_wait_warp(bar(bar_pv<NS>(t)), (gj - 1) & 1, ab, kSiteSmPv)) return false;
+            tc_fence_after();
+            if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
-            for (int ch = 0; ch < D / 32; ++ch) {
-              uint32_t w[32];
-              tmem_ld32(tO + ch * 32, w);
+              for (int ch = 0; ch < D / 32; ++ch) {
+                uint32_t w[32];
+                tmem_ld32(tO + ch * 32, w);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
-              tmem_st32(tO + ch * 32, w);
+                for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
+                tmem_st32(tO + ch * 32, w);
+              }
             }
           }
+          return true;
+        };
+        if (p.split_pv) {
+          exp_half(std::integral_constant<int, 0>{});
+          if constexpr (FP8)
+            tmem_st16(tS, *reinterpret_cast<uint32_t(*)[16]>(&u[0]));
+          else
+            tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+          if (!(ok = correct_o())) break;
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(bar(bar_p<NS>(t)));
+          exp_half(std::integral_constant<int, 1>{});
+          if constexpr (FP8)
+            tmem_st16(tS + 16, *reinterpret_cast<uint32_t(*)[16]>(&u[16]));
+          else
+            tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(bar(bar_ph<NS>(t)));
+        } else {
+          exp_half(std::integral_constant<int, 0>{});
+          exp_half(std::integral_constant<int, 1>{});
+          if constexpr (FP8)
+            tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+          else
+            tmem_st64(tS, *reinterpret_cast<uint32_t(*)[64]>(&u[0]));
+          if (!(ok = correct_o())) break;
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(bar(bar_p<NS>(t)));
         }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(bar(bar_p<NS>(t)));
-        exp_half(std::integral_constant<int, 1>{});
-        if constexpr (FP8)
-          tmem_st16(tS + 16, *reinterpret_cast<uint32_t(*)[16]>(&u[16]));
-        else
-          tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(bar(bar_ph<NS>(t)));
         float sum4[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -589,7 +609,7 @@ __global__ void __launch_bounds__(320, 1) fwd_kernel(const __grid_constant__ Fwd
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }

@@ -51,7 +51,7 @@ struct FwdParams {
   int poly_pairs;       // of every 8 column pairs, how many use the FMA-pipe exp2
   int poly_deg;         // degree of that polynomial (3 or 4)
   int sms;              // multiprocessor count: persistent grid size
-  int split_pv;         // 1: P V issued in two 64-key halves as P arrives; 0: after all of P
+  int split_pv;         // d <= 128: 1: P V issued in two 64-key halves as P arrives; 0: after all of P
   int persistent;       // 1: grid of min(items, SMs) CTAs; 0: one CTA per work item
 };
 
@@ -61,10 +61,12 @@ struct FwdParams {
 // SFU time they free); at d = 64, where the softmax is the bound, half the
 // pairs on the polynomial was fastest.
 constexpr int kDefaultPolyPairsD128 = 0;
-constexpr int kDefaultPolyPairsD64 = 4;
+// d = 64: SFU-only measured fastest with the persistent kernel (642 vs 560-595 TFLOPS non-causal)
+constexpr int kDefaultPolyPairsD64 = 0;
 constexpr int kDefaultPolyPairsD256 = 0;
 constexpr int kDefaultPolyDegree = 4;
-constexpr int kDefaultFwdSplitPv = 1;
+// measured on B200 (cfg B4 H16 N4096 d128 causal: 903 vs 870 TFLOPS; N 16384: 1060 vs 1006)
+constexpr int kDefaultFwdSplitPv = 0;
 constexpr int kDefaultFwdPersistent = 1;
 // FP8 forward: share of the exp2 on the polynomial (pairs of 8)
 constexpr int kDefaultPolyPairsFp8 = 0;

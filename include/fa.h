@@ -257,8 +257,9 @@ fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v8, const fl
  *  FA_TUNE_BWD_PAIR         deterministic backward at d = 128: dK, dV from
  *                           CTA pairs sharing each product (1) or from single
  *                           CTAs (0); same results either way
- *  FA_TUNE_FWD_SPLIT_PV     forward: P V issued in two halves as P arrives (1)
- *                           or after all of P (0)
+ *  FA_TUNE_FWD_SPLIT_PV     forward, d <= 128: P V issued in two halves as P
+ *                           arrives (1) or after all of P (0); the d = 256
+ *                           kernel always splits
  *  FA_TUNE_FWD_PERSISTENT   forward: one CTA per SM walking the work items (1)
  *                           or one CTA per work item (0)
  * value -1 restores the built-in default.  Any other value, or an unknown
