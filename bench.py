@@ -131,9 +131,12 @@ def measured_peaks():
 
 KERNEL_SOURCES = {
     "fwd": ("fa_fwd.cu",),
+    "fwd_tile": ("fa_fwd_tile.cu",),
     "fwd256": ("fa_fwd_d256.cu",),
     "bwd": ("fa_bwd.cu",),
     "bwd_dq": ("fa_bwd_dq.cu",),
+    "bwd_pair": ("fa_bwd_pair.cu",),
+    "bwd256": ("fa_bwd_d256.cu",),
     "fp8": ("fa_fp8.cu",),
 }
 
@@ -569,10 +572,12 @@ def run_ours(args):
                         profiled_traffic("bwd_main_kernel", w["name"], "bwd") if BWD_MODE == "atomic" else None)
         roof_bwd["frac_sustained"] = roof_bwd["achieved"] / sustained
         roof_bwd["frac_nominal_2250"] = roof_bwd["achieved"] / 2250.0
-    fwd_name = "fwd256_kernel" if d == 256 else "fwd_kernel"
-    roof_fwd = roof(stages, per_stage, "fwd_bf16", f"{fwd_name}<{d}, {cz}, bf16> (persistent)",
-                    fwd_bytes(B, H, N, d, H_kv), burst, burst_note,
-                    profiled_traffic(fwd_name, w["name"], "fwd256" if d == 256 else "fwd"))
+    pers = TUNING.get("fwd_persistent") == 1
+    fwd_name, fwd_src = (("fwd256_kernel", "fwd256") if d == 256 else ("fwd_kernel", "fwd") if pers
+                         else ("fwd_tile_kernel", "fwd_tile"))
+    fwd_desc = f"{fwd_name}<{d}, {cz}, bf16>" + (" (persistent)" if d == 256 or pers else " (one CTA per item)")
+    roof_fwd = roof(stages, per_stage, "fwd_bf16", fwd_desc, fwd_bytes(B, H, N, d, H_kv), burst, burst_note,
+                    profiled_traffic(fwd_name, w["name"], fwd_src))
     roof_fwd["frac_sustained"] = roof_fwd["achieved"] / sustained
     roof_fwd["frac_nominal_2250"] = roof_fwd["achieved"] / 2250.0
     line = {
@@ -597,7 +602,8 @@ def run_ours(args):
     if fp8_stages:
         fp8_peak = 2.0 * burst
         fp8_flops = sum(s[2] for s in fp8_stages)
-        rf = roof(fp8_stages, fp8_per_stage, "fwd_fp8", f"fwd_kernel<128, {cz}, e4m3>", None, fp8_peak,
+        fp8_name = "fwd_kernel" if pers else "fwd_tile_kernel"
+        rf = roof(fp8_stages, fp8_per_stage, "fwd_fp8", f"{fp8_name}<128, {cz}, e4m3>", None, fp8_peak,
                   f"2 x {peak_src} bf16_tflops burst (nominal 2:1 ratio of dense E4M3 to bf16; no measured "
                   "FP8 peak)", None)
         rf["algorithmic_bytes"] = fwd_bytes(B, H, N, d, H_kv) - (B * H + 2 * B * H_kv) * N * d

@@ -123,9 +123,10 @@ int fwd_split_pv() {
   return v >= 0 ? v : kDefaultFwdSplitPv;
 }
 
-int fwd_persistent() {
+int fwd_persistent(int d, bool fp8) {
   const int v = tune_raw(FA_TUNE_FWD_PERSISTENT);
-  return v >= 0 ? v : kDefaultFwdPersistent;
+  if (v >= 0) return v;
+  return fp8 ? kDefaultFwdPersistentFp8 : d == 64 ? kDefaultFwdPersistentD64 : kDefaultFwdPersistentD128;
 }
 
 int bwd_pair() {
@@ -280,7 +281,8 @@ extern "C" fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void
   p.o = static_cast<uint16_t*>(o);
   p.sms = di->sms;
   p.split_pv = fwd_split_pv();
-  p.persistent = fwd_persistent();
+  p.persistent = d == 256 ? 1 : fwd_persistent(d, false);
+  if (!p.persistent && !encode_3d(&p.tm_o, o, bf, 2, d, N, BH, 64, kBlockM)) return FA_ERR_INVALID_ARG;
   p.lse = lse;
   p.status = di->status;
   p.N = N;
@@ -298,7 +300,8 @@ extern "C" fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void
   p.poly_deg = poly_degree();
   if (d == 256 && static_cast<long long>(p.n_kv) * BH > kMaxWorkItems) return FA_ERR_UNSUPPORTED;
   cudaError_t e = d == 256 ? launch_fwd_d256(p, causal != 0, static_cast<cudaStream_t>(stream))
-                           : launch_fwd_bf16(p, d, causal != 0, static_cast<cudaStream_t>(stream));
+                  : p.persistent ? launch_fwd_bf16(p, d, causal != 0, static_cast<cudaStream_t>(stream))
+                                 : launch_fwd_tile_bf16(p, d, causal != 0, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     cudaGetLastError();
     return FA_ERR_LAUNCH;
@@ -533,7 +536,10 @@ extern "C" fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v
   p.o = static_cast<uint16_t*>(o);
   p.sms = di->sms;
   p.split_pv = fwd_split_pv();
-  p.persistent = fwd_persistent();
+  p.persistent = fwd_persistent(d, true);
+  if (!p.persistent &&
+      !encode_3d(&p.tm_o, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, BH, 64, kBlockM))
+    return FA_ERR_INVALID_ARG;
   p.lse = lse;
   p.status = di->status;
   p.sq = sq;
@@ -552,7 +558,8 @@ extern "C" fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.poly_pairs = fp8_poly_pairs();
   p.poly_deg = poly_degree();
-  cudaError_t e = launch_fwd_fp8(p, causal != 0, static_cast<cudaStream_t>(stream));
+  cudaError_t e = p.persistent ? launch_fwd_fp8(p, causal != 0, static_cast<cudaStream_t>(stream))
+                               : launch_fwd_tile_fp8(p, causal != 0, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     cudaGetLastError();
     return FA_ERR_LAUNCH;
@@ -601,7 +608,7 @@ extern "C" int fa_get_tuning(int knob, int d) {
     case FA_TUNE_FP8_POLY_PAIRS: return fp8_poly_pairs();
     case FA_TUNE_BWD_PAIR: return d == 128 ? bwd_pair() : 0;
     case FA_TUNE_FWD_SPLIT_PV: return fwd_split_pv();
-    case FA_TUNE_FWD_PERSISTENT: return fwd_persistent();
+    case FA_TUNE_FWD_PERSISTENT: return d == 256 ? 1 : fwd_persistent(d, false);
     default: return -1;
   }
 }

@@ -1,0 +1,594 @@
+// Fused exact attention forward for sm_100a, one CTA per work item (bf16 or
+// E4M3 in, fp32 accumulate).  The default kernel at d = 128; the persistent
+// kernel (fa_fwd.cu) runs the same work items from a grid of one CTA per SM.
+//
+// What it computes: O = softmax(scale * Q K^T [causal]) V and the per-row
+// logsumexp L, exactly as the standard definition ("FlashAttention" concept
+// note, "How it works"), reached by the online softmax of "FlashAttention
+// v1/v2/v3/v4: the librarian who never clears the desk" (online softmax
+// section, eq. 2): per K/V tile the running max m and sum l are updated, the
+// running output is rescaled by 2^(m_old - m_new), and the division by l is
+// deferred to the end (lineage page, "FA2 (2023)", refinement 2).
+//
+// Work unit: one CTA owns two 128-row query tiles of one (b, h) and streams
+// every needed 128-key K/V tile once for both (each K/V tile is read from
+// L2/HBM once per 256 query rows).  With a single item per CTA the softmax
+// warps keep no cross-item state (measured faster at d = 128 than the
+// persistent kernel: its extra live registers cost more than the overlap of
+// one item's epilogue with the next item's start gains), and O leaves
+// through shared memory and a TMA store.  Roles:
+//   warps 0-3  softmax for query tile 0 (thread r owns row r = TMEM lane r)
+//   warps 4-7  softmax for query tile 1
+//   warp  8    TMA producer: Q tiles, then K_0, V_0, K_1, V_1, ... into a
+//              ring of 128 x d shared-memory tiles (full/empty mbarriers)
+//   warp  9    allocates TMEM; one thread issues every tcgen05.mma
+// TMEM (512 columns x 128 lanes, fp32):
+//   [0,128)    S_0 (tile 0 scores); after softmax the first 64 columns hold
+//              P_0 as packed bf16 pairs, read back as the A operand of P V
+//   [128,256)  S_1 / P_1
+//   [256,256+d)        O_0 accumulator
+//   [256+d,256+2d)     O_1 accumulator
+// MMA order per key tile j:  PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), so each
+// softmax warpgroup works on its tile while the tensor core runs the other
+// tile's two products (the lineage page's "pingpong" idea, "FA3 (2024)",
+// carried by two TMEM-resident tiles instead of two register warpgroups).
+// With P over S, S_t(j+1) cannot start before P V_t(j) has read P_t(j), so
+// each tile's softmax waits for its own two products every key tile.  At
+// d = 64 the O accumulators leave 128 columns free, P_t gets
+//   [384 + 64 t, 448 + 64 t)   P_t (d = 64)
+// and S_t(j+1) is issued as soon as the softmax has read S_t(j) out (before
+// its exponentials): S_0(j+1), S_1(j+1), PV_0(j), PV_1(j).
+//
+// Conditional rescaling (librarian page, "FA4", idea 2): a row keeps its
+// stale max m until a new tile's max exceeds it by more than kRescaleTau
+// (log2 units).  p = 2^(x - m) is then at most 2^tau, the same stale m is
+// used for p, l, O and L, and the result is unchanged up to rounding.  The
+// O rescale in TMEM runs only for warps where some row moved its max.
+//
+// Causal: key j visible to query i iff j <= i.  Tiles entirely above the
+// diagonal are never loaded or multiplied; only the diagonal tile and the
+// ragged key tail (keys >= N, zero-filled by TMA) are masked to -inf.
+#include "fa_exp2.cuh"
+#include "fa_internal.h"
+#include "fa_ptx.cuh"
+
+namespace fa {
+namespace {
+
+template <int D, bool FP8 = false>
+struct TileCfg {
+  static constexpr int kElem = FP8 ? 1 : 2;            // bytes per Q/K/V element
+  static constexpr int kPanels = D * kElem / 128;      // 128-byte swizzle panels per row
+  static constexpr int kPanelElems = 128 / kElem;      // elements per panel row
+  static constexpr int kPanelBytes = 128 * 128;        // 128 rows x 128 bytes
+  static constexpr int kTileBytes = kBlockM * D * kElem;   // one 128 x D tile
+  static constexpr int kStages = FP8 ? 8 : ((D == 128) ? 5 : 8);
+  static constexpr int kThreads = 320;
+  static constexpr int kOffQ = 0;                      // two query tiles
+  // bf16 O is staged in the Q tile it replaces; FP8 tiles are half as large,
+  // so FP8 stages O in a buffer of its own (2 x 128 x D bf16).
+  static constexpr int kOffO = FP8 ? 2 * kTileBytes : 0;
+  static constexpr int kOBytes = kBlockM * D * 2;
+  static constexpr int kOffRing = FP8 ? kOffO + 2 * kOBytes : 2 * kTileBytes;
+  static constexpr int kOffBar = kOffRing + kStages * kTileBytes;
+  static constexpr int kNumBars = 2 + 2 * kStages + 9;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 48 + 1024;   // + base alignment slack
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS = 0;       // + 128 * t
+  static constexpr uint32_t kColO = 256;     // + D * t
+  // d = 64: P_t in a region of its own at kColP + 64 t (see the kernel notes);
+  // d = 128 has no room for it and stores P over the consumed S_t
+  static constexpr bool kSepP = (D == 64);
+  static constexpr uint32_t kColP = 384;
+};
+static_assert(TileCfg<128, true>::kSmemBytes <= 232448, "fp8 forward shared memory");
+static_assert(TileCfg<128, false>::kSmemBytes <= 232448, "bf16 forward shared memory");
+
+// barrier slots
+__device__ __forceinline__ int bar_q(int t) { return t; }
+template <int NS> __device__ __forceinline__ int bar_full(int s) { return 2 + s; }
+template <int NS> __device__ __forceinline__ int bar_empty(int s) { return 2 + NS + s; }
+template <int NS> __device__ __forceinline__ int bar_s(int t) { return 2 + 2 * NS + t; }
+template <int NS> __device__ __forceinline__ int bar_p(int t) { return 4 + 2 * NS + t; }
+template <int NS> __device__ __forceinline__ int bar_pv(int t) { return 6 + 2 * NS + t; }
+template <int NS> __device__ __forceinline__ int bar_drain() { return 8 + 2 * NS; }
+template <int NS> __device__ __forceinline__ int bar_sfree(int t) { return 9 + 2 * NS + t; }   // S_t read out
+
+// wait-site codes reported in bits 8..15 of the status word
+enum : unsigned int { kSiteProdEmpty = 1, kSiteMmaQ, kSiteMmaFull, kSiteMmaP, kSiteSmS, kSiteSmPv,
+                      kSiteEpiPv, kSiteDrain, kSiteMmaSfree };
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+// E4M3 byte pair <- (lo, hi), round to nearest even, saturating at +-448.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  unsigned short lo, hi;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
+// NPOLY of every 8 column pairs take the polynomial exp2 (degree DEG), the
+// rest the SFU.  FP8: Q, K, V are E4M3 with per-128-row block scales and both
+// products run as kind::f8f6f4 (see the FP8 notes at the softmax).
+template <int D, bool CAUSAL, int NPOLY, int DEG, bool FP8>
+__global__ void __launch_bounds__(320, 1) fwd_tile_kernel(const __grid_constant__ FwdParams p) {
+  using C = TileCfg<D, FP8>;
+  constexpr int NS = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sbase + C::kOffBar + 8 * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  // Causal: the heaviest pairs of every head first (longest-first balances
+  // the uneven work).  Non-causal: head-major, so the resident CTAs cover a
+  // few heads whose K and V stay in L2.  Both orders measured on B200.
+  const int bh = CAUSAL ? blockIdx.x % p.BH : blockIdx.x / p.n_pairs;
+  const int pair = CAUSAL ? p.n_pairs - 1 - blockIdx.x / p.BH : blockIdx.x % p.n_pairs;
+  // Grouped K/V heads: query head h of batch b reads K/V head b * H_kv + h / G,
+  // which in the flattened [B * H] index is bh / G.
+  const int kvh = bh / p.kv_group;
+  const int qt0 = 2 * pair;
+  // Sliding window (causal only): key j is visible to query i iff
+  // i - window <= j <= i.  Key blocks wholly left of tile 0's window are
+  // never loaded; both tiles start at the same block (tile 1's first block
+  // may then be fully masked for it, which the softmax handles).
+  const int j_start = CAUSAL ? max(0, qt0 * kBlockM - p.window) / kBlockN : 0;
+  int n_t[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) n_t[t] = (CAUSAL ? min(qt0 + t + 1, p.n_kv) : p.n_kv) - j_start;
+  const int n_iter = n_t[1];
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(bar_q(0)), 1);
+    mbar_init(bar(bar_q(1)), 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar(bar_full<NS>(s)), 1);
+      mbar_init(bar(bar_empty<NS>(s)), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(bar_s<NS>(t)), 1);
+      mbar_init(bar(bar_p<NS>(t)), 128);
+      mbar_init(bar(bar_pv<NS>(t)), 1);
+      mbar_init(bar(bar_sfree<NS>(t)), 128);
+    }
+    mbar_init(bar(bar_drain<NS>()), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Abort ab{abort_flag, p.status};
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_q);
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
+      for (int t = 0; t < 2; ++t) {
+        mbar_arrive_expect_tx(bar(bar_q(t)), C::kTileBytes);
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_3d(sbase + C::kOffQ + t * C::kTileBytes + pn * C::kPanelBytes, &p.tm_q,
+                      bar(bar_q(t)), pn * C::kPanelElems, (qt0 + t) * kBlockM, bh);
+      }
+      int seq = 0;
+      bool ok = true;
+      for (int j = 0; j < n_iter && ok; ++j) {
+        for (int w = 0; w < 2 && ok; ++w) {
+          const int s = seq % NS;
+          const uint32_t ph = (seq / NS) & 1;
+          if (!mbar_wait(bar(bar_empty<NS>(s)), ph ^ 1, ab, kSiteProdEmpty)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(bar_full<NS>(s)), C::kTileBytes);
+          const CUtensorMap* m = (w == 0) ? &p.tm_k : &p.tm_v;
+          for (int pn = 0; pn < C::kPanels; ++pn)
+            tma_load_3d(sbase + C::kOffRing + s * C::kTileBytes + pn * C::kPanelBytes, m,
+                        bar(bar_full<NS>(s)), pn * C::kPanelElems, (j_start + j) * kBlockN, kvh);
+          ++seq;
+        }
+      }
+      if (*abort_flag) {
+        // Another role gave up: let every copy this thread started land before
+        // the CTA exits (bounded, ignoring the abort flag).
+        volatile int never = 0;
+        const Abort drain{&never, p.status};
+        for (int t = 0; t < 2; ++t) mbar_wait(bar(bar_q(t)), 0, drain, kSiteDrain);
+        const int first = seq > NS ? seq - NS : 0;
+        for (int q = first; q < seq; ++q)
+          mbar_wait(bar(bar_full<NS>(q % NS)), (q / NS) & 1, drain, kSiteDrain);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdescS =
+          FP8 ? idesc_e4m3_f32(128, 128, false, false) : idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t kIdescO =
+          FP8 ? idesc_e4m3_f32(128, D, false, true) : idesc_bf16_f32(128, D, false, true);
+      constexpr int kK = FP8 ? 32 : 16;            // K elements per MMA (32 bytes)
+      const uint32_t q_addr[2] = {sbase + C::kOffQ, sbase + C::kOffQ + C::kTileBytes};
+      auto ring = [&](int s) -> uint32_t { return sbase + C::kOffRing + s * C::kTileBytes; };
+      auto issue_s = [&](int t, uint32_t k_addr) {
+#pragma unroll
+        for (int kk = 0; kk < D / kK; ++kk) {
+          const uint32_t off = (kk / 4) * C::kPanelBytes + (kk % 4) * 32;
+          const uint64_t a = smem_desc_sw128(q_addr[t] + off, 16, 1024);
+          const uint64_t b = smem_desc_sw128(k_addr + off, 16, 1024);
+          if constexpr (FP8)
+            mma_f8_ss(tmem + C::kColS + 128 * t, a, b, kIdescS, kk > 0 ? 1u : 0u);
+          else
+            mma_f16_ss(tmem + C::kColS + 128 * t, a, b, kIdescS, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(bar_s<NS>(t)));
+      };
+      auto issue_pv = [&](int t, uint32_t v_addr, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < kBlockN / kK; ++kk) {
+          // V is MN-major (d contiguous); one K step is kK key rows of 128 bytes.
+          // P in TMEM packs 32 bits per column: 2 bf16 or 4 E4M3 keys.
+          const uint64_t b = smem_desc_sw128(v_addr + kk * kK * 128, C::kPanelBytes, 1024);
+          if constexpr (FP8)
+            mma_f8_ts(tmem + C::kColO + D * t, tmem + C::kColS + 128 * t + kk * 8, b, kIdescO,
+                      (acc || kk > 0) ? 1u : 0u);
+          else
+            mma_f16_ts(tmem + C::kColO + D * t,
+                       tmem + (C::kSepP ? C::kColP + 64 * t : C::kColS + 128 * t) + kk * 8, b, kIdescO,
+                       (acc || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(bar(bar_pv<NS>(t)));
+      };
+      bool ok = mbar_wait(bar(bar_q(0)), 0, ab, kSiteMmaQ) && mbar_wait(bar(bar_q(1)), 0, ab, kSiteMmaQ);
+      int seq = 0;
+      int ks = 0;
+      if (ok) ok = mbar_wait(bar(bar_full<NS>(0)), 0, ab, kSiteMmaFull);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, ring(0));
+        issue_s(1, ring(0));
+        tc_commit(bar(bar_empty<NS>(0)));
+        seq = 1;
+      }
+      for (int j = 0; j < n_iter && ok; ++j) {
+        const int vs = seq % NS;
+        if (!(ok = mbar_wait(bar(bar_full<NS>(vs)), (seq / NS) & 1, ab, kSiteMmaFull))) break;
+        ++seq;
+        const bool has_next = j + 1 < n_iter;
+        if (has_next) {
+          ks = seq % NS;
+          if (!(ok = mbar_wait(bar(bar_full<NS>(ks)), (seq / NS) & 1, ab, kSiteMmaFull))) break;
+          ++seq;
+        }
+        tc_fence_after();
+        if constexpr (C::kSepP) {
+          // S_t(j+1) as soon as the softmax has read S_t(j) out (P_t(j) has
+          // a region of its own), then the P V products as P arrives
+          if (has_next) {
+            if (j + 1 < n_t[0]) {
+              if (!(ok = mbar_wait(bar(bar_sfree<NS>(0)), j & 1, ab, kSiteMmaSfree))) break;
+              tc_fence_after();
+              issue_s(0, ring(ks));
+            }
+            if (!(ok = mbar_wait(bar(bar_sfree<NS>(1)), j & 1, ab, kSiteMmaSfree))) break;
+            tc_fence_after();
+            issue_s(1, ring(ks));
+            tc_commit(bar(bar_empty<NS>(ks)));
+          }
+          if (j < n_t[0]) {
+            if (!(ok = mbar_wait(bar(bar_p<NS>(0)), j & 1, ab, kSiteMmaP))) break;
+            tc_fence_after();
+            issue_pv(0, ring(vs), j > 0);
+          }
+          if (!(ok = mbar_wait(bar(bar_p<NS>(1)), j & 1, ab, kSiteMmaP))) break;
+          tc_fence_after();
+          issue_pv(1, ring(vs), j > 0);
+          tc_commit(bar(bar_empty<NS>(vs)));
+        } else {
+          if (j < n_t[0]) {
+            if (!(ok = mbar_wait(bar(bar_p<NS>(0)), j & 1, ab, kSiteMmaP))) break;
+            tc_fence_after();
+            issue_pv(0, ring(vs), j > 0);
+            if (j + 1 < n_t[0]) issue_s(0, ring(ks));
+          }
+          if (!(ok = mbar_wait(bar(bar_p<NS>(1)), j & 1, ab, kSiteMmaP))) break;
+          tc_fence_after();
+          issue_pv(1, ring(vs), j > 0);
+          tc_commit(bar(bar_empty<NS>(vs)));
+          if (has_next) {
+            issue_s(1, ring(ks));
+            tc_commit(bar(bar_empty<NS>(ks)));
+          }
+        }
+      }
+      // Every MMA issued above must be finished before TMEM is released,
+      // also when a role gave up part-way.
+      tc_commit(bar(bar_drain<NS>()));
+      volatile int never = 0;
+      const Abort drain{&never, p.status};
+      mbar_wait(bar(bar_drain<NS>()), 0, drain, kSiteDrain);
+    }
+    __syncwarp();
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ softmax
+    const int t = warp >> 2;                 // query tile of this warpgroup
+    const int r = threadIdx.x - 128 * t;     // row within the tile == TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + C::kColS + 128 * t + lane_off;
+    const uint32_t tO = tmem + C::kColO + D * t + lane_off;
+    const uint32_t tP = tmem + C::kColP + 64 * t + lane_off;   // d = 64 only
+    const int qi = qt0 + t;
+    const int row = qi * kBlockM + r;
+    const int n = n_t[t];
+    // FP8: scores are dequantised per tile pair with s_q(i) * s_k(j); P is
+    // stored as E4M3 times 256 * s_v(j) / max_j s_v(j), which folds V's block
+    // scale into P (p <= 2^0.75 because FP8 rescales once the max has grown by
+    // more than kRescaleTauFp8, so P <= 430.5 < 448), and O is multiplied back
+    // by max s_v / 256 at the end.
+    const size_t sc_base = static_cast<size_t>(bh) * p.n_kv;      // Q's block scales
+    const size_t kv_base = static_cast<size_t>(kvh) * p.n_kv;     // K's and V's
+    float c_q = p.scale_log2;
+    float v_max = 1.f;
+    float sk_next = 1.f, sv_next = 1.f;
+    if constexpr (FP8) {
+      c_q *= (qi < p.n_kv) ? p.sq[sc_base + qi] : 1.f;
+      // max over this head's V block scales: strided over the warpgroup's
+      // 128 threads, then a shuffle and a shared-memory reduction
+      float vm = 0.f;
+      for (int jj = r; jj < p.n_kv; jj += 128) vm = fmaxf(vm, p.sv[kv_base + jj]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, off));
+      float* red = reinterpret_cast<float*>(smem + C::kOffMisc + 8) + 4 * t;   // 4 floats per tile
+      if (lane == 0) red[warp & 3] = vm;
+      named_bar_sync(1 + t, 128);
+      v_max = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+      sk_next = p.sk[kv_base + j_start];
+      sv_next = p.sv[kv_base + j_start];
+    }
+    constexpr float kTau = FP8 ? kRescaleTauFp8 : kRescaleTau;
+    float m_use = -INFINITY;
+    float l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int jb = j_start + j;      // key block; j counts this tile's iterations
+      if (!(ok = mbar_wait_warp(bar(bar_s<NS>(t)), j & 1, ab, kSiteSmS))) break;
+      tc_fence_after();
+      uint32_t u[128];
+      tmem_ld128(tS, u);
+      if constexpr (C::kSepP) {   // S_t may be overwritten by S_t(j+1) from here on
+        tc_fence_before();
+        mbar_arrive(bar(bar_sfree<NS>(t)));
+      }
+      const float c = c_q * sk_next;   // FP8: dequantise with s_q(i) s_k(j); bf16: sk_next = 1
+      const float sv_j = sv_next;
+      if constexpr (FP8) {             // next tile's scales, loaded while this one is processed
+        if (j + 1 < n) {
+          sk_next = p.sk[kv_base + jb + 1];
+          sv_next = p.sv[kv_base + jb + 1];
+        }
+      }
+      // ALiBi sends every block through this path: the bias is added to the
+      // scaled scores before the row maximum is taken.
+      const bool masked = (CAUSAL && (jb == qi || jb * kBlockN < qi * kBlockM + kBlockM - 1 - p.window)) ||
+                          ((jb + 1) * kBlockN > p.N) || p.alibi != nullptr;
+      if (masked) {
+        // scaled scores with -inf where the key is hidden or past N: column i
+        // is visible iff lo <= i < hi
+        const int key0 = jb * kBlockN;
+        const int hi = (CAUSAL ? min(row + 1, p.N) : p.N) - key0;
+        const int lo = CAUSAL ? row - p.window - key0 : 0;
+        if (p.alibi != nullptr) {   // + this query head's slope log2(e) * -|key - row|
+          const float sl2 = p.alibi[bh % p.H] * 1.4426950408889634f;
+          const float dk = static_cast<float>(key0 - row);
+#pragma unroll
+          for (int i = 0; i < 128; ++i) {
+            const bool vis = i >= lo && i < hi;
+            const float bias = -sl2 * fabsf(dk + static_cast<float>(i));
+            u[i] = __float_as_uint(vis ? fmaf(__uint_as_float(u[i]), c, bias) : -INFINITY);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 128; ++i) {
+            const bool vis = i >= lo && i < hi;
+            u[i] = __float_as_uint(vis ? __uint_as_float(u[i]) * c : -INFINITY);
+          }
+        }
+      }
+      float mt;
+      {
+        float a[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) a[k] = fmaxf(__uint_as_float(u[k]), __uint_as_float(u[8 + k]));
+#pragma unroll
+        for (int i = 16; i < 128; i += 16) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            a[k] = max3f(a[k], __uint_as_float(u[i + k]), __uint_as_float(u[i + 8 + k]));
+        }
+        mt = max3f(max3f(a[0], a[1], a[2]), max3f(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+        if (!masked) mt *= c;
+      }
+      const float m_new = fmaxf(m_use, mt);
+      const bool need = m_new > m_use + kTau;
+      float alpha = 1.f;
+      if (need) {
+        alpha = ex2_sfu(m_use - m_new);
+        m_use = m_new;
+      }
+      // a row that has seen only hidden keys so far (sliding window) keeps
+      // m = -inf; its p must be 0, not exp2(-inf + inf)
+      const float neg_m = m_use == -INFINITY ? 0.f : -m_use;
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+      if constexpr (FP8) {
+        const float f8 = 256.f * sv_j / v_max;
+        const uint64_t c2 = f2_pack(c, c);
+        const uint64_t nm2 = f2_pack(neg_m, neg_m);
+        float keep0 = 0.f, keep1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const uint64_t s2 = f2_pack(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]));
+          const uint64_t x2 = masked ? f2_add(s2, nm2) : f2_fma(s2, c2, nm2);
+          const uint64_t p2 = ((i & 7) < NPOLY) ? exp2_poly_f2<DEG>(x2) : exp2_sfu_f2(x2);
+          acc[i & 3] = f2_add(acc[i & 3], p2);
+          float p0, p1;
+          f2_unpack(p2, p0, p1);
+          if (i & 1)
+            u[i / 2] = pack_e4m3x4(keep0 * f8, keep1 * f8, p0 * f8, p1 * f8);
+          keep0 = p0;
+          keep1 = p1;
+        }
+        tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+      } else {
+        if (masked) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const float p0 = ex2_sfu(__uint_as_float(u[2 * i]) + neg_m);
+            const float p1 = ex2_sfu(__uint_as_float(u[2 * i + 1]) + neg_m);
+            acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
+            u[i] = pack_bf16x2(p0, p1);       // P overwrites the consumed scores
+          }
+        } else {
+          const uint64_t c2 = f2_pack(c, c);
+          const uint64_t nm2 = f2_pack(neg_m, neg_m);
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const uint64_t x2 =
+                f2_fma(f2_pack(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1])), c2, nm2);
+            const uint64_t p2 = ((i & 7) < NPOLY) ? exp2_poly_f2<DEG>(x2) : exp2_sfu_f2(x2);
+            acc[i & 3] = f2_add(acc[i & 3], p2);
+            float p0, p1;
+            f2_unpack(p2, p0, p1);
+            u[i] = pack_bf16x2(p0, p1);
+          }
+        }
+        if constexpr (!C::kSepP) tmem_st64(tS, *reinterpret_cast<uint32_t(*)[64]>(&u[0]));
+      }
+      if constexpr (!C::kSepP) tmem_st_wait();
+      float sum4[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float lo, hi;
+        f2_unpack(acc[k], lo, hi);
+        sum4[k] = lo + hi;
+      }
+      l = l * alpha + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
+      if (j > 0) {
+        // PV(j-1) must be done before O is touched or PV(j) is released;
+        // waiting every tile also keeps this waiter within one phase.
+        if (!(ok = mbar_wait_warp(bar(bar_pv<NS>(t)), (j - 1) & 1, ab, kSiteSmPv))) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t u[32];
+            tmem_ld32(tO + ch * 32, u);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+            tmem_st32(tO + ch * 32, u);
+          }
+          tmem_st_wait();
+        }
+      }
+      if constexpr (C::kSepP) {   // P_t's region is free once P V_t(j-1) is done (waited above)
+        tmem_st64(tP, *reinterpret_cast<uint32_t(*)[64]>(&u[0]));
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      mbar_arrive(bar(bar_p<NS>(t)));
+    }
+    if (ok) ok = mbar_wait_warp(bar(bar_pv<NS>(t)), (n - 1) & 1, ab, kSiteEpiPv);
+    // All 128 threads of the warpgroup reach this barrier (every wait above is
+    // bounded) and take the epilogue together or not at all.
+    ok = named_bar_and(1 + t, 128, ok);
+    if (ok) {
+      tc_fence_after();
+      // ---------------------------------------------------------- epilogue
+      const float inv_l = (FP8 ? v_max * (1.f / 256.f) : 1.f) / l;
+      // bf16: stage O in Q_t, no longer read; FP8: in its own buffer
+      const uint32_t o_stage = FP8 ? sbase + C::kOffO + t * C::kOBytes : sbase + C::kOffQ + t * C::kTileBytes;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t u[32];
+        tmem_ld32(tO + ch * 32, u);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack_bf16x2(__uint_as_float(u[2 * i]) * inv_l, __uint_as_float(u[2 * i + 1]) * inv_l);
+        const int col0 = ch * 32;
+        const uint32_t panel = o_stage + (col0 / 64) * C::kPanelBytes + r * 128;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t chunk = ((col0 % 64) / 8 + q) ^ (r & 7);
+          st_shared_v4(panel + (chunk << 4), pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1 + t, 128);
+      if (r == 0 && qi * kBlockM < p.N) {   // a tile wholly past N is padding
+        for (int pn = 0; pn < D / 64; ++pn)
+          tma_store_3d(&p.tm_o, o_stage + pn * C::kPanelBytes, pn * 64, qi * kBlockM, bh);   // bf16 O
+        tma_store_commit();
+        tma_store_wait_all();
+      }
+      if (row < p.N) p.lse[static_cast<size_t>(bh) * p.N + row] = (m_use + log2f(l)) * 0.69314718055994531f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int D, bool CAUSAL, int NPOLY, int DEG, bool FP8>
+cudaError_t launch_impl(const FwdParams& p, cudaStream_t stream) {
+  using C = TileCfg<D, FP8>;
+  auto kern = fwd_tile_kernel<D, CAUSAL, NPOLY, DEG, FP8>;
+  cudaError_t e = set_smem_once<fwd_tile_kernel<D, CAUSAL, NPOLY, DEG, FP8>>(C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(p.n_pairs) * static_cast<unsigned>(p.BH);
+  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(p);
+  return cudaGetLastError();
+}
+
+// The exp2 split (pairs of 8 on the polynomial) and the polynomial's degree.
+template <int D, bool CAUSAL, bool FP8>
+cudaError_t launch_np(const FwdParams& p, cudaStream_t stream) {
+  const bool deg4 = p.poly_deg == 4;
+  switch (p.poly_pairs) {
+    case 0: return launch_impl<D, CAUSAL, 0, 3, FP8>(p, stream);
+    case 4: return deg4 ? launch_impl<D, CAUSAL, 4, 4, FP8>(p, stream) : launch_impl<D, CAUSAL, 4, 3, FP8>(p, stream);
+    default: return deg4 ? launch_impl<D, CAUSAL, 2, 4, FP8>(p, stream) : launch_impl<D, CAUSAL, 2, 3, FP8>(p, stream);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_tile_bf16(const FwdParams& p, int d, bool causal, cudaStream_t stream) {
+  if (d == 64) return causal ? launch_np<64, true, false>(p, stream) : launch_np<64, false, false>(p, stream);
+  return causal ? launch_np<128, true, false>(p, stream) : launch_np<128, false, false>(p, stream);
+}
+
+cudaError_t launch_fwd_tile_fp8(const FwdParams& p, bool causal, cudaStream_t stream) {
+  return causal ? launch_np<128, true, true>(p, stream) : launch_np<128, false, true>(p, stream);
+}
+
+}  // namespace fa

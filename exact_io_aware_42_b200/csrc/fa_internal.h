@@ -25,12 +25,18 @@ cudaError_t set_smem_once(int bytes) {
 constexpr int kBlockM = 128;      // query rows per tile (one TMEM lane per row)
 constexpr int kBlockN = 128;      // keys per K/V tile
 constexpr float kRescaleTau = 8.0f;   // log2 units; see the forward kernel
+// FP8 forward: P is stored as E4M3 of p * f with f <= 256, so p may exceed 1
+// by at most 2^0.75 (430.5 < 448, the largest E4M3 value); measured faster
+// than rescaling on every increase of the max (B2 H16 N8192: 1142 vs 1106
+// TFLOPS)
+constexpr float kRescaleTauFp8 = 0.75f;
 constexpr int kNoWindow = 1 << 30;    // window value meaning "no sliding window" (> any N + 128)
 
 struct FwdParams {
   CUtensorMap tm_q;     // [BH, N, d] bf16 or e4m3, box {64 or 128 elems, 128, 1}
   CUtensorMap tm_k;
   CUtensorMap tm_v;
+  CUtensorMap tm_o;     // bf16 output, box {64, 128, 1}: the one-CTA-per-item kernel's TMA store
   uint16_t* o;          // bf16 output [BH, N, d]
   float* lse;           // [BH, N]
   unsigned int* status;
@@ -52,7 +58,7 @@ struct FwdParams {
   int poly_deg;         // degree of that polynomial (3 or 4)
   int sms;              // multiprocessor count: persistent grid size
   int split_pv;         // d <= 128: 1: P V issued in two 64-key halves as P arrives; 0: after all of P
-  int persistent;       // 1: grid of min(items, SMs) CTAs; 0: one CTA per work item
+  int persistent;       // 1: persistent kernel, min(items, SMs) CTAs; 0: one CTA per work item
 };
 
 // Default share of the softmax exp2 taken by the polynomial (of 8 column
@@ -67,11 +73,21 @@ constexpr int kDefaultPolyPairsD256 = 0;
 constexpr int kDefaultPolyDegree = 4;
 // measured on B200 (cfg B4 H16 N4096 d128 causal: 903 vs 870 TFLOPS; N 16384: 1060 vs 1006)
 constexpr int kDefaultFwdSplitPv = 0;
-constexpr int kDefaultFwdPersistent = 1;
+// d <= 128: which forward kernel runs by default, chosen by measurement on
+// B200 (same-process A/B): one CTA per work item was faster at d = 128
+// (bf16 B4 H16 N4096 causal 932 vs 901 TFLOPS; FP8 B2 H16 N8192 1106 vs
+// 957) and at d = 64 (B4 H32 N4096 causal 533 vs 520).
+constexpr int kDefaultFwdPersistentD128 = 0;
+constexpr int kDefaultFwdPersistentD64 = 0;
+constexpr int kDefaultFwdPersistentFp8 = 0;
 // FP8 forward: share of the exp2 on the polynomial (pairs of 8)
 constexpr int kDefaultPolyPairsFp8 = 0;
 
+// Persistent kernel (d = 64, 128; FP8 d = 128): min(items, SMs) CTAs.
 cudaError_t launch_fwd_bf16(const FwdParams& p, int d, bool causal, cudaStream_t stream);
+// One CTA per work item (d = 64, 128; FP8 d = 128); needs tm_o.
+cudaError_t launch_fwd_tile_bf16(const FwdParams& p, int d, bool causal, cudaStream_t stream);
+cudaError_t launch_fwd_tile_fp8(const FwdParams& p, bool causal, cudaStream_t stream);
 // Head dim 256 (one query tile per work item, K/V streamed as 64-column panels).
 cudaError_t launch_fwd_d256(const FwdParams& p, bool causal, cudaStream_t stream);
 // One CTA waiting on an mbarrier nothing arrives on (failure-path self-test).

@@ -24,7 +24,7 @@ import torch
 
 import oracle
 from exact_io_aware_42_b200 import inputs
-from tests.helpers import FP8_REL_RMS, f64, rel_rms
+from tests.helpers import FP8_REL_RMS, LSE_MAX_ABS, f64, rel_rms
 
 pytestmark = pytest.mark.gpu
 
@@ -262,3 +262,31 @@ def test_fp8_fwd_exp2_split_variants(pairs):
         o_ref, _ = oracle.attn_fwd_ref(deq[0], deq[1], deq[2], 1 / math.sqrt(128), causal)
         assert rel_rms(o.cpu(), o_ref) <= FP8_KERNEL_REL_RMS
         assert rel_rms(o.cpu(), o_sfu.cpu()) <= 1e-2
+
+
+@pytest.mark.parametrize("persistent", [0, 1])
+def test_fp8_fwd_kernel_variants_and_lse(persistent):
+    """Both FP8 forward kernels (one CTA per work item; the persistent grid):
+    O within the E4M3 rounding bound of P against the oracle on the
+    dequantised inputs, and L within the bf16 path's bound (the scores are
+    exact products of the dequantised inputs, and the row sum is fp32), on
+    more work items than SMs."""
+    fa = _fa()
+    q, k, v = inputs.make_qkv(1, 24, 1500, 128, seed=97 + persistent, outliers=True)
+    q8, sq = fa.quant_fp8(q.cuda())
+    k8, sk = fa.quant_fp8(k.cuda())
+    v8, sv = fa.quant_fp8(v.cuda())
+    deq = [oracle.dequant_fp8_ref(c.cpu().numpy(), s_.cpu().numpy()) for c, s_ in ((q8, sq), (k8, sk), (v8, sv))]
+    fa.set_tuning("fwd_persistent", persistent)
+    try:
+        for causal in (False, True):
+            o, lse = fa.fwd_fp8(q8, k8, v8, sq, sk, sv, causal=causal)
+            torch.cuda.synchronize()
+            assert fa.get_status() == 0
+            for h in (0, 11, 23):
+                sl = (slice(0, 1), slice(h, h + 1))
+                o_ref, l_ref = oracle.attn_fwd_ref(deq[0][sl], deq[1][sl], deq[2][sl], 1 / math.sqrt(128), causal)
+                assert rel_rms(o[sl].cpu(), o_ref) <= FP8_KERNEL_REL_RMS, (h, causal)
+                assert np.max(np.abs(f64(lse[sl].cpu()) - l_ref)) <= LSE_MAX_ABS, (h, causal)
+    finally:
+        fa.set_tuning("fwd_persistent", -1)

@@ -12,7 +12,8 @@ import torch
 
 import oracle
 from exact_io_aware_42_b200 import inputs
-from tests.helpers import assert_fwd_close, f64, LSE_MAX_ABS, O_MAX_ABS
+from tests.helpers import (assert_fwd_close, f64, LSE_MAX_ABS, max_abs, max_scaled_err, O_MAX_ABS,
+                           O_REL_RMS, rel_rms)
 
 pytestmark = pytest.mark.gpu
 
@@ -165,6 +166,39 @@ def test_fwd_exp2_split_variants(d, pairs, deg, causal, restore_tuning):
     o, lse = run_fwd(q, k, v, causal)
     o_ref, l_ref = oracle.attn_fwd_ref(q, k, v, 1 / math.sqrt(d), causal)
     assert_fwd_close(o, lse, o_ref, l_ref, f"d={d} pairs={pairs} deg={deg} causal={causal}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("persistent,split", [(0, 0), (1, 0), (1, 1)])
+def test_fwd_kernel_variants_every_head(d, persistent, split, restore_tuning):
+    """Both forward kernels (one CTA per work item; the persistent grid, with
+    and without the split P V) on a problem with more work items than SMs:
+    every head matches the oracle on sampled rows, causal and not, plus one
+    whole head."""
+    fa = _fa()
+    fa.set_tuning("fwd_persistent", persistent)
+    fa.set_tuning("fwd_split_pv", split)
+    assert fa.get_tuning("fwd_persistent", d) == persistent
+    N, H = 2048, 40
+    q, k, v = inputs.make_qkv(1, H, N, d, seed=700 + d + 2 * persistent + split)
+    # causal rows 0 and 1 average one or two keys, so |O| reaches a few units
+    # and one bf16 half-ulp of O alone approaches 1e-2: O's elementwise bound
+    # is taken relative to max(1, |O|) here (the masks tests' reading)
+    rows = np.array([0, 1, 127, 128, 255, 256, 1023, 1500, 2046, 2047])
+    for causal in (False, True):
+        o, lse = run_fwd(q, k, v, causal)
+        for h in list(range(H)) + [None]:
+            if h is None:    # one whole head
+                sl = (slice(0, 1), slice(33, 34))
+                o_r, l_r = oracle.attn_fwd_ref(q[sl], k[sl], v[sl], 1 / math.sqrt(d), causal)
+                o_k, l_k = o[sl], lse[sl]
+            else:
+                o_r, l_r = oracle.attn_fwd_rows_ref(q[0, h], k[0, h], v[0, h], 1 / math.sqrt(d), causal, rows)
+                o_k, l_k = o[0, h, rows], lse[0, h, rows]
+            tag = f"h={h} causal={causal}"
+            assert max_scaled_err(o_k, o_r) <= O_MAX_ABS, tag
+            assert rel_rms(o_k, o_r) <= O_REL_RMS, tag
+            assert max_abs(l_k, l_r) <= LSE_MAX_ABS, tag
 
 
 @pytest.mark.parametrize("causal", [False, True])
