@@ -19,7 +19,8 @@ from typing import Optional
 import torch
 
 from ._lib import (TUNE_BWD_PAIR, TUNE_BWD_POLY_GROUPS, TUNE_DQ_POLY_PAIRS, TUNE_FP8_POLY_PAIRS,
-                   TUNE_FWD_PERSISTENT, TUNE_FWD_POLY_DEGREE, TUNE_FWD_POLY_PAIRS, TUNE_FWD_SPLIT_PV, check, lib)
+                   TUNE_FWD_PERSISTENT, TUNE_FWD_POLY_DEGREE, TUNE_FWD_POLY_PAIRS,
+                   TUNE_FWD_SPLIT_PV, check, lib)
 
 __all__ = ["fwd", "bwd", "bwd_workspace_size", "bwd_noalloc", "quant_fp8", "fwd_fp8", "get_status",
            "clear_status", "n_blocks", "set_tuning", "get_tuning", "TUNING_KNOBS"]

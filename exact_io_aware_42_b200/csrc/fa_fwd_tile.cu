@@ -81,6 +81,8 @@ struct TileCfg {
   // d = 128 has no room for it and stores P over the consumed S_t
   static constexpr bool kSepP = (D == 64);
   static constexpr uint32_t kColP = 384;
+  // P outside S: S_t(j+1) may start as soon as S_t(j) has been read out
+  static constexpr bool kEarlyS = kSepP;
 };
 static_assert(TileCfg<128, true>::kSmemBytes <= 232448, "fp8 forward shared memory");
 static_assert(TileCfg<128, false>::kSmemBytes <= 232448, "bf16 forward shared memory");
@@ -277,9 +279,9 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(const __grid_constant_
           ++seq;
         }
         tc_fence_after();
-        if constexpr (C::kSepP) {
-          // S_t(j+1) as soon as the softmax has read S_t(j) out (P_t(j) has
-          // a region of its own), then the P V products as P arrives
+        if constexpr (C::kEarlyS) {
+          // S_t(j+1) as soon as the softmax has read S_t(j) out (P_t(j) is
+          // elsewhere), then the P V products as P arrives
           if (has_next) {
             if (j + 1 < n_t[0]) {
               if (!(ok = mbar_wait(bar(bar_sfree<NS>(0)), j & 1, ab, kSiteMmaSfree))) break;
@@ -371,7 +373,7 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(const __grid_constant_
       tc_fence_after();
       uint32_t u[128];
       tmem_ld128(tS, u);
-      if constexpr (C::kSepP) {   // S_t may be overwritten by S_t(j+1) from here on
+      if constexpr (C::kEarlyS) {   // S_t may be overwritten by S_t(j+1) from here on
         tc_fence_before();
         mbar_arrive(bar(bar_sfree<NS>(t)));
       }
@@ -477,9 +479,9 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(const __grid_constant_
             u[i] = pack_bf16x2(p0, p1);
           }
         }
-        if constexpr (!C::kSepP) tmem_st64(tS, *reinterpret_cast<uint32_t(*)[64]>(&u[0]));
+        if constexpr (!C::kEarlyS) tmem_st64(tS, *reinterpret_cast<uint32_t(*)[64]>(&u[0]));
       }
-      if constexpr (!C::kSepP) tmem_st_wait();
+      if constexpr (!C::kEarlyS) tmem_st_wait();
       float sum4[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -489,26 +491,25 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(const __grid_constant_
       }
       l = l * alpha + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
       if (j > 0) {
-        // PV(j-1) must be done before O is touched or PV(j) is released;
-        // waiting every tile also keeps this waiter within one phase.
+        // PV(j-1) must be done before O is touched or PV(j) is released (and,
+        // with P outside S, before P_t is overwritten); waiting every tile
+        // also keeps this waiter within one phase.
         if (!(ok = mbar_wait_warp(bar(bar_pv<NS>(t)), (j - 1) & 1, ab, kSiteSmPv))) break;
         tc_fence_after();
-        if (__any_sync(0xffffffffu, need)) {
+      }
+      // P outside S goes out first, so its registers are free for the O rescale
+      if constexpr (C::kSepP) tmem_st64(tP, *reinterpret_cast<uint32_t(*)[64]>(&u[0]));
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
-          for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t u[32];
-            tmem_ld32(tO + ch * 32, u);
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t w[32];
+          tmem_ld32(tO + ch * 32, w);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-            tmem_st32(tO + ch * 32, u);
-          }
-          tmem_st_wait();
+          for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
+          tmem_st32(tO + ch * 32, w);
         }
       }
-      if constexpr (C::kSepP) {   // P_t's region is free once P V_t(j-1) is done (waited above)
-        tmem_st64(tP, *reinterpret_cast<uint32_t(*)[64]>(&u[0]));
-        tmem_st_wait();
-      }
+      if (C::kSepP || (j > 0 && __any_sync(0xffffffffu, need))) tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(bar_p<NS>(t)));
     }

@@ -27,8 +27,8 @@ constexpr int kBlockN = 128;      // keys per K/V tile
 constexpr float kRescaleTau = 8.0f;   // log2 units; see the forward kernel
 // FP8 forward: P is stored as E4M3 of p * f with f <= 256, so p may exceed 1
 // by at most 2^0.75 (430.5 < 448, the largest E4M3 value); measured faster
-// than rescaling on every increase of the max (B2 H16 N8192: 1142 vs 1106
-// TFLOPS)
+// than rescaling on every increase of the max (B2 H16 N8192, two same-process
+// A/B runs: 1126 and 1142 vs 1114 and 1106 TFLOPS)
 constexpr float kRescaleTauFp8 = 0.75f;
 constexpr int kNoWindow = 1 << 30;    // window value meaning "no sliding window" (> any N + 128)
 
@@ -75,8 +75,9 @@ constexpr int kDefaultPolyDegree = 4;
 constexpr int kDefaultFwdSplitPv = 0;
 // d <= 128: which forward kernel runs by default, chosen by measurement on
 // B200 (same-process A/B): one CTA per work item was faster at d = 128
-// (bf16 B4 H16 N4096 causal 932 vs 901 TFLOPS; FP8 B2 H16 N8192 1106 vs
-// 957) and at d = 64 (B4 H32 N4096 causal 533 vs 520).
+// (bf16 B4 H16 N4096 causal 926-939 vs 901-913 TFLOPS; FP8 B2 H16 N8192
+// 1106-1126 vs 957) and at d = 64, where it also keeps P in TMEM columns of
+// its own (B4 H32 N4096 causal 574-579 vs 520).
 constexpr int kDefaultFwdPersistentD128 = 0;
 constexpr int kDefaultFwdPersistentD64 = 0;
 constexpr int kDefaultFwdPersistentFp8 = 0;
