@@ -437,6 +437,7 @@ def config_block(graph: bool):
                          if w["d"] == 128 else "none (the FP8 forward is built for d = 128)"),
             "bwd_pair": TUNING.get("bwd_pair"),
             "fwd_split_pv": TUNING.get("fwd_split_pv"), "fwd_persistent": TUNING.get("fwd_persistent"),
+            "fwd_causal_group": TUNING.get("fwd_causal_group"),
             "exp2_split": {"fwd_poly_pairs": TUNING.get("fwd_poly_pairs"),
                            "fwd_poly_degree": TUNING.get("fwd_poly_degree"),
                            "fp8_poly_pairs": TUNING.get("fp8_poly_pairs")}}
@@ -471,11 +472,12 @@ def run_ours(args):
         fa.set_tuning("fp8_poly_pairs", args.fp8_poly_pairs)
     if args.bwd_pair is not None:
         fa.set_tuning("bwd_pair", args.bwd_pair)
-    for knob in ("fwd_split_pv", "fwd_persistent"):
+    for knob in ("fwd_split_pv", "fwd_persistent", "fwd_causal_group"):
         if getattr(args, knob) is not None:
             fa.set_tuning(knob, getattr(args, knob))
     TUNING.update({k_: fa.get_tuning(k_, d) for k_ in ("fwd_poly_pairs", "fwd_poly_degree", "fp8_poly_pairs",
-                                                       "bwd_pair", "fwd_split_pv", "fwd_persistent")})
+                                                       "bwd_pair", "fwd_split_pv", "fwd_persistent",
+                                                       "fwd_causal_group")})
     graph = {"auto": latency_bound(w), "on": True, "off": False}[args.graph]
     hq, hk, hv, hdo = inputs.make_gqa(B, H, H_kv, N, d, w["seed"] + rank, with_do=True)
     signs = inputs.signs(d).to(dev)
@@ -647,6 +649,8 @@ def main():
                     help="deterministic backward at d = 128: dK, dV on CTA pairs (1) or single CTAs (0)")
     ap.add_argument("--fwd-split-pv", type=int, choices=[0, 1], default=None)
     ap.add_argument("--fwd-persistent", type=int, choices=[0, 1], default=None)
+    ap.add_argument("--fwd-causal-group", type=int, choices=[0, 1], default=None,
+                    help="causal forward: longest first within L2-sized head groups (1) or over all heads (0)")
     ap.add_argument("--fp8-poly-pairs", type=int, choices=[0, 2, 4], default=None,
                     help="FP8 forward exp2 split for a measurement (default: the library's)")
     args = ap.parse_args()

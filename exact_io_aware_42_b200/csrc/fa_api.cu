@@ -129,6 +129,20 @@ int fwd_persistent(int d, bool fp8) {
   return fp8 ? kDefaultFwdPersistentFp8 : d == 64 ? kDefaultFwdPersistentD64 : kDefaultFwdPersistentD128;
 }
 
+int fwd_causal_group() {
+  const int v = tune_raw(FA_TUNE_FWD_CAUSAL_GROUP);
+  return v >= 0 ? v : kDefaultFwdCausalGroup;
+}
+
+// Heads per group of the causal item order (see FwdParams::group_heads):
+// K and V of the group's K/V heads within kCausalGroupBytes.
+int fwd_group_heads(int BH, int kv_group, int N, int d, int elem_bytes) {
+  if (!fwd_causal_group()) return BH;
+  const long long kv_bytes = 2ll * N * d * elem_bytes;   // K and V of one K/V head
+  const long long g = kCausalGroupBytes / kv_bytes * kv_group;
+  return static_cast<int>(g < 1 ? 1 : g > BH ? BH : g);
+}
+
 int bwd_pair() {
   const int v = tune_raw(FA_TUNE_BWD_PAIR);
   return v >= 0 ? v : kDefaultBwdPair;
@@ -282,6 +296,7 @@ extern "C" fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void
   p.sms = di->sms;
   p.split_pv = fwd_split_pv();
   p.persistent = d == 256 ? 1 : fwd_persistent(d, false);
+  p.group_heads = fwd_group_heads(B * H, H / H_kv, N, d, 2);
   if (!p.persistent && !encode_3d(&p.tm_o, o, bf, 2, d, N, BH, 64, kBlockM)) return FA_ERR_INVALID_ARG;
   p.lse = lse;
   p.status = di->status;
@@ -537,6 +552,7 @@ extern "C" fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v
   p.sms = di->sms;
   p.split_pv = fwd_split_pv();
   p.persistent = fwd_persistent(d, true);
+  p.group_heads = fwd_group_heads(B * H, H / H_kv, N, d, 1);
   if (!p.persistent &&
       !encode_3d(&p.tm_o, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, BH, 64, kBlockM))
     return FA_ERR_INVALID_ARG;
@@ -587,6 +603,7 @@ bool tuning_value_ok(int knob, int value) {
     case FA_TUNE_BWD_PAIR: return value == 0 || value == 1;
     case FA_TUNE_FWD_SPLIT_PV: return value == 0 || value == 1;
     case FA_TUNE_FWD_PERSISTENT: return value == 0 || value == 1;
+    case FA_TUNE_FWD_CAUSAL_GROUP: return value == 0 || value == 1;
     default: return false;
   }
 }
@@ -609,6 +626,7 @@ extern "C" int fa_get_tuning(int knob, int d) {
     case FA_TUNE_BWD_PAIR: return d == 128 ? bwd_pair() : 0;
     case FA_TUNE_FWD_SPLIT_PV: return fwd_split_pv();
     case FA_TUNE_FWD_PERSISTENT: return d == 256 ? 1 : fwd_persistent(d, false);
+    case FA_TUNE_FWD_CAUSAL_GROUP: return fwd_causal_group();
     default: return -1;
   }
 }

@@ -133,11 +133,23 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(const __grid_constant_
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Causal: the heaviest pairs of every head first (longest-first balances
-  // the uneven work).  Non-causal: head-major, so the resident CTAs cover a
-  // few heads whose K and V stay in L2.  Both orders measured on B200.
-  const int bh = CAUSAL ? blockIdx.x % p.BH : blockIdx.x / p.n_pairs;
-  const int pair = CAUSAL ? p.n_pairs - 1 - blockIdx.x / p.BH : blockIdx.x % p.n_pairs;
+  // Causal: within each group of group_heads heads, the heaviest pairs first
+  // (longest-first balances the uneven work; the hardware hands out CTAs in
+  // index order as SMs free up, so group boundaries cost no balance, and a
+  // group's K and V stay in L2 while its CTAs run).  Non-causal: head-major,
+  // so the resident CTAs cover a few heads whose K and V stay in L2.
+  int bh, pair;
+  if constexpr (CAUSAL) {
+    const int per_group = p.group_heads * p.n_pairs;
+    const int g = static_cast<int>(blockIdx.x) / per_group;
+    const int rr = static_cast<int>(blockIdx.x) - g * per_group;
+    const int gh = min(p.group_heads, p.BH - g * p.group_heads);   // the last group may be short
+    bh = g * p.group_heads + rr % gh;
+    pair = p.n_pairs - 1 - rr / gh;
+  } else {
+    bh = blockIdx.x / p.n_pairs;
+    pair = blockIdx.x % p.n_pairs;
+  }
   // Grouped K/V heads: query head h of batch b reads K/V head b * H_kv + h / G,
   // which in the flattened [B * H] index is bh / G.
   const int kvh = bh / p.kv_group;

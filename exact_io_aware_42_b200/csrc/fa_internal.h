@@ -59,6 +59,8 @@ struct FwdParams {
   int sms;              // multiprocessor count: persistent grid size
   int split_pv;         // d <= 128: 1: P V issued in two 64-key halves as P arrives; 0: after all of P
   int persistent;       // 1: persistent kernel, min(items, SMs) CTAs; 0: one CTA per work item
+  int group_heads;      // one-CTA-per-item kernel, causal: CTA order longest first within groups
+                        // of this many heads (>= BH: one group over all heads)
 };
 
 // Default share of the softmax exp2 taken by the polynomial (of 8 column
@@ -81,6 +83,14 @@ constexpr int kDefaultFwdSplitPv = 0;
 constexpr int kDefaultFwdPersistentD128 = 0;
 constexpr int kDefaultFwdPersistentD64 = 0;
 constexpr int kDefaultFwdPersistentFp8 = 0;
+// Causal CTA order of the one-CTA-per-item kernel, measured (same-process
+// A/B): grouping heads helped only once K and V of all heads far exceed L2
+// (B8 H16 N4096 d128: 948 vs 910 TFLOPS) and cost about 1% at B4 H16 N4096
+// (926 vs 932) and B1 H16 N16384, so the global longest-first order is the
+// default.
+constexpr int kDefaultFwdCausalGroup = 0;
+// K and V bytes of one head group in that order
+constexpr long long kCausalGroupBytes = 32ll << 20;
 // FP8 forward: share of the exp2 on the polynomial (pairs of 8)
 constexpr int kDefaultPolyPairsFp8 = 0;
 

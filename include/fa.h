@@ -262,6 +262,9 @@ fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v8, const fl
  *                           kernel always splits
  *  FA_TUNE_FWD_PERSISTENT   forward: one CTA per SM walking the work items (1)
  *                           or one CTA per work item (0)
+ *  FA_TUNE_FWD_CAUSAL_GROUP causal forward, one CTA per work item: longest
+ *                           first within groups of heads whose K and V fit in
+ *                           L2 together (1), or over all heads (0)
  * value -1 restores the built-in default.  Any other value, or an unknown
  * knob, is FA_ERR_INVALID_ARG.  fa_get_tuning returns the value a call with
  * head dim d would use now.
@@ -275,7 +278,8 @@ typedef enum fa_tune_knob {
   FA_TUNE_BWD_PAIR = 6,
   FA_TUNE_FWD_SPLIT_PV = 7,
   FA_TUNE_FWD_PERSISTENT = 8,
-  FA_TUNE_COUNT = 9
+  FA_TUNE_FWD_CAUSAL_GROUP = 9,
+  FA_TUNE_COUNT = 10
 } fa_tune_knob;
 fa_status fa_set_tuning(int knob, int value);
 int fa_get_tuning(int knob, int d);

@@ -169,18 +169,20 @@ def test_fwd_exp2_split_variants(d, pairs, deg, causal, restore_tuning):
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("persistent,split", [(0, 0), (1, 0), (1, 1)])
-def test_fwd_kernel_variants_every_head(d, persistent, split, restore_tuning):
-    """Both forward kernels (one CTA per work item; the persistent grid, with
-    and without the split P V) on a problem with more work items than SMs:
-    every head matches the oracle on sampled rows, causal and not, plus one
-    whole head."""
+@pytest.mark.parametrize("persistent,split,group", [(0, 0, 1), (0, 0, 0), (1, 0, 0), (1, 1, 0)])
+def test_fwd_kernel_variants_every_head(d, persistent, split, group, restore_tuning):
+    """Both forward kernels (one CTA per work item, with the grouped and the
+    global causal order; the persistent grid, with and without the split
+    P V) on a problem with more work items than SMs and, at d = 128, two head
+    groups (32 and 8 heads of N = 2048): every head matches the oracle on
+    sampled rows, causal and not, plus one whole head."""
     fa = _fa()
     fa.set_tuning("fwd_persistent", persistent)
     fa.set_tuning("fwd_split_pv", split)
+    fa.set_tuning("fwd_causal_group", group)
     assert fa.get_tuning("fwd_persistent", d) == persistent
     N, H = 2048, 40
-    q, k, v = inputs.make_qkv(1, H, N, d, seed=700 + d + 2 * persistent + split)
+    q, k, v = inputs.make_qkv(1, H, N, d, seed=700 + d + 4 * group + 2 * persistent + split)
     # causal rows 0 and 1 average one or two keys, so |O| reaches a few units
     # and one bf16 half-ulp of O alone approaches 1e-2: O's elementwise bound
     # is taken relative to max(1, |O|) here (the masks tests' reading)
