@@ -132,6 +132,7 @@ def measured_peaks():
 KERNEL_SOURCES = {
     "fwd": ("fa_fwd.cu",),
     "fwd_tile": ("fa_fwd_tile.cu",),
+    "fwd_q1": ("fa_fwd_q1.cu",),
     "fwd256": ("fa_fwd_d256.cu",),
     "bwd": ("fa_bwd.cu",),
     "bwd_dq": ("fa_bwd_dq.cu",),
@@ -437,7 +438,7 @@ def config_block(graph: bool):
                          if w["d"] == 128 else "none (the FP8 forward is built for d = 128)"),
             "bwd_pair": TUNING.get("bwd_pair"),
             "fwd_split_pv": TUNING.get("fwd_split_pv"), "fwd_persistent": TUNING.get("fwd_persistent"),
-            "fwd_causal_group": TUNING.get("fwd_causal_group"),
+            "fwd_causal_group": TUNING.get("fwd_causal_group"), "fwd_q1": TUNING.get("fwd_q1"),
             "exp2_split": {"fwd_poly_pairs": TUNING.get("fwd_poly_pairs"),
                            "fwd_poly_degree": TUNING.get("fwd_poly_degree"),
                            "fp8_poly_pairs": TUNING.get("fp8_poly_pairs")}}
@@ -472,12 +473,12 @@ def run_ours(args):
         fa.set_tuning("fp8_poly_pairs", args.fp8_poly_pairs)
     if args.bwd_pair is not None:
         fa.set_tuning("bwd_pair", args.bwd_pair)
-    for knob in ("fwd_split_pv", "fwd_persistent", "fwd_causal_group"):
+    for knob in ("fwd_split_pv", "fwd_persistent", "fwd_causal_group", "fwd_q1"):
         if getattr(args, knob) is not None:
             fa.set_tuning(knob, getattr(args, knob))
     TUNING.update({k_: fa.get_tuning(k_, d) for k_ in ("fwd_poly_pairs", "fwd_poly_degree", "fp8_poly_pairs",
                                                        "bwd_pair", "fwd_split_pv", "fwd_persistent",
-                                                       "fwd_causal_group")})
+                                                       "fwd_causal_group", "fwd_q1")})
     graph = {"auto": latency_bound(w), "on": True, "off": False}[args.graph]
     hq, hk, hv, hdo = inputs.make_gqa(B, H, H_kv, N, d, w["seed"] + rank, with_do=True)
     signs = inputs.signs(d).to(dev)
@@ -575,9 +576,16 @@ def run_ours(args):
         roof_bwd["frac_sustained"] = roof_bwd["achieved"] / sustained
         roof_bwd["frac_nominal_2250"] = roof_bwd["achieved"] / 2250.0
     pers = TUNING.get("fwd_persistent") == 1
-    fwd_name, fwd_src = (("fwd256_kernel", "fwd256") if d == 256 else ("fwd_kernel", "fwd") if pers
-                         else ("fwd_tile_kernel", "fwd_tile"))
-    fwd_desc = f"{fwd_name}<{d}, {cz}, bf16>" + (" (persistent)" if d == 256 or pers else " (one CTA per item)")
+    # the one-tile kernel: chosen explicitly, or by the library when the
+    # two-tile kernel would have fewer work items than SMs
+    n_pairs = ((N + 127) // 128 + 1) // 2
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    q1 = d != 256 and (TUNING.get("fwd_q1") == 1 or (TUNING.get("fwd_q1") == -1 and n_pairs * B * H < sms))
+    fwd_name, fwd_src = (("fwd256_kernel", "fwd256") if d == 256 else ("fwd_q1_kernel", "fwd_q1") if q1
+                         else ("fwd_kernel", "fwd") if pers else ("fwd_tile_kernel", "fwd_tile"))
+    fwd_desc = f"{fwd_name}<{d}, {cz}, bf16>" + (
+        " (persistent, one query tile per item)" if q1 else " (persistent)" if d == 256 or pers
+        else " (one CTA per item)")
     roof_fwd = roof(stages, per_stage, "fwd_bf16", fwd_desc, fwd_bytes(B, H, N, d, H_kv), burst, burst_note,
                     profiled_traffic(fwd_name, w["name"], fwd_src))
     roof_fwd["frac_sustained"] = roof_fwd["achieved"] / sustained
@@ -649,6 +657,8 @@ def main():
                     help="deterministic backward at d = 128: dK, dV on CTA pairs (1) or single CTAs (0)")
     ap.add_argument("--fwd-split-pv", type=int, choices=[0, 1], default=None)
     ap.add_argument("--fwd-persistent", type=int, choices=[0, 1], default=None)
+    ap.add_argument("--fwd-q1", type=int, choices=[0, 1], default=None,
+                    help="bf16 forward, d <= 128: one query tile per item with two score buffers (1)")
     ap.add_argument("--fwd-causal-group", type=int, choices=[0, 1], default=None,
                     help="causal forward: longest first within L2-sized head groups (1) or over all heads (0)")
     ap.add_argument("--fp8-poly-pairs", type=int, choices=[0, 2, 4], default=None,

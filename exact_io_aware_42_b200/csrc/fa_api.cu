@@ -129,6 +129,13 @@ int fwd_persistent(int d, bool fp8) {
   return fp8 ? kDefaultFwdPersistentFp8 : d == 64 ? kDefaultFwdPersistentD64 : kDefaultFwdPersistentD128;
 }
 
+// The one-tile forward kernel: set explicitly, or (default) when the
+// two-tile kernel would have fewer work items than SMs.
+int fwd_q1(long long pair_items, int sms) {
+  const int v = tune_raw(FA_TUNE_FWD_Q1);
+  return v >= 0 ? v : (pair_items < sms ? 1 : 0);
+}
+
 int fwd_causal_group() {
   const int v = tune_raw(FA_TUNE_FWD_CAUSAL_GROUP);
   return v >= 0 ? v : kDefaultFwdCausalGroup;
@@ -314,7 +321,10 @@ extern "C" fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void
   p.poly_pairs = poly_pairs(d);
   p.poly_deg = poly_degree();
   if (d == 256 && static_cast<long long>(p.n_kv) * BH > kMaxWorkItems) return FA_ERR_UNSUPPORTED;
+  const bool q1 = d != 256 && fwd_q1(static_cast<long long>(p.n_pairs) * BH, p.sms);
+  if (q1 && static_cast<long long>(p.n_kv) * BH > kMaxWorkItems) return FA_ERR_UNSUPPORTED;
   cudaError_t e = d == 256 ? launch_fwd_d256(p, causal != 0, static_cast<cudaStream_t>(stream))
+                  : q1 ? launch_fwd_q1_bf16(p, d, causal != 0, static_cast<cudaStream_t>(stream))
                   : p.persistent ? launch_fwd_bf16(p, d, causal != 0, static_cast<cudaStream_t>(stream))
                                  : launch_fwd_tile_bf16(p, d, causal != 0, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
@@ -604,6 +614,7 @@ bool tuning_value_ok(int knob, int value) {
     case FA_TUNE_FWD_SPLIT_PV: return value == 0 || value == 1;
     case FA_TUNE_FWD_PERSISTENT: return value == 0 || value == 1;
     case FA_TUNE_FWD_CAUSAL_GROUP: return value == 0 || value == 1;
+    case FA_TUNE_FWD_Q1: return value == 0 || value == 1;
     default: return false;
   }
 }
@@ -627,6 +638,7 @@ extern "C" int fa_get_tuning(int knob, int d) {
     case FA_TUNE_FWD_SPLIT_PV: return fwd_split_pv();
     case FA_TUNE_FWD_PERSISTENT: return d == 256 ? 1 : fwd_persistent(d, false);
     case FA_TUNE_FWD_CAUSAL_GROUP: return fwd_causal_group();
+    case FA_TUNE_FWD_Q1: return d == 256 ? 0 : tune_raw(FA_TUNE_FWD_Q1);   // -1: chosen per call
     default: return -1;
   }
 }

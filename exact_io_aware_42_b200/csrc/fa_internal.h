@@ -89,6 +89,11 @@ constexpr int kDefaultFwdPersistentFp8 = 0;
 // (926 vs 932) and B1 H16 N16384, so the global longest-first order is the
 // default.
 constexpr int kDefaultFwdCausalGroup = 0;
+// bf16 forward at d <= 128: the one-tile kernel with two score buffers runs
+// by default only where the two-tile kernel would have fewer work items
+// (pairs of query tiles) than SMs; measured on B200: B2 H8 N1024 d64 causal
+// 105 vs 87 TFLOPS, while with at least one pair per SM the two-tile kernel
+// wins (B4 H16 N4096 d128 causal 926 vs 776).
 // K and V bytes of one head group in that order
 constexpr long long kCausalGroupBytes = 32ll << 20;
 // FP8 forward: share of the exp2 on the polynomial (pairs of 8)
@@ -96,6 +101,8 @@ constexpr int kDefaultPolyPairsFp8 = 0;
 
 // Persistent kernel (d = 64, 128; FP8 d = 128): min(items, SMs) CTAs.
 cudaError_t launch_fwd_bf16(const FwdParams& p, int d, bool causal, cudaStream_t stream);
+// One 128-row query tile per work item, two score buffers, persistent grid (bf16, d = 64, 128).
+cudaError_t launch_fwd_q1_bf16(const FwdParams& p, int d, bool causal, cudaStream_t stream);
 // One CTA per work item (d = 64, 128; FP8 d = 128); needs tm_o.
 cudaError_t launch_fwd_tile_bf16(const FwdParams& p, int d, bool causal, cudaStream_t stream);
 cudaError_t launch_fwd_tile_fp8(const FwdParams& p, bool causal, cudaStream_t stream);

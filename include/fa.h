@@ -265,6 +265,12 @@ fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v8, const fl
  *  FA_TUNE_FWD_CAUSAL_GROUP causal forward, one CTA per work item: longest
  *                           first within groups of heads whose K and V fit in
  *                           L2 together (1), or over all heads (0)
+ *  FA_TUNE_FWD_Q1           bf16 forward, d <= 128: one 128-row query tile per
+ *                           work item with two score buffers (1), or two query
+ *                           tiles per CTA (0; FA_TUNE_FWD_PERSISTENT picks which);
+ *                           by default chosen per call (the one-tile kernel when
+ *                           the problem has fewer pairs of query tiles than the
+ *                           device has SMs), which fa_get_tuning reports as -1
  * value -1 restores the built-in default.  Any other value, or an unknown
  * knob, is FA_ERR_INVALID_ARG.  fa_get_tuning returns the value a call with
  * head dim d would use now.
@@ -279,7 +285,8 @@ typedef enum fa_tune_knob {
   FA_TUNE_FWD_SPLIT_PV = 7,
   FA_TUNE_FWD_PERSISTENT = 8,
   FA_TUNE_FWD_CAUSAL_GROUP = 9,
-  FA_TUNE_COUNT = 10
+  FA_TUNE_FWD_Q1 = 10,
+  FA_TUNE_COUNT = 11
 } fa_tune_knob;
 fa_status fa_set_tuning(int knob, int value);
 int fa_get_tuning(int knob, int d);

@@ -143,10 +143,11 @@ def test_tuning_controls(L):
     assert L.fa_get_tuning(TUNE_FWD_POLY_DEGREE, 64) in (3, 4)
     assert L.fa_get_tuning(TUNE_DQ_POLY_PAIRS, 128) == 0
     assert L.fa_get_tuning(99, 64) == -1
-    from exact_io_aware_42_b200._lib import TUNE_FWD_CAUSAL_GROUP, TUNE_FWD_PERSISTENT
-    for knob in (TUNE_FWD_PERSISTENT, TUNE_FWD_CAUSAL_GROUP):
+    from exact_io_aware_42_b200._lib import TUNE_FWD_CAUSAL_GROUP, TUNE_FWD_PERSISTENT, TUNE_FWD_Q1
+    assert L.fa_get_tuning(TUNE_FWD_Q1, 128) == -1      # chosen per call by default
+    for knob in (TUNE_FWD_PERSISTENT, TUNE_FWD_CAUSAL_GROUP, TUNE_FWD_Q1):
         default = L.fa_get_tuning(knob, 128)
-        assert default in (0, 1)
+        assert default in ((-1,) if knob == TUNE_FWD_Q1 else (0, 1))
         for v in (0, 1):
             assert L.fa_set_tuning(knob, v) == 0 and L.fa_get_tuning(knob, 128) == v
         assert L.fa_set_tuning(knob, 2) == 1

@@ -169,8 +169,9 @@ def test_fwd_exp2_split_variants(d, pairs, deg, causal, restore_tuning):
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("persistent,split,group", [(0, 0, 1), (0, 0, 0), (1, 0, 0), (1, 1, 0)])
-def test_fwd_kernel_variants_every_head(d, persistent, split, group, restore_tuning):
+@pytest.mark.parametrize("persistent,split,group,q1", [(0, 0, 1, 0), (0, 0, 0, 0), (1, 0, 0, 0), (1, 1, 0, 0),
+                                                      (0, 0, 0, 1)])
+def test_fwd_kernel_variants_every_head(d, persistent, split, group, q1, restore_tuning):
     """Both forward kernels (one CTA per work item, with the grouped and the
     global causal order; the persistent grid, with and without the split
     P V) on a problem with more work items than SMs and, at d = 128, two head
@@ -180,9 +181,10 @@ def test_fwd_kernel_variants_every_head(d, persistent, split, group, restore_tun
     fa.set_tuning("fwd_persistent", persistent)
     fa.set_tuning("fwd_split_pv", split)
     fa.set_tuning("fwd_causal_group", group)
-    assert fa.get_tuning("fwd_persistent", d) == persistent
+    fa.set_tuning("fwd_q1", q1)
+    assert fa.get_tuning("fwd_persistent", d) == persistent and fa.get_tuning("fwd_q1", d) == q1
     N, H = 2048, 40
-    q, k, v = inputs.make_qkv(1, H, N, d, seed=700 + d + 4 * group + 2 * persistent + split)
+    q, k, v = inputs.make_qkv(1, H, N, d, seed=700 + d + 8 * q1 + 4 * group + 2 * persistent + split)
     # causal rows 0 and 1 average one or two keys, so |O| reaches a few units
     # and one bf16 half-ulp of O alone approaches 1e-2: O's elementwise bound
     # is taken relative to max(1, |O|) here (the masks tests' reading)
@@ -238,3 +240,32 @@ def test_fwd_d256_exp2_split(pairs, deg, restore_tuning):
         assert_fwd_close(o, lse, o_ref, l_ref, f"d=256 pairs={pairs} deg={deg} causal={causal}")
 
 
+
+
+@pytest.mark.parametrize("q1", [0, 1])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N", [1, 7, 127, 129, 255, 300, 513])
+def test_fwd_kernels_ragged_masks_groups(N, d, q1, restore_tuning):
+    """Both bf16 forward kernels for d <= 128 (two query tiles per CTA; one
+    query tile with two score buffers and P in its own TMEM columns, which
+    the library picks by itself for problems this small) on ragged N, causal
+    and not, with grouped K/V heads, a sliding window and ALiBi: the same
+    tolerances as every other forward variant (O elementwise relative to
+    max(1, |O|) where masks leave few keys)."""
+    fa = _fa()
+    fa.set_tuning("fwd_q1", q1)
+    assert fa.get_tuning("fwd_q1", d) == q1
+    q, k, v = inputs.make_gqa(2, 4, 2, N, d, seed=900 + N + d + q1)
+    scale = 1 / math.sqrt(d)
+    slopes = torch.tensor([2.0 ** (-8 * (h + 1) / 4) for h in range(4)], dtype=torch.float32)
+    for causal, window, alibi in ((False, None, None), (True, None, None), (True, 100, None), (True, None, slopes)):
+        o, lse = fa.fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, window=window,
+                        alibi=None if alibi is None else alibi.cuda())
+        torch.cuda.synchronize()
+        assert fa.get_status() == 0
+        o_ref, l_ref = oracle.attn_fwd_gqa_ref(q, k, v, scale, causal, window=window,
+                                              alibi=None if alibi is None else alibi.numpy())
+        tag = f"N={N} d={d} causal={causal} window={window} alibi={alibi is not None}"
+        assert max_scaled_err(o.cpu(), o_ref) <= O_MAX_ABS, tag
+        assert rel_rms(o.cpu(), o_ref) <= O_REL_RMS, tag
+        assert max_abs(lse.cpu(), l_ref) <= LSE_MAX_ABS, tag
