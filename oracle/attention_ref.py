@@ -40,7 +40,7 @@ forms, permutation and shift invariances, and the hand-worked fixture in
 """
 from __future__ import annotations
 
-from typing import NamedTuple, Sequence
+from typing import Optional, NamedTuple, Sequence
 
 import numpy as np
 
@@ -217,7 +217,8 @@ def online_softmax_ref(x, block_sizes: Sequence[int]):
     return m, ell, np.exp(x - m) / ell
 
 
-def attn_fwd_online_ref(q, k, v, scale: float, causal: bool, block_sizes: Sequence[int]):
+def attn_fwd_online_ref(q, k, v, scale: float, causal: bool, block_sizes: Sequence[int],
+                        tau_log2: float = 0.0, stats: Optional[dict] = None):
     """Attention for one head with K/V streamed in blocks, fp64.
 
     This is the algorithm the pages describe ([Concept] "How it works",
@@ -226,6 +227,14 @@ def attn_fwd_online_ref(q, k, v, scale: float, causal: bool, block_sizes: Sequen
     the running output o by the same factor e^{m_old - m_new} and add the new
     block's e^{S - m_new} V; after the last block divide by l once (deferred
     normalisation, [Lineage] "FA2 (2023)", refinement 2) and emit L = m + ln l.
+
+    ``tau_log2`` > 0 is the conditional rescale ([Librarian] "FA4", idea 2;
+    [Lineage] "FA4 (2026)", change 2), in the reading that the pages leave
+    open: the running max moves only when a block's max exceeds it by more
+    than tau (log2 units, i.e. by a factor 2^tau); until then the stale max
+    is used for p, l, o and L alike, so p <= 2^tau and the result is the
+    same up to rounding.  ``stats``, if given, receives the number of
+    rescales and the largest p used.
 
     q: [N_q, d], k and v: [N_k, d].  Returns (O [N_q, d], L [N_q]).
     """
@@ -236,6 +245,8 @@ def attn_fwd_online_ref(q, k, v, scale: float, causal: bool, block_sizes: Sequen
     n_q = q.shape[0]
     o = np.zeros((n_q, v.shape[1]))
     lse = np.zeros(n_q)
+    tau = float(tau_log2) * np.log(2.0)       # the threshold in the natural-log units of S
+    rescales, p_max = 0, 0.0
     for i in range(n_q):
         m, ell = -np.inf, 0.0
         acc = np.zeros(v.shape[1])
@@ -246,16 +257,22 @@ def attn_fwd_online_ref(q, k, v, scale: float, causal: bool, block_sizes: Sequen
             start += bs
             if s_blk.size == 0:
                 continue
-            m_next = max(m, float(np.max(s_blk)))
-            if m_next == -np.inf:
+            m_blk = float(np.max(s_blk))
+            if m_blk == -np.inf and m == -np.inf:
                 continue
-            alpha = 0.0 if m == -np.inf else np.exp(m - m_next)
-            p_blk = np.exp(s_blk - m_next)
+            alpha = 1.0
+            if m == -np.inf or m_blk > m + tau:   # move the running max
+                alpha = 0.0 if m == -np.inf else np.exp(m - m_blk)
+                m = m_blk
+                rescales += 1
+            p_blk = np.exp(s_blk - m)
+            p_max = max(p_max, float(np.max(p_blk)))
             ell = alpha * ell + float(np.sum(p_blk))
             acc = alpha * acc + p_blk @ v_blk
-            m = m_next
         o[i] = acc / ell
         lse[i] = m + np.log(ell)
+    if stats is not None:
+        stats["rescales"], stats["p_max"] = rescales, p_max
     return o, lse
 
 

@@ -243,6 +243,32 @@ def test_online_attention_matches_definition():
             np.testing.assert_allclose(lse, l_ref[0, 0], rtol=1e-12, atol=1e-13)
 
 
+def test_conditional_rescale_is_exact_and_bounded():
+    """The reading of the conditional rescale (the running max kept until a
+    block's max exceeds it by more than tau, log2 units; the stale max used
+    for p, l, o and L alike): O and L equal the two-pass definition for
+    tau = 0, 8 and 20 to fp64 rounding, p never exceeds 2^tau, and a larger
+    tau moves the max less often on scores that grow along the key axis."""
+    rng = np.random.default_rng(21)
+    n, d = 160, 8
+    q, k, v = (rng.standard_normal((n, d)) for _ in range(3))
+    q[:, 0] = np.abs(q[:, 0]) + 1.0
+    k[:, 0] += np.linspace(0.0, 12.0, n)          # scores grow with the key index
+    sizes = [16] * 10
+    for causal in (False, True):
+        o_ref, l_ref = oracle.attn_fwd_ref(q[None, None], k[None, None], v[None, None], 0.9, causal)
+        moves = {}
+        for tau in (0.0, 8.0, 20.0):
+            st = {}
+            o, lse = oracle.attn_fwd_online_ref(q, k, v, 0.9, causal, sizes, tau_log2=tau, stats=st)
+            np.testing.assert_allclose(o, o_ref[0, 0], rtol=1e-11, atol=1e-12)
+            np.testing.assert_allclose(lse, l_ref[0, 0], rtol=1e-12, atol=1e-12)
+            assert st["p_max"] <= 2.0 ** tau * (1 + 1e-12)
+            moves[tau] = st["rescales"]
+        assert moves[8.0] < moves[0.0] and moves[20.0] <= moves[8.0]
+        assert moves[20.0] >= n                   # every row sets its max at least once
+
+
 def test_accepts_bf16_torch_exactly():
     g = torch.Generator().manual_seed(0)
     q, k, v = (torch.randn(1, 1, 5, 4, generator=g).to(torch.bfloat16) for _ in range(3))
