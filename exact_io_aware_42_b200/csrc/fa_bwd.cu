@@ -64,8 +64,12 @@ struct BwdCfg {
   static constexpr int kOffDO = kOffQ + kStagesQ * kTileBytes;        // + s * kTileBytes
   static constexpr int kOffDS = kOffDO + kStagesD * kTileBytes;       // dS^T, 128 x 128 bf16 (dQ only)
   static constexpr int kOffL = kOffDS + (DQ ? 128 * 128 * 2 : 0);     // + s * 512: L log2 e [128], Q ring
-  static constexpr int kOffDl = kOffL + kStagesQ * 512;               // + s * 512: D [128], dO ring
-  static constexpr int kOffBar = kOffDl + kStagesD * 512;
+  // D_i is staged beside Q_i with dQ (the dO slot is then released as soon
+  // as dV has read dO), beside dO_i without dQ (no room for a third D slot)
+  static constexpr bool kDWithQ = DQ;
+  static constexpr int kDSlots = kDWithQ ? kStagesQ : kStagesD;
+  static constexpr int kOffDl = kOffL + kStagesQ * 512;               // + s * 512: D [128]
+  static constexpr int kOffBar = kOffDl + kDSlots * 512;
   static constexpr int kNumBars = 1 + 2 * kStagesQ + 2 * kStagesD + 10;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
@@ -280,26 +284,37 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
         tma_load_3d(vAddr + pn * C::kPanelBytes, &p.tm_v, bar(B_KV), pn * 64, j * 128, kvh);
       }
     }
-    // Per query block: L_i (log2 units, +inf past N) beside Q_i, D_i (0 past
-    // N) beside dO_i; each is written by the warp before the arrive that
-    // publishes its slot.
-    auto stage_rows = [&](float* dst, const float* src, int qh, int i, float mul, float pad) {
-      float v4[4];
+    // Per query block: L_i (log2 units, +inf past N) and D_i (0 past N) beside
+    // Q_i (the Q slot is held until dK, after the dS phase has read them; the
+    // dO slot is released as soon as dV has read dO); both are written by
+    // the warp before the arrive that publishes the slot.  The values of the next block are loaded into
+    // registers right after this block's copies are issued, so the load
+    // latency runs while the warp waits for the next free slots instead of
+    // delaying the next copies.
+    auto fetch_rows = [&](int idx, float4& l4, float4& d4) {
+      const int i = q_block(idx), qh = q_head(idx);
+      float lv[4], dv[4];
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         const int q = i * 128 + lane * 4 + t;
-        v4[t] = q < p.N ? src[static_cast<size_t>(qh) * p.N + q] * mul : pad;
+        const size_t g = static_cast<size_t>(qh) * p.N + q;
+        lv[t] = q < p.N ? p.lse[g] * 1.4426950408889634f : INFINITY;
+        dv[t] = q < p.N ? p.delta[g] : 0.f;
       }
-      reinterpret_cast<float4*>(dst)[lane] = make_float4(v4[0], v4[1], v4[2], v4[3]);
-      __syncwarp();
+      l4 = make_float4(lv[0], lv[1], lv[2], lv[3]);
+      d4 = make_float4(dv[0], dv[1], dv[2], dv[3]);
     };
+    float4 l_next = make_float4(0.f, 0.f, 0.f, 0.f), d_next = l_next;
+    if (n_it > 0) fetch_rows(0, l_next, d_next);
     for (int idx = 0; idx < n_it && ok; ++idx) {
       const int i = q_block(idx), qh = q_head(idx);
       const int sq = idx % NQ, sd = idx % ND;
       bool w = true;
       if (lane == 0) w = mbar_wait(bar(B_QE(sq)), ((idx / NQ) & 1) ^ 1, ab, kSiteBProd);
       if (!(ok = __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0)) break;
-      stage_rows(reinterpret_cast<float*>(smem + C::kOffL + sq * 512), p.lse, qh, i, 1.4426950408889634f, INFINITY);
+      reinterpret_cast<float4*>(smem + C::kOffL + sq * 512)[lane] = l_next;
+      if constexpr (C::kDWithQ) reinterpret_cast<float4*>(smem + C::kOffDl + sq * 512)[lane] = d_next;
+      __syncwarp();
       if (lane == 0) {
         mbar_arrive_expect_tx(bar(B_QF(sq)), C::kTileBytes);
         for (int pn = 0; pn < C::kPanels; ++pn)
@@ -308,13 +323,17 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
         w = mbar_wait(bar(B_DE(sd)), ((idx / ND) & 1) ^ 1, ab, kSiteBProd);
       }
       if (!(ok = __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0)) break;
-      stage_rows(reinterpret_cast<float*>(smem + C::kOffDl + sd * 512), p.delta, qh, i, 1.f, 0.f);
+      if constexpr (!C::kDWithQ) {
+        reinterpret_cast<float4*>(smem + C::kOffDl + sd * 512)[lane] = d_next;
+        __syncwarp();
+      }
       if (lane == 0) {
         mbar_arrive_expect_tx(bar(B_DF(sd)), C::kTileBytes);
         for (int pn = 0; pn < C::kPanels; ++pn)
           tma_load_3d(doAddr(sd) + pn * C::kPanelBytes, &p.tm_do, bar(B_DF(sd)), pn * 64, i * 128, qh);
         ++issued_d;
       }
+      if (idx + 1 < n_it) fetch_rows(idx + 1, l_next, d_next);
     }
     if (lane == 0 && *abort_flag) {   // let the copies in flight land before the CTA leaves
       volatile int never = 0;
@@ -365,6 +384,7 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
         if (!(ok = mbar_wait(bar(B_P), idx & 1, ab, kSiteBMmaP))) break;
         tc_fence_after();
         gemm_ts(C::kColDV, C::kColA, doAddr(sd), idx > 0);       // dV += P^T dO
+        if constexpr (C::kDWithQ) tc_commit(bar(B_DE(sd)));   // dP^T and dV, dO_i's readers, are done
         // S^T of the next block goes to region A right behind dV, which is
         // the last reader of P^T there (the dS phase keeps its own copy of P
         // in registers), so the next P phase overlaps dK and dP.
@@ -391,9 +411,10 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
         // Without dQ, region B takes dP^T of the next block after this dK in
         // issue order, and its completion (B_DP) implies dK has read dS^T.
         // dK is the last reader of Q_i, and it follows the dS phase, the last
-        // reader of L_i and D_i: both slots are free once it completes.
+        // reader of L_i and D_i: the Q slot (and without dQ the dO slot, which
+        // holds D_i) is free once it completes.
         tc_commit(bar(B_QE(sq)));
-        tc_commit(bar(B_DE(sd)));
+        if constexpr (!C::kDWithQ) tc_commit(bar(B_DE(sd)));
       }
       tc_commit(bar(B_FINAL));
       tc_commit(bar(B_DRAIN));
@@ -419,7 +440,7 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
     for (int idx = 0; idx < n_it && ok; ++idx) {
       const int i = q_block(idx);
       const float4* L4 = reinterpret_cast<const float4*>(smem + C::kOffL + (idx % NQ) * 512) + 16 * wg;
-      const float4* D4 = reinterpret_cast<const float4*>(smem + C::kOffDl + (idx % ND) * 512) + 16 * wg;
+      const float4* D4 = reinterpret_cast<const float4*>(smem + C::kOffDl + (idx % (C::kDWithQ ? NQ : ND)) * 512) + 16 * wg;
       // Visible query columns of this thread's key: c_lo <= column <= c_hi
       // (column c is query i * 128 + c): after the key on the diagonal block,
       // within the sliding window, and none at all for a key past N.
