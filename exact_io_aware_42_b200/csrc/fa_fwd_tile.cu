@@ -119,7 +119,9 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
 // NPOLY of every 8 column pairs take the polynomial exp2 (degree DEG), the
 // rest the SFU.  FP8: Q, K, V are E4M3 with per-128-row block scales and both
 // products run as kind::f8f6f4 (see the FP8 notes at the softmax).
-template <int D, bool CAUSAL, int NPOLY, int DEG, bool FP8>
+// ALIBI: the bias of p.alibi (a separate build, so that the plain kernel
+// carries none of its code).
+template <int D, bool CAUSAL, int NPOLY, int DEG, bool FP8, bool ALIBI>
 __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(const __grid_constant__ FwdParams p) {
   using C = TileCfg<D, FP8>;
   constexpr int NS = C::kStages;
@@ -399,15 +401,38 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(const __grid_constant_
       }
       // ALiBi sends every block through this path: the bias is added to the
       // scaled scores before the row maximum is taken.
-      const bool masked = (CAUSAL && (jb == qi || jb * kBlockN < qi * kBlockM + kBlockM - 1 - p.window)) ||
-                          ((jb + 1) * kBlockN > p.N) || p.alibi != nullptr;
-      if (masked) {
+      // edge: the diagonal tile, the window's edge, the key tail (and with
+      // ALiBi the diagonal tile, where keys lie on both sides of a row)
+      const bool edge = (CAUSAL && (jb == qi || jb * kBlockN < qi * kBlockM + kBlockM - 1 - p.window)) ||
+                        ((jb + 1) * kBlockN > p.N) || (ALIBI && jb == qi);
+      // ALiBi off the diagonal tile: every key lies on the same side of every
+      // row, so the bias -slope |key - row| is linear in the column
+      const bool alibi_lin = ALIBI && !edge;
+      const bool masked = edge || alibi_lin;   // u holds scaled (biased) scores
+      if (alibi_lin) {
+        const float sl2 = p.alibi[bh % p.H] * 1.4426950408889634f;
+        const int key0 = jb * kBlockN;
+        const float b0 = -sl2 * fabsf(static_cast<float>(key0 - row));
+        const float bs = jb < qi ? sl2 : -sl2;
+        const uint64_t c2 = f2_pack(c, c), bs2 = f2_pack(bs, bs), b02 = f2_pack(b0, b0);
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const uint64_t bias2 =
+              f2_fma(bs2, f2_pack(static_cast<float>(2 * i), static_cast<float>(2 * i + 1)), b02);
+          const uint64_t r2 = f2_fma(f2_pack(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1])), c2, bias2);
+          float r0, r1;
+          f2_unpack(r2, r0, r1);
+          u[2 * i] = __float_as_uint(r0);
+          u[2 * i + 1] = __float_as_uint(r1);
+        }
+      }
+      if (edge) {
         // scaled scores with -inf where the key is hidden or past N: column i
         // is visible iff lo <= i < hi
         const int key0 = jb * kBlockN;
         const int hi = (CAUSAL ? min(row + 1, p.N) : p.N) - key0;
         const int lo = CAUSAL ? row - p.window - key0 : 0;
-        if (p.alibi != nullptr) {   // + this query head's slope log2(e) * -|key - row|
+        if constexpr (ALIBI) {   // + this query head's slope log2(e) * -|key - row|
           const float sl2 = p.alibi[bh % p.H] * 1.4426950408889634f;
           const float dk = static_cast<float>(key0 - row);
 #pragma unroll
@@ -469,7 +494,18 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(const __grid_constant_
         }
         tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
       } else {
-        if (masked) {
+        if (ALIBI && masked) {   // scores already scaled: p = 2^(u - m)
+          const uint64_t nm2 = f2_pack(neg_m, neg_m);
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const uint64_t p2 =
+                exp2_sfu_f2(f2_add(f2_pack(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1])), nm2));
+            acc[i & 3] = f2_add(acc[i & 3], p2);
+            float p0, p1;
+            f2_unpack(p2, p0, p1);
+            u[i] = pack_bf16x2(p0, p1);       // P overwrites the consumed scores
+          }
+        } else if (masked) {
 #pragma unroll
           for (int i = 0; i < 64; ++i) {
             const float p0 = ex2_sfu(__uint_as_float(u[2 * i]) + neg_m);
@@ -571,11 +607,11 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(const __grid_constant_
   }
 }
 
-template <int D, bool CAUSAL, int NPOLY, int DEG, bool FP8>
+template <int D, bool CAUSAL, int NPOLY, int DEG, bool FP8, bool ALIBI = false>
 cudaError_t launch_impl(const FwdParams& p, cudaStream_t stream) {
   using C = TileCfg<D, FP8>;
-  auto kern = fwd_tile_kernel<D, CAUSAL, NPOLY, DEG, FP8>;
-  cudaError_t e = set_smem_once<fwd_tile_kernel<D, CAUSAL, NPOLY, DEG, FP8>>(C::kSmemBytes);
+  auto kern = fwd_tile_kernel<D, CAUSAL, NPOLY, DEG, FP8, ALIBI>;
+  cudaError_t e = set_smem_once<fwd_tile_kernel<D, CAUSAL, NPOLY, DEG, FP8, ALIBI>>(C::kSmemBytes);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(p.n_pairs) * static_cast<unsigned>(p.BH);
   kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(p);
@@ -585,6 +621,7 @@ cudaError_t launch_impl(const FwdParams& p, cudaStream_t stream) {
 // The exp2 split (pairs of 8 on the polynomial) and the polynomial's degree.
 template <int D, bool CAUSAL, bool FP8>
 cudaError_t launch_np(const FwdParams& p, cudaStream_t stream) {
+  if (p.alibi != nullptr) return launch_impl<D, CAUSAL, 0, 3, FP8, true>(p, stream);   // SFU-only exp2
   const bool deg4 = p.poly_deg == 4;
   switch (p.poly_pairs) {
     case 0: return launch_impl<D, CAUSAL, 0, 3, FP8>(p, stream);
