@@ -83,6 +83,9 @@ struct TileCfg {
   static constexpr uint32_t kColP = 384;
   // P outside S: S_t(j+1) may start as soon as S_t(j) has been read out
   static constexpr bool kEarlyS = kSepP;
+  // bf16: the first copies go out before the CTA-wide sync (the FP8 build
+  // measured slower that way)
+  static constexpr bool kEarlyLoads = !FP8;
 };
 static_assert(TileCfg<128, true>::kSmemBytes <= 232448, "fp8 forward shared memory");
 static_assert(TileCfg<128, false>::kSmemBytes <= 232448, "bf16 forward shared memory");
@@ -166,7 +169,26 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(const __grid_constant_
   for (int t = 0; t < 2; ++t) n_t[t] = (CAUSAL ? min(qt0 + t + 1, p.n_kv) : p.n_kv) - j_start;
   const int n_iter = n_t[1];
 
-  if (threadIdx.x == 0) {
+  // The producer thread initialises the barriers and starts the copies of
+  // Q_0, K(0), Q_1 and the rest of the first ring round before the CTA-wide
+  // sync, so that their latency overlaps the TMEM allocation and the sync
+  // (no other thread touches a barrier before the sync).
+  auto load_kv = [&](int sq) {   // ring copy number sq: K(sq / 2) or V(sq / 2)
+    const int s = sq % NS;
+    mbar_arrive_expect_tx(bar(bar_full<NS>(s)), C::kTileBytes);
+    const CUtensorMap* m = (sq & 1) ? &p.tm_v : &p.tm_k;
+    for (int pn = 0; pn < C::kPanels; ++pn)
+      tma_load_3d(sbase + C::kOffRing + s * C::kTileBytes + pn * C::kPanelBytes, m, bar(bar_full<NS>(s)),
+                  pn * C::kPanelElems, (j_start + sq / 2) * kBlockN, kvh);
+  };
+  auto load_q = [&](int t) {
+    mbar_arrive_expect_tx(bar(bar_q(t)), C::kTileBytes);
+    for (int pn = 0; pn < C::kPanels; ++pn)
+      tma_load_3d(sbase + C::kOffQ + t * C::kTileBytes + pn * C::kPanelBytes, &p.tm_q, bar(bar_q(t)),
+                  pn * C::kPanelElems, (qt0 + t) * kBlockM, bh);
+  };
+  const int n_first = C::kEarlyLoads ? min(NS, 2 * n_iter) : 0;   // ring copies that need no free slot
+  if (warp == 8 && lane == 0) {
     mbar_init(bar(bar_q(0)), 1);
     mbar_init(bar(bar_q(1)), 1);
     for (int s = 0; s < NS; ++s) {
@@ -182,6 +204,15 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(const __grid_constant_
     mbar_init(bar(bar_drain<NS>()), 1);
     *abort_flag = 0;
     fence_mbar_init();
+    if constexpr (C::kEarlyLoads) {
+      tma_prefetch_desc(&p.tm_q);
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
+      load_q(0);
+      load_kv(0);
+      load_q(1);
+      for (int sq = 1; sq < n_first; ++sq) load_kv(sq);
+    }
   }
   if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
@@ -196,29 +227,17 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(const __grid_constant_
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      tma_prefetch_desc(&p.tm_q);
-      tma_prefetch_desc(&p.tm_k);
-      tma_prefetch_desc(&p.tm_v);
-      for (int t = 0; t < 2; ++t) {
-        mbar_arrive_expect_tx(bar(bar_q(t)), C::kTileBytes);
-        for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_3d(sbase + C::kOffQ + t * C::kTileBytes + pn * C::kPanelBytes, &p.tm_q,
-                      bar(bar_q(t)), pn * C::kPanelElems, (qt0 + t) * kBlockM, bh);
+      if constexpr (!C::kEarlyLoads) {
+        tma_prefetch_desc(&p.tm_q);
+        tma_prefetch_desc(&p.tm_k);
+        tma_prefetch_desc(&p.tm_v);
+        load_q(0);
+        load_q(1);
       }
-      int seq = 0;
-      bool ok = true;
-      for (int j = 0; j < n_iter && ok; ++j) {
-        for (int w = 0; w < 2 && ok; ++w) {
-          const int s = seq % NS;
-          const uint32_t ph = (seq / NS) & 1;
-          if (!mbar_wait(bar(bar_empty<NS>(s)), ph ^ 1, ab, kSiteProdEmpty)) { ok = false; break; }
-          mbar_arrive_expect_tx(bar(bar_full<NS>(s)), C::kTileBytes);
-          const CUtensorMap* m = (w == 0) ? &p.tm_k : &p.tm_v;
-          for (int pn = 0; pn < C::kPanels; ++pn)
-            tma_load_3d(sbase + C::kOffRing + s * C::kTileBytes + pn * C::kPanelBytes, m,
-                        bar(bar_full<NS>(s)), pn * C::kPanelElems, (j_start + j) * kBlockN, kvh);
-          ++seq;
-        }
+      int seq = n_first;   // bf16: the first ring round went out before the sync
+      for (; seq < 2 * n_iter; ++seq) {
+        if (!mbar_wait(bar(bar_empty<NS>(seq % NS)), ((seq / NS) & 1) ^ 1, ab, kSiteProdEmpty)) break;
+        load_kv(seq);
       }
       if (*abort_flag) {
         // Another role gave up: let every copy this thread started land before
@@ -271,13 +290,17 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(const __grid_constant_
         }
         tc_commit(bar(bar_pv<NS>(t)));
       };
-      bool ok = mbar_wait(bar(bar_q(0)), 0, ab, kSiteMmaQ) && mbar_wait(bar(bar_q(1)), 0, ab, kSiteMmaQ);
+      // S_0(0) as soon as Q_0 and K(0) are in, S_1(0) once Q_1 is
+      bool ok = mbar_wait(bar(bar_q(0)), 0, ab, kSiteMmaQ) && mbar_wait(bar(bar_full<NS>(0)), 0, ab, kSiteMmaFull);
       int seq = 0;
       int ks = 0;
-      if (ok) ok = mbar_wait(bar(bar_full<NS>(0)), 0, ab, kSiteMmaFull);
       if (ok) {
         tc_fence_after();
         issue_s(0, ring(0));
+        ok = mbar_wait(bar(bar_q(1)), 0, ab, kSiteMmaQ);
+      }
+      if (ok) {
+        tc_fence_after();
         issue_s(1, ring(0));
         tc_commit(bar(bar_empty<NS>(0)));
         seq = 1;
@@ -593,7 +616,7 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(const __grid_constant_
         for (int pn = 0; pn < D / 64; ++pn)
           tma_store_3d(&p.tm_o, o_stage + pn * C::kPanelBytes, pn * 64, qi * kBlockM, bh);   // bf16 O
         tma_store_commit();
-        tma_store_wait_all();
+        tma_store_wait_read_all();   // the stores complete after the CTA has exited
       }
       if (row < p.N) p.lse[static_cast<size_t>(bh) * p.N + row] = (m_use + log2f(l)) * 0.69314718055994531f;
     }
