@@ -130,7 +130,6 @@ def measured_peaks():
 
 
 KERNEL_SOURCES = {
-    "fwd": ("fa_fwd.cu",),
     "fwd_tile": ("fa_fwd_tile.cu",),
     "fwd_q1": ("fa_fwd_q1.cu",),
     "fwd256": ("fa_fwd_d256.cu",),
@@ -437,7 +436,7 @@ def config_block(graph: bool):
             "fp8_loop": ("quant_fp8 (Q, K rotated; V) + fwd_fp8 in a second loop of K steps, key fp8"
                          if w["d"] == 128 else "none (the FP8 forward is built for d = 128)"),
             "bwd_pair": TUNING.get("bwd_pair"),
-            "fwd_split_pv": TUNING.get("fwd_split_pv"), "fwd_persistent": TUNING.get("fwd_persistent"),
+            "fwd_persistent": TUNING.get("fwd_persistent"),
             "fwd_causal_group": TUNING.get("fwd_causal_group"), "fwd_q1": TUNING.get("fwd_q1"),
             "exp2_split": {"fwd_poly_pairs": TUNING.get("fwd_poly_pairs"),
                            "fwd_poly_degree": TUNING.get("fwd_poly_degree"),
@@ -473,11 +472,11 @@ def run_ours(args):
         fa.set_tuning("fp8_poly_pairs", args.fp8_poly_pairs)
     if args.bwd_pair is not None:
         fa.set_tuning("bwd_pair", args.bwd_pair)
-    for knob in ("fwd_split_pv", "fwd_persistent", "fwd_causal_group", "fwd_q1"):
+    for knob in ("fwd_persistent", "fwd_causal_group", "fwd_q1"):
         if getattr(args, knob) is not None:
             fa.set_tuning(knob, getattr(args, knob))
     TUNING.update({k_: fa.get_tuning(k_, d) for k_ in ("fwd_poly_pairs", "fwd_poly_degree", "fp8_poly_pairs",
-                                                       "bwd_pair", "fwd_split_pv", "fwd_persistent",
+                                                       "bwd_pair", "fwd_persistent",
                                                        "fwd_causal_group", "fwd_q1")})
     graph = {"auto": latency_bound(w), "on": True, "off": False}[args.graph]
     hq, hk, hv, hdo = inputs.make_gqa(B, H, H_kv, N, d, w["seed"] + rank, with_do=True)
@@ -575,14 +574,20 @@ def run_ours(args):
                         profiled_traffic("bwd_main_kernel", w["name"], "bwd") if BWD_MODE == "atomic" else None)
         roof_bwd["frac_sustained"] = roof_bwd["achieved"] / sustained
         roof_bwd["frac_nominal_2250"] = roof_bwd["achieved"] / 2250.0
-    pers = TUNING.get("fwd_persistent") == 1
+    # the two-tile forward's grid: set explicitly, or (-1) the library's
+    # per-call default: persistent for bf16 non-causal and FP8 causal, one CTA
+    # per item with ALiBi or a polynomial exp2 share
+    pk = TUNING.get("fwd_persistent")
+    plain = not w["alibi"]
+    pers = plain and TUNING.get("fwd_poly_pairs") == 0 and (pk == 1 or (pk == -1 and not causal))
+    pers8 = plain and TUNING.get("fp8_poly_pairs") == 0 and (pk == 1 or (pk == -1 and causal))
     # the one-tile kernel: chosen explicitly, or by the library when the
     # two-tile kernel would have fewer work items than SMs
     n_pairs = ((N + 127) // 128 + 1) // 2
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     q1 = d != 256 and (TUNING.get("fwd_q1") == 1 or (TUNING.get("fwd_q1") == -1 and n_pairs * B * H < sms))
     fwd_name, fwd_src = (("fwd256_kernel", "fwd256") if d == 256 else ("fwd_q1_kernel", "fwd_q1") if q1
-                         else ("fwd_kernel", "fwd") if pers else ("fwd_tile_kernel", "fwd_tile"))
+                         else ("fwd_tile_kernel", "fwd_tile"))
     fwd_desc = f"{fwd_name}<{d}, {cz}, bf16>" + (
         " (persistent, one query tile per item)" if q1 else " (persistent)" if d == 256 or pers
         else " (one CTA per item)")
@@ -612,8 +617,8 @@ def run_ours(args):
     if fp8_stages:
         fp8_peak = 2.0 * burst
         fp8_flops = sum(s[2] for s in fp8_stages)
-        fp8_name = "fwd_kernel" if pers else "fwd_tile_kernel"
-        rf = roof(fp8_stages, fp8_per_stage, "fwd_fp8", f"{fp8_name}<128, {cz}, e4m3>", None, fp8_peak,
+        rf = roof(fp8_stages, fp8_per_stage, "fwd_fp8",
+                  f"fwd_tile_kernel<128, {cz}, e4m3> ({'persistent' if pers8 else 'one CTA per item'})", None, fp8_peak,
                   f"2 x {peak_src} bf16_tflops burst (nominal 2:1 ratio of dense E4M3 to bf16; no measured "
                   "FP8 peak)", None)
         rf["algorithmic_bytes"] = fwd_bytes(B, H, N, d, H_kv) - (B * H + 2 * B * H_kv) * N * d
@@ -655,8 +660,8 @@ def main():
     ap.add_argument("--fwd-poly-degree", type=int, choices=[3, 4], default=None)
     ap.add_argument("--bwd-pair", type=int, choices=[0, 1], default=None,
                     help="deterministic backward at d = 128: dK, dV on CTA pairs (1) or single CTAs (0)")
-    ap.add_argument("--fwd-split-pv", type=int, choices=[0, 1], default=None)
-    ap.add_argument("--fwd-persistent", type=int, choices=[0, 1], default=None)
+    ap.add_argument("--fwd-persistent", type=int, choices=[0, 1], default=None,
+                    help="two-tile forward: persistent grid (1) or one CTA per work item (0)")
     ap.add_argument("--fwd-q1", type=int, choices=[0, 1], default=None,
                     help="bf16 forward, d <= 128: one query tile per item with two score buffers (1)")
     ap.add_argument("--fwd-causal-group", type=int, choices=[0, 1], default=None,

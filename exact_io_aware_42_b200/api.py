@@ -20,7 +20,7 @@ import torch
 
 from ._lib import (TUNE_BWD_PAIR, TUNE_BWD_POLY_GROUPS, TUNE_DQ_POLY_PAIRS, TUNE_FP8_POLY_PAIRS,
                    TUNE_FWD_CAUSAL_GROUP, TUNE_FWD_PERSISTENT, TUNE_FWD_Q1, TUNE_FWD_POLY_DEGREE, TUNE_FWD_POLY_PAIRS,
-                   TUNE_FWD_SPLIT_PV, check, lib)
+                   check, lib)
 
 __all__ = ["fwd", "bwd", "bwd_workspace_size", "bwd_noalloc", "quant_fp8", "fwd_fp8", "get_status",
            "clear_status", "n_blocks", "set_tuning", "get_tuning", "TUNING_KNOBS"]
@@ -231,7 +231,7 @@ def bwd_noalloc(q, k, v, o, do, lse, causal: bool = False, scale: Optional[float
 TUNING_KNOBS = {"fwd_poly_pairs": TUNE_FWD_POLY_PAIRS, "fwd_poly_degree": TUNE_FWD_POLY_DEGREE,
                 "bwd_poly_groups": TUNE_BWD_POLY_GROUPS, "dq_poly_pairs": TUNE_DQ_POLY_PAIRS,
                 "fp8_poly_pairs": TUNE_FP8_POLY_PAIRS, "bwd_pair": TUNE_BWD_PAIR,
-                "fwd_split_pv": TUNE_FWD_SPLIT_PV, "fwd_persistent": TUNE_FWD_PERSISTENT,
+                "fwd_persistent": TUNE_FWD_PERSISTENT,
                 "fwd_causal_group": TUNE_FWD_CAUSAL_GROUP, "fwd_q1": TUNE_FWD_Q1}
 
 

@@ -118,15 +118,14 @@ int bwd_poly_groups() {
   return v >= 0 ? v : kDefaultBwdPolyGroups;
 }
 
-int fwd_split_pv() {
-  const int v = tune_raw(FA_TUNE_FWD_SPLIT_PV);
-  return v >= 0 ? v : kDefaultFwdSplitPv;
-}
-
-int fwd_persistent(int d, bool fp8) {
+// The two-tile forward's grid; the persistent mode is built for the SFU-only
+// exp2 without ALiBi (the exp2 split is a measurement control).
+int fwd_persistent(bool fp8, bool causal, int poly, const float* alibi) {
+  if (poly != 0 || alibi != nullptr) return 0;
   const int v = tune_raw(FA_TUNE_FWD_PERSISTENT);
   if (v >= 0) return v;
-  return fp8 ? kDefaultFwdPersistentFp8 : d == 64 ? kDefaultFwdPersistentD64 : kDefaultFwdPersistentD128;
+  if (fp8) return causal ? kDefaultFwdPersistentFp8Causal : kDefaultFwdPersistentFp8NonCausal;
+  return causal ? kDefaultFwdPersistentCausal : kDefaultFwdPersistentNonCausal;
 }
 
 // The one-tile forward kernel: set explicitly, or (default) when the
@@ -301,8 +300,7 @@ extern "C" fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void
     return FA_ERR_INVALID_ARG;
   p.o = static_cast<uint16_t*>(o);
   p.sms = di->sms;
-  p.split_pv = fwd_split_pv();
-  p.persistent = d == 256 ? 1 : fwd_persistent(d, false);
+  p.persistent = d == 256 ? 1 : fwd_persistent(false, causal != 0, poly_pairs(d), alibi_slopes);
   p.group_heads = fwd_group_heads(B * H, H / H_kv, N, d, 2);
   if (!p.persistent && !encode_3d(&p.tm_o, o, bf, 2, d, N, BH, 64, kBlockM)) return FA_ERR_INVALID_ARG;
   p.lse = lse;
@@ -325,8 +323,7 @@ extern "C" fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void
   if (q1 && static_cast<long long>(p.n_kv) * BH > kMaxWorkItems) return FA_ERR_UNSUPPORTED;
   cudaError_t e = d == 256 ? launch_fwd_d256(p, causal != 0, static_cast<cudaStream_t>(stream))
                   : q1 ? launch_fwd_q1_bf16(p, d, causal != 0, static_cast<cudaStream_t>(stream))
-                  : p.persistent ? launch_fwd_bf16(p, d, causal != 0, static_cast<cudaStream_t>(stream))
-                                 : launch_fwd_tile_bf16(p, d, causal != 0, static_cast<cudaStream_t>(stream));
+                  : launch_fwd_tile_bf16(p, d, causal != 0, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     cudaGetLastError();
     return FA_ERR_LAUNCH;
@@ -560,8 +557,7 @@ extern "C" fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v
     return FA_ERR_INVALID_ARG;
   p.o = static_cast<uint16_t*>(o);
   p.sms = di->sms;
-  p.split_pv = fwd_split_pv();
-  p.persistent = fwd_persistent(d, true);
+  p.persistent = fwd_persistent(true, causal != 0, fp8_poly_pairs(), alibi_slopes);
   p.group_heads = fwd_group_heads(B * H, H / H_kv, N, d, 1);
   if (!p.persistent &&
       !encode_3d(&p.tm_o, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, BH, 64, kBlockM))
@@ -584,8 +580,7 @@ extern "C" fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.poly_pairs = fp8_poly_pairs();
   p.poly_deg = poly_degree();
-  cudaError_t e = p.persistent ? launch_fwd_fp8(p, causal != 0, static_cast<cudaStream_t>(stream))
-                               : launch_fwd_tile_fp8(p, causal != 0, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_fwd_tile_fp8(p, causal != 0, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     cudaGetLastError();
     return FA_ERR_LAUNCH;
@@ -611,7 +606,6 @@ bool tuning_value_ok(int knob, int value) {
     case FA_TUNE_DQ_POLY_PAIRS: return value == 0 || value == 2 || value == 4;
     case FA_TUNE_FP8_POLY_PAIRS: return value == 0 || value == 2 || value == 4;
     case FA_TUNE_BWD_PAIR: return value == 0 || value == 1;
-    case FA_TUNE_FWD_SPLIT_PV: return value == 0 || value == 1;
     case FA_TUNE_FWD_PERSISTENT: return value == 0 || value == 1;
     case FA_TUNE_FWD_CAUSAL_GROUP: return value == 0 || value == 1;
     case FA_TUNE_FWD_Q1: return value == 0 || value == 1;
@@ -635,8 +629,7 @@ extern "C" int fa_get_tuning(int knob, int d) {
     case FA_TUNE_DQ_POLY_PAIRS: return d == 64 ? dq_poly_pairs() : 0;
     case FA_TUNE_FP8_POLY_PAIRS: return fp8_poly_pairs();
     case FA_TUNE_BWD_PAIR: return d == 128 ? bwd_pair() : 0;
-    case FA_TUNE_FWD_SPLIT_PV: return fwd_split_pv();
-    case FA_TUNE_FWD_PERSISTENT: return d == 256 ? 1 : fwd_persistent(d, false);
+    case FA_TUNE_FWD_PERSISTENT: return d == 256 ? 1 : tune_raw(FA_TUNE_FWD_PERSISTENT);   // -1: chosen per call
     case FA_TUNE_FWD_CAUSAL_GROUP: return fwd_causal_group();
     case FA_TUNE_FWD_Q1: return d == 256 ? 0 : tune_raw(FA_TUNE_FWD_Q1);   // -1: chosen per call
     default: return -1;

@@ -1,6 +1,6 @@
 // Fused exact attention forward for head dim 256 on sm_100a (bf16 in, fp32
 // accumulate).  Computes the same O and logsumexp L as the d <= 128 kernel
-// (fa_fwd.cu) by the same online softmax ("FlashAttention v1/v2/v3/v4: the
+// (fa_fwd_tile.cu) by the same online softmax ("FlashAttention v1/v2/v3/v4: the
 // librarian who never clears the desk", online softmax section, eq. 2;
 // deferred normalisation, lineage page "FA2 (2023)", refinement 2); the
 // librarian page lists d = 256 among the head dims FlashAttention serves
@@ -30,7 +30,7 @@
 // tiles above the diagonal are never loaded; the diagonal block, key tails
 // past N, window edges and ALiBi take the masked path, as at d <= 128.
 // Conditional rescaling with the stale-max threshold kRescaleTau as in
-// fa_fwd.cu.  Every wait is bounded (fa_ptx.cuh).
+// fa_fwd_tile.cu.  Every wait is bounded (fa_ptx.cuh).
 #include <type_traits>
 
 #include "fa_exp2.cuh"

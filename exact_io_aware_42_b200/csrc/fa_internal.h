@@ -57,8 +57,7 @@ struct FwdParams {
   int poly_pairs;       // of every 8 column pairs, how many use the FMA-pipe exp2
   int poly_deg;         // degree of that polynomial (3 or 4)
   int sms;              // multiprocessor count: persistent grid size
-  int split_pv;         // d <= 128: 1: P V issued in two 64-key halves as P arrives; 0: after all of P
-  int persistent;       // 1: persistent kernel, min(items, SMs) CTAs; 0: one CTA per work item
+  int persistent;       // 1: persistent grid of min(items, SMs) CTAs; 0: one CTA per work item
   int group_heads;      // one-CTA-per-item kernel, causal: CTA order longest first within groups
                         // of this many heads (>= BH: one group over all heads)
 };
@@ -73,16 +72,18 @@ constexpr int kDefaultPolyPairsD128 = 0;
 constexpr int kDefaultPolyPairsD64 = 0;
 constexpr int kDefaultPolyPairsD256 = 0;
 constexpr int kDefaultPolyDegree = 4;
-// measured on B200 (cfg B4 H16 N4096 d128 causal: 903 vs 870 TFLOPS; N 16384: 1060 vs 1006)
-constexpr int kDefaultFwdSplitPv = 0;
-// d <= 128: which forward kernel runs by default, chosen by measurement on
-// B200 (same-process A/B): one CTA per work item was faster at d = 128
-// (bf16 B4 H16 N4096 causal 926-939 vs 901-913 TFLOPS; FP8 B2 H16 N8192
-// 1106-1126 vs 957) and at d = 64, where it also keeps P in TMEM columns of
-// its own (B4 H32 N4096 causal 574-579 vs 520).
-constexpr int kDefaultFwdPersistentD128 = 0;
-constexpr int kDefaultFwdPersistentD64 = 0;
-constexpr int kDefaultFwdPersistentFp8 = 0;
+// d <= 128: the two-tile forward's grid by default, chosen by measurement on
+// B200 (same-process A/B, TFLOPS, one CTA per item vs persistent): bf16
+// non-causal gains from the persistent grid (B4 H16 N4096 d128 1112 vs 1140,
+// d64 677 vs 682); bf16 causal loses (935 vs 923; B1 H16 N16384 1140 vs
+// 1104), where the hardware's in-order CTA hand-out is a dynamic
+// longest-first schedule and the persistent grid's static one is not; FP8
+// gains causal (B4 H16 N4096 837 vs 864) and loses non-causal (B2 H16 N8192
+// 1084 vs 1066).
+constexpr int kDefaultFwdPersistentCausal = 0;
+constexpr int kDefaultFwdPersistentNonCausal = 1;
+constexpr int kDefaultFwdPersistentFp8Causal = 1;
+constexpr int kDefaultFwdPersistentFp8NonCausal = 0;
 // Causal CTA order of the one-CTA-per-item kernel, measured (same-process
 // A/B): grouping heads helped only once K and V of all heads far exceed L2
 // (B8 H16 N4096 d128: 948 vs 910 TFLOPS) and cost about 1% at B4 H16 N4096
@@ -99,11 +100,10 @@ constexpr long long kCausalGroupBytes = 32ll << 20;
 // FP8 forward: share of the exp2 on the polynomial (pairs of 8)
 constexpr int kDefaultPolyPairsFp8 = 0;
 
-// Persistent kernel (d = 64, 128; FP8 d = 128): min(items, SMs) CTAs.
-cudaError_t launch_fwd_bf16(const FwdParams& p, int d, bool causal, cudaStream_t stream);
 // One 128-row query tile per work item, two score buffers, persistent grid (bf16, d = 64, 128).
 cudaError_t launch_fwd_q1_bf16(const FwdParams& p, int d, bool causal, cudaStream_t stream);
-// One CTA per work item (d = 64, 128; FP8 d = 128); needs tm_o.
+// Two query tiles per work item (d = 64, 128; FP8 d = 128): one CTA per item
+// (needs tm_o) or, with p.persistent (SFU-only exp2, no ALiBi), a persistent grid.
 cudaError_t launch_fwd_tile_bf16(const FwdParams& p, int d, bool causal, cudaStream_t stream);
 cudaError_t launch_fwd_tile_fp8(const FwdParams& p, bool causal, cudaStream_t stream);
 // Head dim 256 (one query tile per work item, K/V streamed as 64-column panels).
@@ -112,8 +112,6 @@ cudaError_t launch_fwd_d256(const FwdParams& p, bool causal, cudaStream_t stream
 cudaError_t launch_selftest_wait(unsigned int* status, cudaStream_t stream);
 // y[i] = 2^x[i] by the softmax's exp2 (degree 0: the SFU; 3, 4, 5: the polynomial).
 cudaError_t launch_selftest_exp2(const float* x, float* y, long long n, int degree, cudaStream_t stream);
-// E4M3 forward (d = 128): tm_q/tm_k/tm_v are uint8 maps, sq/sk/sv block scales.
-cudaError_t launch_fwd_fp8(const FwdParams& p, bool causal, cudaStream_t stream);
 // Block quantisation of one bf16 tensor to E4M3 (signs == nullptr: no rotation).
 struct QuantParams {
   CUtensorMap tm_x;     // bf16 [BH, N, 128], box {64, 128, 1}, 128-byte swizzle

@@ -257,11 +257,13 @@ fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v8, const fl
  *  FA_TUNE_BWD_PAIR         deterministic backward at d = 128: dK, dV from
  *                           CTA pairs sharing each product (1) or from single
  *                           CTAs (0); same results either way
- *  FA_TUNE_FWD_SPLIT_PV     forward, d <= 128: P V issued in two halves as P
- *                           arrives (1) or after all of P (0); the d = 256
- *                           kernel always splits
- *  FA_TUNE_FWD_PERSISTENT   forward: one CTA per SM walking the work items (1)
- *                           or one CTA per work item (0)
+ *  FA_TUNE_FWD_PERSISTENT   two-tile forward (d <= 128, bf16 and FP8): a
+ *                           persistent grid of one CTA per SM walking the work
+ *                           items (1) or one CTA per work item (0); by default
+ *                           chosen per call (persistent for bf16 non-causal and
+ *                           FP8 causal), which fa_get_tuning reports as -1; calls
+ *                           with ALiBi or a polynomial exp2 share use one CTA
+ *                           per item
  *  FA_TUNE_FWD_CAUSAL_GROUP causal forward, one CTA per work item: longest
  *                           first within groups of heads whose K and V fit in
  *                           L2 together (1), or over all heads (0)
@@ -282,7 +284,6 @@ typedef enum fa_tune_knob {
   FA_TUNE_DQ_POLY_PAIRS = 4,
   FA_TUNE_FP8_POLY_PAIRS = 5,
   FA_TUNE_BWD_PAIR = 6,
-  FA_TUNE_FWD_SPLIT_PV = 7,
   FA_TUNE_FWD_PERSISTENT = 8,
   FA_TUNE_FWD_CAUSAL_GROUP = 9,
   FA_TUNE_FWD_Q1 = 10,

@@ -23,9 +23,9 @@ def _fa():
     return fa
 
 
-def run_fwd(q, k, v, causal, scale=None):
+def run_fwd(q, k, v, causal, scale=None, window=None):
     fa = _fa()
-    o, lse = fa.fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, scale=scale)
+    o, lse = fa.fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, scale=scale, window=window)
     torch.cuda.synchronize()
     assert fa.get_status() == 0
     return o.cpu(), lse.cpu()
@@ -169,22 +169,20 @@ def test_fwd_exp2_split_variants(d, pairs, deg, causal, restore_tuning):
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("persistent,split,group,q1", [(0, 0, 1, 0), (0, 0, 0, 0), (1, 0, 0, 0), (1, 1, 0, 0),
-                                                      (0, 0, 0, 1)])
-def test_fwd_kernel_variants_every_head(d, persistent, split, group, q1, restore_tuning):
-    """Both forward kernels (one CTA per work item, with the grouped and the
-    global causal order; the persistent grid, with and without the split
-    P V) on a problem with more work items than SMs and, at d = 128, two head
-    groups (32 and 8 heads of N = 2048): every head matches the oracle on
-    sampled rows, causal and not, plus one whole head."""
+@pytest.mark.parametrize("persistent,group,q1", [(0, 1, 0), (0, 0, 0), (1, 0, 0), (0, 0, 1)])
+def test_fwd_kernel_variants_every_head(d, persistent, group, q1, restore_tuning):
+    """The forward kernels (two query tiles per item: one CTA per work item,
+    with the grouped and the global causal order, or the persistent grid; one
+    query tile per item) on a problem with more work items than SMs and, at
+    d = 128, two head groups (32 and 8 heads of N = 2048): every head matches
+    the oracle on sampled rows, causal and not, plus one whole head."""
     fa = _fa()
     fa.set_tuning("fwd_persistent", persistent)
-    fa.set_tuning("fwd_split_pv", split)
     fa.set_tuning("fwd_causal_group", group)
     fa.set_tuning("fwd_q1", q1)
     assert fa.get_tuning("fwd_persistent", d) == persistent and fa.get_tuning("fwd_q1", d) == q1
     N, H = 2048, 40
-    q, k, v = inputs.make_qkv(1, H, N, d, seed=700 + d + 8 * q1 + 4 * group + 2 * persistent + split)
+    q, k, v = inputs.make_qkv(1, H, N, d, seed=700 + d + 8 * q1 + 4 * group + 2 * persistent)
     # causal rows 0 and 1 average one or two keys, so |O| reaches a few units
     # and one bf16 half-ulp of O alone approaches 1e-2: O's elementwise bound
     # is taken relative to max(1, |O|) here (the masks tests' reading)
@@ -203,6 +201,26 @@ def test_fwd_kernel_variants_every_head(d, persistent, split, group, q1, restore
             assert max_scaled_err(o_k, o_r) <= O_MAX_ABS, tag
             assert rel_rms(o_k, o_r) <= O_REL_RMS, tag
             assert max_abs(l_k, l_r) <= LSE_MAX_ABS, tag
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("B,H,G,N,causal,window", [(2, 3, 1, 300, True, None), (2, 3, 1, 777, False, None),
+                                                   (1, 4, 1, 1000, True, 200), (2, 8, 4, 1536, True, None),
+                                                   (1, 2, 2, 2049, False, None), (3, 5, 1, 4100, True, None)])
+def test_fwd_persistent_grid_matches_one_cta_per_item(d, B, H, G, N, causal, window, restore_tuning):
+    """The two-tile forward's persistent grid runs the same arithmetic as one
+    CTA per work item, item by item: O and L agree bit for bit, over ragged
+    tails, GQA, a sliding window, and more work items than SMs."""
+    fa = _fa()
+    fa.set_tuning("fwd_q1", 0)
+    q, k, v = inputs.make_gqa(B, H, H // G, N, d, seed=900 + N + d)
+    out = {}
+    for mode in (0, 1):
+        fa.set_tuning("fwd_persistent", mode)
+        o, lse = run_fwd(q, k, v, causal, window=window)
+        out[mode] = (o.clone(), lse.clone())
+    assert torch.equal(out[0][0], out[1][0]) and torch.equal(out[0][1], out[1][1])
+    assert fa.get_status() == 0
 
 
 @pytest.mark.parametrize("causal", [False, True])
