@@ -575,11 +575,11 @@ def run_ours(args):
         roof_bwd["frac_sustained"] = roof_bwd["achieved"] / sustained
         roof_bwd["frac_nominal_2250"] = roof_bwd["achieved"] / 2250.0
     # the two-tile forward's grid: set explicitly, or (-1) the library's
-    # per-call default: persistent for bf16 non-causal and FP8 causal, one CTA
-    # per item with ALiBi or a polynomial exp2 share
+    # per-call default: persistent except for the FP8 non-causal forward, one
+    # CTA per item with ALiBi or a polynomial exp2 share
     pk = TUNING.get("fwd_persistent")
     plain = not w["alibi"]
-    pers = plain and TUNING.get("fwd_poly_pairs") == 0 and (pk == 1 or (pk == -1 and not causal))
+    pers = plain and TUNING.get("fwd_poly_pairs") == 0 and pk in (1, -1)
     pers8 = plain and TUNING.get("fp8_poly_pairs") == 0 and (pk == 1 or (pk == -1 and causal))
     # the one-tile kernel: chosen explicitly, or by the library when the
     # two-tile kernel would have fewer work items than SMs

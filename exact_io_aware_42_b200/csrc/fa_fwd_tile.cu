@@ -16,7 +16,9 @@
 // hands CTAs to SMs in index order as SMs free up, which with the items
 // ordered longest first is a dynamic longest-first schedule, and O leaves
 // through shared memory and a TMA store.  Persistent (PERS): min(items, SMs)
-// CTAs walk the items in snake order; one item's last products overlap the
+// CTAs walk the items (causal: a longest-processing-time-first deal made on
+// the host; otherwise, or for tables too large, rounds in snake order); one
+// item's last products overlap the
 // next item's Q and K/V copies (Q_t is reloaded as soon as the item's last
 // S_t product has read it) and its first S products, and O is written from
 // registers.  Roles:
@@ -51,12 +53,32 @@
 // Causal: key j visible to query i iff j <= i.  Tiles entirely above the
 // diagonal are never loaded or multiplied; only the diagonal tile and the
 // ragged key tail (keys >= N, zero-filled by TMA) are masked to -inf.
+#include <algorithm>
+#include <cstring>
+#include <numeric>
+#include <type_traits>
+#include <vector>
+
 #include "fa_exp2.cuh"
 #include "fa_internal.h"
 #include "fa_ptx.cuh"
 
 namespace fa {
 namespace {
+
+// Persistent causal grid: each CTA's work items, dealt by the host longest
+// processing time first (every item to the CTA with the least work so far,
+// items in order of decreasing cost), passed as a kernel parameter.  With
+// more items or CTAs than the table holds (n = 0) the kernel deals in snake
+// order instead.
+constexpr int kSchedMaxItems = 8192;
+constexpr int kSchedMaxCtas = 256;
+struct FwdSched {
+  int n;                                   // items in the table (0: none)
+  uint16_t off[kSchedMaxCtas + 1];         // CTA c: item[off[c] .. off[c + 1])
+  uint16_t item[kSchedMaxItems];
+};
+struct FwdSchedNone {};
 
 template <int D, bool FP8 = false>
 struct TileCfg {
@@ -130,11 +152,15 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
 // ALIBI: the bias of p.alibi (a separate build, so that the plain kernel
 // carries none of its code).
 // PERS: a persistent grid of at most one CTA per SM walks the work items
-// (snake order over the longest-first list), so that one item's end overlaps
-// the next item's copies and first products; O is then written from
-// registers (the Q buffer takes the next item's Q early).
+// (sch: the causal deal, see FwdSched), so that one item's end overlaps the
+// next item's copies and first products; O is then written from registers
+// (the Q buffer takes the next item's Q early).
 template <int D, bool CAUSAL, int NPOLY, int DEG, bool FP8, bool ALIBI, bool PERS = false>
-__global__ void __launch_bounds__(320, 1) fwd_tile_kernel(const __grid_constant__ FwdParams p) {
+using SchedFor = std::conditional_t<PERS && CAUSAL, FwdSched, FwdSchedNone>;
+
+template <int D, bool CAUSAL, int NPOLY, int DEG, bool FP8, bool ALIBI, bool PERS = false>
+__global__ void __launch_bounds__(320, 1) fwd_tile_kernel(
+    const __grid_constant__ FwdParams p, const __grid_constant__ SchedFor<D, CAUSAL, NPOLY, DEG, FP8, ALIBI, PERS> sch) {
   using C = TileCfg<D, FP8>;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -189,11 +215,20 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(const __grid_constant_
   auto my_item = [&](int k) -> int {
     if constexpr (PERS) {
       const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+      if constexpr (CAUSAL) {
+        if (sch.n > 0) {
+          const int i = sch.off[c] + k;
+          return i < sch.off[c + 1] ? static_cast<int>(sch.item[i]) : n_items;
+        }
+      }
       return k * G + ((k & 1) ? G - 1 - c : c);
     } else {
       return k == 0 ? static_cast<int>(blockIdx.x) : n_items;
     }
   };
+  // the first item (its copies start before the CTA-wide sync); the
+  // persistent bf16 build decodes every item afresh in the role loops, which
+  // keeps fewer values live across them
   const Item it0 = item_at(my_item(0));
 
   // The producer thread initialises the barriers and starts the copies of
@@ -270,7 +305,7 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(const __grid_constant_
       for (int k = 0; ok && (PERS || k == 0); ++k) {
         const int o = my_item(k);
         if (o >= n_items) break;
-        const Item it = k == 0 ? it0 : item_at(o);
+        const Item it = ((!PERS || FP8) && k == 0) ? it0 : item_at(o);
         const int seq0 = (k == 0) ? 0 : seq;   // this item's first ring copy
         // Q_t of this item once the previous item's last S_t has read the
         // buffer: Q_0, K(0), Q_1, then the rest of the item's K and V
@@ -356,7 +391,7 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(const __grid_constant_
       for (int k = 0; ok && (PERS || k == 0); ++k) {
         const int o = my_item(k);
         if (o >= n_items) break;
-        const Item it = k == 0 ? it0 : item_at(o);
+        const Item it = ((!PERS || FP8) && k == 0) ? it0 : item_at(o);
         const int n_t[2] = {it.n0, it.n1};
         const int n_iter = it.n1;
         // S_0(0) as soon as Q_0 and K(0) are in, S_1(0) once Q_1 is
@@ -455,7 +490,7 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(const __grid_constant_
     for (int k = 0; ok && (PERS || k == 0); ++k) {
       const int o = my_item(k);
       if (o >= n_items) break;
-      const Item it = k == 0 ? it0 : item_at(o);
+      const Item it = ((!PERS || FP8) && k == 0) ? it0 : item_at(o);
       const int bh = it.bh, kvh = it.kvh, j_start = it.j_start;
       const int qi = it.qt0 + t;
       const int row = qi * kBlockM + r;
@@ -738,6 +773,59 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(const __grid_constant_
   }
 }
 
+// The longest-processing-time-first deal of the causal items over G CTAs:
+// an item's cost is its number of key blocks per tile pair (2 n_1, the two
+// tiles' blocks plus the last single-tile block) plus one for its start; the
+// kernel's item order (item_at) and key-block counts are followed exactly.
+// Cached per thread for the last shape.
+const FwdSched* causal_schedule(const FwdParams& p, int G) {
+  struct Key {
+    int n_pairs, BH, group_heads, window, n_kv, G;
+    bool operator==(const Key& o) const {
+      return n_pairs == o.n_pairs && BH == o.BH && group_heads == o.group_heads && window == o.window &&
+             n_kv == o.n_kv && G == o.G;
+    }
+  };
+  thread_local Key key{-1, -1, -1, -1, -1, -1};
+  thread_local FwdSched sched;
+  const Key k{p.n_pairs, p.BH, p.group_heads, p.window, p.n_kv, G};
+  if (k == key) return &sched;
+  const long long items = static_cast<long long>(p.n_pairs) * p.BH;
+  sched.n = 0;
+  if (items <= kSchedMaxItems && G <= kSchedMaxCtas && G > 0) {
+    std::vector<int> cost(items);
+    for (int o = 0; o < items; ++o) {
+      const int per_group = p.group_heads * p.n_pairs;
+      const int g = o / per_group, rr = o - g * per_group;
+      const int gh = std::min(p.group_heads, p.BH - g * p.group_heads);
+      const int pair = p.n_pairs - 1 - rr / gh;
+      const int qt0 = 2 * pair;
+      const int j_start = std::max(0, qt0 * kBlockM - p.window) / kBlockN;
+      const int n1 = std::min(qt0 + 2, p.n_kv) - j_start;
+      cost[o] = 2 * n1 + 1;
+    }
+    std::vector<int> order(items);
+    std::iota(order.begin(), order.end(), 0);
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return cost[a] > cost[b]; });
+    std::vector<long long> load(G, 0);
+    std::vector<std::vector<int>> lists(G);
+    for (const int o : order) {
+      const int c = static_cast<int>(std::min_element(load.begin(), load.end()) - load.begin());
+      load[c] += cost[o];
+      lists[c].push_back(o);
+    }
+    int at = 0;
+    for (int c = 0; c < G; ++c) {
+      sched.off[c] = static_cast<uint16_t>(at);
+      for (const int o : lists[c]) sched.item[at++] = static_cast<uint16_t>(o);
+    }
+    sched.off[G] = static_cast<uint16_t>(at);
+    sched.n = at;
+  }
+  key = k;
+  return &sched;
+}
+
 template <int D, bool CAUSAL, int NPOLY, int DEG, bool FP8, bool ALIBI = false, bool PERS = false>
 cudaError_t launch_impl(const FwdParams& p, cudaStream_t stream) {
   using C = TileCfg<D, FP8>;
@@ -746,7 +834,11 @@ cudaError_t launch_impl(const FwdParams& p, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   const long long items = static_cast<long long>(p.n_pairs) * p.BH;
   const unsigned grid = static_cast<unsigned>((PERS && items > p.sms) ? p.sms : items);
-  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(p);
+  if constexpr (PERS && CAUSAL) {
+    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(p, *causal_schedule(p, static_cast<int>(grid)));
+  } else {
+    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(p, FwdSchedNone{});
+  }
   return cudaGetLastError();
 }
 

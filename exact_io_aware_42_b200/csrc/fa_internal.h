@@ -74,13 +74,12 @@ constexpr int kDefaultPolyPairsD256 = 0;
 constexpr int kDefaultPolyDegree = 4;
 // d <= 128: the two-tile forward's grid by default, chosen by measurement on
 // B200 (same-process A/B, TFLOPS, one CTA per item vs persistent): bf16
-// non-causal gains from the persistent grid (B4 H16 N4096 d128 1112 vs 1140,
-// d64 677 vs 682); bf16 causal loses (935 vs 923; B1 H16 N16384 1140 vs
-// 1104), where the hardware's in-order CTA hand-out is a dynamic
-// longest-first schedule and the persistent grid's static one is not; FP8
-// gains causal (B4 H16 N4096 837 vs 864) and loses non-causal (B2 H16 N8192
-// 1084 vs 1066).
-constexpr int kDefaultFwdPersistentCausal = 0;
+// gains from the persistent grid non-causal (B4 H16 N4096 d128 1112 vs
+// 1140, d64 677 vs 682) and, with its causal items dealt longest processing
+// time first, causal (B4 H16 N4096 d128 942 vs 962, N2048 693 vs 722, d64
+// 587 vs 603; N >= 8192 even); FP8 gains causal (B4 H16 N4096 850 vs 863)
+// and loses non-causal (B2 H16 N8192 1104 vs 1066).
+constexpr int kDefaultFwdPersistentCausal = 1;
 constexpr int kDefaultFwdPersistentNonCausal = 1;
 constexpr int kDefaultFwdPersistentFp8Causal = 1;
 constexpr int kDefaultFwdPersistentFp8NonCausal = 0;

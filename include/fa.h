@@ -260,8 +260,8 @@ fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v8, const fl
  *  FA_TUNE_FWD_PERSISTENT   two-tile forward (d <= 128, bf16 and FP8): a
  *                           persistent grid of one CTA per SM walking the work
  *                           items (1) or one CTA per work item (0); by default
- *                           chosen per call (persistent for bf16 non-causal and
- *                           FP8 causal), which fa_get_tuning reports as -1; calls
+ *                           chosen per call (persistent except for the FP8
+ *                           non-causal forward), which fa_get_tuning reports as -1; calls
  *                           with ALiBi or a polynomial exp2 share use one CTA
  *                           per item
  *  FA_TUNE_FWD_CAUSAL_GROUP causal forward, one CTA per work item: longest

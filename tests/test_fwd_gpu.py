@@ -223,6 +223,24 @@ def test_fwd_persistent_grid_matches_one_cta_per_item(d, B, H, G, N, causal, win
     assert fa.get_status() == 0
 
 
+def test_fwd_persistent_causal_beyond_the_deal_table(restore_tuning):
+    """A causal problem with more work items than the host-made deal holds
+    (9216 > 8192): the persistent grid falls back to rounds in snake order and
+    still matches one CTA per work item bit for bit."""
+    fa = _fa()
+    fa.set_tuning("fwd_q1", 0)
+    g = torch.Generator(device="cuda").manual_seed(77)
+    q, k, v = (torch.randn(9, 32, 8192, 64, device="cuda", generator=g).to(torch.bfloat16) for _ in range(3))
+    out = {}
+    for mode in (0, 1):
+        fa.set_tuning("fwd_persistent", mode)
+        o, lse = fa.fwd(q, k, v, causal=True)
+        torch.cuda.synchronize()
+        out[mode] = (o, lse)
+    assert torch.equal(out[0][0], out[1][0]) and torch.equal(out[0][1], out[1][1])
+    assert fa.get_status() == 0
+
+
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", [1, 7, 127, 128, 129, 255, 257, 383, 513, 1000])
 def test_fwd_d256_ragged(N, causal):
