@@ -438,6 +438,7 @@ def config_block(graph: bool):
             "bwd_pair": TUNING.get("bwd_pair"),
             "fwd_persistent": TUNING.get("fwd_persistent"),
             "fwd_causal_group": TUNING.get("fwd_causal_group"), "fwd_q1": TUNING.get("fwd_q1"),
+            "bwd_causal_group": TUNING.get("bwd_causal_group"),
             "exp2_split": {"fwd_poly_pairs": TUNING.get("fwd_poly_pairs"),
                            "fwd_poly_degree": TUNING.get("fwd_poly_degree"),
                            "fp8_poly_pairs": TUNING.get("fp8_poly_pairs")}}
@@ -472,11 +473,11 @@ def run_ours(args):
         fa.set_tuning("fp8_poly_pairs", args.fp8_poly_pairs)
     if args.bwd_pair is not None:
         fa.set_tuning("bwd_pair", args.bwd_pair)
-    for knob in ("fwd_persistent", "fwd_causal_group", "fwd_q1"):
+    for knob in ("fwd_persistent", "fwd_causal_group", "fwd_q1", "bwd_causal_group"):
         if getattr(args, knob) is not None:
             fa.set_tuning(knob, getattr(args, knob))
     TUNING.update({k_: fa.get_tuning(k_, d) for k_ in ("fwd_poly_pairs", "fwd_poly_degree", "fp8_poly_pairs",
-                                                       "bwd_pair", "fwd_persistent",
+                                                       "bwd_pair", "fwd_persistent", "bwd_causal_group",
                                                        "fwd_causal_group", "fwd_q1")})
     graph = {"auto": latency_bound(w), "on": True, "off": False}[args.graph]
     hq, hk, hv, hdo = inputs.make_gqa(B, H, H_kv, N, d, w["seed"] + rank, with_do=True)
@@ -664,6 +665,8 @@ def main():
                     help="two-tile forward: persistent grid (1) or one CTA per work item (0)")
     ap.add_argument("--fwd-q1", type=int, choices=[0, 1], default=None,
                     help="bf16 forward, d <= 128: one query tile per item with two score buffers (1)")
+    ap.add_argument("--bwd-causal-group", type=int, choices=[0, 1], default=None,
+                    help="causal backward: CTAs longest first within L2-sized head groups (1) or head by head (0)")
     ap.add_argument("--fwd-causal-group", type=int, choices=[0, 1], default=None,
                     help="causal forward: longest first within L2-sized head groups (1) or over all heads (0)")
     ap.add_argument("--fp8-poly-pairs", type=int, choices=[0, 2, 4], default=None,

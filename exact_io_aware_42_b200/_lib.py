@@ -54,7 +54,8 @@ STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_E
 
 # fa_tune_knob values (include/fa.h)
 (TUNE_FWD_POLY_PAIRS, TUNE_FWD_POLY_DEGREE, TUNE_BWD_POLY_GROUPS, TUNE_DQ_POLY_PAIRS, TUNE_FP8_POLY_PAIRS,
- TUNE_BWD_PAIR, TUNE_FWD_PERSISTENT, TUNE_FWD_CAUSAL_GROUP, TUNE_FWD_Q1) = 1, 2, 3, 4, 5, 6, 8, 9, 10
+ TUNE_BWD_PAIR, TUNE_FWD_PERSISTENT, TUNE_FWD_CAUSAL_GROUP, TUNE_FWD_Q1, TUNE_BWD_CAUSAL_GROUP) = \
+    1, 2, 3, 4, 5, 6, 8, 9, 10, 11
 
 
 class FaError(RuntimeError):

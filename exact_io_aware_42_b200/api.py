@@ -18,7 +18,7 @@ from typing import Optional
 
 import torch
 
-from ._lib import (TUNE_BWD_PAIR, TUNE_BWD_POLY_GROUPS, TUNE_DQ_POLY_PAIRS, TUNE_FP8_POLY_PAIRS,
+from ._lib import (TUNE_BWD_CAUSAL_GROUP, TUNE_BWD_PAIR, TUNE_BWD_POLY_GROUPS, TUNE_DQ_POLY_PAIRS, TUNE_FP8_POLY_PAIRS,
                    TUNE_FWD_CAUSAL_GROUP, TUNE_FWD_PERSISTENT, TUNE_FWD_Q1, TUNE_FWD_POLY_DEGREE, TUNE_FWD_POLY_PAIRS,
                    check, lib)
 
@@ -232,7 +232,8 @@ TUNING_KNOBS = {"fwd_poly_pairs": TUNE_FWD_POLY_PAIRS, "fwd_poly_degree": TUNE_F
                 "bwd_poly_groups": TUNE_BWD_POLY_GROUPS, "dq_poly_pairs": TUNE_DQ_POLY_PAIRS,
                 "fp8_poly_pairs": TUNE_FP8_POLY_PAIRS, "bwd_pair": TUNE_BWD_PAIR,
                 "fwd_persistent": TUNE_FWD_PERSISTENT,
-                "fwd_causal_group": TUNE_FWD_CAUSAL_GROUP, "fwd_q1": TUNE_FWD_Q1}
+                "fwd_causal_group": TUNE_FWD_CAUSAL_GROUP, "fwd_q1": TUNE_FWD_Q1,
+                "bwd_causal_group": TUNE_BWD_CAUSAL_GROUP}
 
 
 def set_tuning(knob: str, value: int) -> None:

@@ -149,6 +149,19 @@ int fwd_group_heads(int BH, int kv_group, int N, int d, int elem_bytes) {
   return static_cast<int>(g < 1 ? 1 : g > BH ? BH : g);
 }
 
+int bwd_causal_group() {
+  const int v = tune_raw(FA_TUNE_BWD_CAUSAL_GROUP);
+  return v >= 0 ? v : kDefaultBwdCausalGroup;
+}
+
+// K/V heads per group of the causal backward's CTA order.
+int bwd_group_kv(int BHkv, int kv_group, int N, int d) {
+  if (!bwd_causal_group()) return 1;
+  const long long per_kv = static_cast<long long>(N) * d * (4 + 8ll * kv_group);   // K, V; Q, dO, dQ acc
+  const long long g = kBwdGroupBytes / per_kv;
+  return static_cast<int>(g < 1 ? 1 : g > BHkv ? BHkv : g);
+}
+
 int bwd_pair() {
   const int v = tune_raw(FA_TUNE_BWD_PAIR);
   return v >= 0 ? v : kDefaultBwdPair;
@@ -438,6 +451,7 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.poly_groups = bwd_poly_groups();
   p.dq_poly = dq_poly_pairs();
+  p.group_kv = bwd_group_kv(BHkv, H / H_kv, N, d);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = launch_bwd_preprocess(static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout),
                                         delta, dq_acc, rows, d, s);
@@ -609,6 +623,7 @@ bool tuning_value_ok(int knob, int value) {
     case FA_TUNE_FWD_PERSISTENT: return value == 0 || value == 1;
     case FA_TUNE_FWD_CAUSAL_GROUP: return value == 0 || value == 1;
     case FA_TUNE_FWD_Q1: return value == 0 || value == 1;
+    case FA_TUNE_BWD_CAUSAL_GROUP: return value == 0 || value == 1;
     default: return false;
   }
 }
@@ -632,6 +647,7 @@ extern "C" int fa_get_tuning(int knob, int d) {
     case FA_TUNE_FWD_PERSISTENT: return d == 256 ? 1 : tune_raw(FA_TUNE_FWD_PERSISTENT);   // -1: chosen per call
     case FA_TUNE_FWD_CAUSAL_GROUP: return fwd_causal_group();
     case FA_TUNE_FWD_Q1: return d == 256 ? 0 : tune_raw(FA_TUNE_FWD_Q1);   // -1: chosen per call
+    case FA_TUNE_BWD_CAUSAL_GROUP: return bwd_causal_group();
     default: return -1;
   }
 }

@@ -223,9 +223,15 @@ __global__ void __launch_bounds__(BwdCfg<D, DQ>::kThreads, 1) bwd_main_kernel(co
   // With kv_split = S > 1 (few K/V heads) the G query heads of a group are
   // shared out over S CTAs per key block, G / S heads each; their dK, dV go
   // to fp32 partials that a reduction kernel sums in split order.
-  const int kvh = blockIdx.x / (p.n_kv * p.kv_split);
-  const int split = (blockIdx.x / p.n_kv) % p.kv_split;
-  const int j = blockIdx.x % p.n_kv;
+  // Causal: longest first within groups of K/V heads (causal_kv_order).
+  int kvh, split, j;
+  if (CAUSAL) {
+    causal_kv_order(static_cast<int>(blockIdx.x), p.n_kv, p.kv_split, p.group_kv, p.BH / p.kv_group, kvh, split, j);
+  } else {
+    kvh = blockIdx.x / (p.n_kv * p.kv_split);
+    split = (blockIdx.x / p.n_kv) % p.kv_split;
+    j = blockIdx.x % p.n_kv;
+  }
   const int g_per = p.kv_group / p.kv_split;   // query heads of this CTA
   const int i0 = CAUSAL ? j : 0;
   // Sliding window (causal): the last query block that sees a key of block j.

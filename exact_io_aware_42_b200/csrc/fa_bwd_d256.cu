@@ -92,9 +92,15 @@ __global__ void __launch_bounds__(320, 1) bwd_dq256_kernel(const __grid_constant
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // head-major; within a head, causal query blocks with the most key blocks first
-  const int bh = blockIdx.x / p.n_q;
-  const int i = CAUSAL ? p.n_q - 1 - static_cast<int>(blockIdx.x % p.n_q) : static_cast<int>(blockIdx.x % p.n_q);
+  // head-major non-causal; causal: longest first within groups of heads
+  // (causal_q_order)
+  int bh, i;
+  if (CAUSAL) {
+    causal_q_order(static_cast<int>(blockIdx.x), p.n_q, p.group_kv * p.kv_group, p.BH, bh, i);
+  } else {
+    bh = blockIdx.x / p.n_q;
+    i = static_cast<int>(blockIdx.x % p.n_q);
+  }
   const int n_kb = (p.N + 63) / 64;                   // 64-key blocks
   const int j_start = CAUSAL ? max(0, i * 128 - p.window) / 64 : 0;
   const int n_j = (CAUSAL ? min(2 * i + 2, n_kb) : n_kb) - j_start;
@@ -384,11 +390,18 @@ __global__ void __launch_bounds__(320, 1) bwd_kv256_kernel(const __grid_constant
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   // CTA -> (K/V head, split, key block j, head-dim half h); head-major
+  // non-causal; causal: longest first within groups of K/V heads
+  // (causal_kv_order), the two halves of a key block adjacent
   const int h = blockIdx.x & 1;
   const int rest = blockIdx.x >> 1;
-  const int kvh = rest / (p.n_kv * p.kv_split);
-  const int split = (rest / p.n_kv) % p.kv_split;
-  const int j = rest % p.n_kv;
+  int kvh, split, j;
+  if (CAUSAL) {
+    causal_kv_order(rest, p.n_kv, p.kv_split, p.group_kv, p.BH / p.kv_group, kvh, split, j);
+  } else {
+    kvh = rest / (p.n_kv * p.kv_split);
+    split = (rest / p.n_kv) % p.kv_split;
+    j = rest % p.n_kv;
+  }
   const int g_per = p.kv_group / p.kv_split;
   const int n_qb = (p.N + 63) / 64;                          // 64-query blocks
   const int i0 = CAUSAL ? 2 * j : 0;

@@ -93,9 +93,17 @@ __global__ void __launch_bounds__(320, 1) bwd_dq_kernel(const __grid_constant__ 
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Head-major; within a head, causal query blocks with the most key blocks first.
-  const int bh = blockIdx.x / p.n_q;
-  const int i = CAUSAL ? p.n_q - 1 - static_cast<int>(blockIdx.x % p.n_q) : static_cast<int>(blockIdx.x % p.n_q);
+  // Head-major non-causal.  Causal: within each group of group_kv K/V heads
+  // (their query heads), query blocks with the most key blocks first across
+  // the group's heads (the hardware hands CTAs out in index order: a
+  // longest-first schedule whose working set stays in L2).
+  int bh, i;
+  if (CAUSAL) {
+    causal_q_order(static_cast<int>(blockIdx.x), p.n_q, p.group_kv * p.kv_group, p.BH, bh, i);
+  } else {
+    bh = blockIdx.x / p.n_q;
+    i = static_cast<int>(blockIdx.x % p.n_q);
+  }
   // Sliding window (causal): key blocks wholly left of the window are skipped.
   const int j_start = CAUSAL ? max(0, i * 128 - p.window) / 128 : 0;
   const int n_j = (CAUSAL ? i + 1 : p.n_kv) - j_start;   // iterations; block = j_start + j

@@ -118,11 +118,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
   const int lane = threadIdx.x & 31;
   // Pair index -> (K/V head, split, 256-key block J); this CTA's keys are
   // [256 J + 128 rank, 256 J + 128 rank + 128), key block j = 2 J + rank.
+  // Head-major non-causal; causal: longest first within groups of K/V heads
+  // (causal_kv_order over 256-key blocks).
   const int n_kv2 = (p.N + 255) / 256;
   const int pair = blockIdx.x >> 1;
-  const int kvh = pair / (n_kv2 * p.kv_split);
-  const int split = (pair / n_kv2) % p.kv_split;
-  const int J = pair % n_kv2;
+  int kvh, split, J;
+  if (CAUSAL) {
+    causal_kv_order(pair, n_kv2, p.kv_split, p.group_kv, p.BH / p.kv_group, kvh, split, J);
+  } else {
+    kvh = pair / (n_kv2 * p.kv_split);
+    split = (pair / n_kv2) % p.kv_split;
+    J = pair % n_kv2;
+  }
   const int j = 2 * J + static_cast<int>(rank);
   const int g_per = p.kv_group / p.kv_split;
   // query blocks of the pair: causal from the first block that sees key

@@ -157,9 +157,15 @@ struct BwdParams {
   float scale_log2;     // scale * log2(e)
   float scale;
   int poly_groups;      // of every 4 groups of 4 columns, how many use the FMA-pipe exp2
+  int group_kv;         // causal CTA order: longest first within groups of this many K/V heads
+                        // (1: head by head)
 };
 
 constexpr int kDefaultBwdPolyGroups = 0;
+// Causal backward CTA order: longest first within groups of K/V heads whose
+// K, V, Q, dO and dQ accumulator take about this many bytes (1: head by head).
+constexpr long long kBwdGroupBytes = 48ll << 20;
+constexpr int kDefaultBwdCausalGroup = 1;
 // dK, dV of the deterministic backward at d = 128 on CTA pairs (1) or single CTAs (0)
 constexpr int kDefaultBwdPair = 0;
 constexpr int kDefaultDqPolyPairsD64 = 0;   // measured: the polynomial share did not help (latency-bound)
@@ -182,5 +188,32 @@ cudaError_t launch_bwd_kv_reduce(const float* part, uint16_t* dv, uint16_t* dk, 
 // dq <- bf16(scale * dq_acc)
 cudaError_t launch_bwd_postprocess(const float* dq_acc, uint16_t* dq, long long n, float scale,
                                    cudaStream_t stream);
+
+// Causal backward CTA order.  The hardware hands CTAs to SMs in index order
+// as SMs free up, so ordering the CTAs by decreasing work gives a dynamic
+// longest-first schedule; doing it within groups of group_kv K/V heads keeps
+// each group's K, V, Q, dO and dQ accumulator in L2 while its CTAs run.
+// Key-block CTAs (u over groups x key blocks j, small j first x the group's
+// K/V heads x splits):
+__device__ __forceinline__ void causal_kv_order(int u, int n_kv, int kv_split, int group_kv, int BHkv, int& kvh,
+                                                int& split, int& j) {
+  const int per_group = group_kv * kv_split * n_kv;
+  const int g = u / per_group;
+  const int rr = u - g * per_group;
+  const int lanes = min(group_kv, BHkv - g * group_kv) * kv_split;
+  j = rr / lanes;
+  kvh = g * group_kv + (rr % lanes) / kv_split;
+  split = (rr % lanes) % kv_split;
+}
+// Query-block CTAs (u over groups of gq query heads x query blocks i, large i
+// first x the group's query heads):
+__device__ __forceinline__ void causal_q_order(int u, int n_q, int gq, int BH, int& bh, int& i) {
+  const int per_group = gq * n_q;
+  const int g = u / per_group;
+  const int rr = u - g * per_group;
+  const int lanes = min(gq, BH - g * gq);
+  i = n_q - 1 - rr / lanes;
+  bh = g * gq + rr % lanes;
+}
 
 }  // namespace fa

@@ -273,6 +273,9 @@ fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v8, const fl
  *                           by default chosen per call (the one-tile kernel when
  *                           the problem has fewer pairs of query tiles than the
  *                           device has SMs), which fa_get_tuning reports as -1
+ *  FA_TUNE_BWD_CAUSAL_GROUP causal backward (main and dQ kernels): CTAs ordered
+ *                           longest first within groups of heads whose working
+ *                           set fits in L2 (1), or head by head (0)
  * value -1 restores the built-in default.  Any other value, or an unknown
  * knob, is FA_ERR_INVALID_ARG.  fa_get_tuning returns the value a call with
  * head dim d would use now.
@@ -287,7 +290,8 @@ typedef enum fa_tune_knob {
   FA_TUNE_FWD_PERSISTENT = 8,
   FA_TUNE_FWD_CAUSAL_GROUP = 9,
   FA_TUNE_FWD_Q1 = 10,
-  FA_TUNE_COUNT = 11
+  FA_TUNE_BWD_CAUSAL_GROUP = 11,
+  FA_TUNE_COUNT = 12
 } fa_tune_knob;
 fa_status fa_set_tuning(int knob, int value);
 int fa_get_tuning(int knob, int d);

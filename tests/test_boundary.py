@@ -143,12 +143,14 @@ def test_tuning_controls(L):
     assert L.fa_get_tuning(TUNE_FWD_POLY_DEGREE, 64) in (3, 4)
     assert L.fa_get_tuning(TUNE_DQ_POLY_PAIRS, 128) == 0
     assert L.fa_get_tuning(99, 64) == -1
-    from exact_io_aware_42_b200._lib import TUNE_FWD_CAUSAL_GROUP, TUNE_FWD_PERSISTENT, TUNE_FWD_Q1
+    from exact_io_aware_42_b200._lib import (TUNE_BWD_CAUSAL_GROUP, TUNE_FWD_CAUSAL_GROUP, TUNE_FWD_PERSISTENT,
+                                             TUNE_FWD_Q1)
     assert L.fa_get_tuning(TUNE_FWD_Q1, 128) == -1      # chosen per call by default
     assert L.fa_get_tuning(TUNE_FWD_PERSISTENT, 128) == -1
     assert L.fa_get_tuning(TUNE_FWD_PERSISTENT, 256) == 1   # the d = 256 kernel is always persistent
     assert L.fa_set_tuning(7, 0) == 1                   # a retired knob number
-    for knob in (TUNE_FWD_PERSISTENT, TUNE_FWD_CAUSAL_GROUP, TUNE_FWD_Q1):
+    assert L.fa_get_tuning(TUNE_BWD_CAUSAL_GROUP, 128) == 1
+    for knob in (TUNE_FWD_PERSISTENT, TUNE_FWD_CAUSAL_GROUP, TUNE_FWD_Q1, TUNE_BWD_CAUSAL_GROUP):
         default = L.fa_get_tuning(knob, 128)
         assert default in ((-1,) if knob in (TUNE_FWD_Q1, TUNE_FWD_PERSISTENT) else (0, 1))
         for v in (0, 1):

@@ -102,6 +102,31 @@ def test_det_bwd_bitwise_reproducible_and_matches_atomic_dk_dv(causal):
     assert rel_rms(a[0], atomic[0]) <= 5e-3
 
 
+@pytest.mark.parametrize("d,H,H_kv,N,pair", [(128, 16, 16, 2048, 0), (64, 12, 4, 1300, 0), (128, 8, 8, 1536, 1),
+                                              (256, 4, 2, 1000, 0), (128, 4, 1, 2048, 0)])
+def test_det_bwd_causal_cta_order_does_not_change_results(d, H, H_kv, N, pair):
+    """The causal CTA order (longest first within L2-sized head groups, or
+    head by head) only changes which SM runs which block: the deterministic
+    dQ, dK, dV agree bit for bit, for the single-CTA, CTA-pair (d = 128) and
+    d = 256 kernels, grouped K/V heads and the split MQA path."""
+    fa = _fa()
+    q, k, v, do = (t.cuda() for t in inputs.make_gqa(2, H, H_kv, N, d, seed=4000 + N + d, with_do=True))
+    o, lse = fa.fwd(q, k, v, causal=True)
+    out = {}
+    try:
+        fa.set_tuning("bwd_pair", pair)
+        for grouped in (0, 1):
+            fa.set_tuning("bwd_causal_group", grouped)
+            out[grouped] = fa.bwd(q, k, v, o, do, lse, causal=True, deterministic=True)
+            torch.cuda.synchronize()
+    finally:
+        fa.set_tuning("bwd_causal_group", -1)
+        fa.set_tuning("bwd_pair", -1)
+    assert fa.get_status() == 0
+    for a_, b_ in zip(out[0], out[1]):
+        assert torch.equal(a_, b_)
+
+
 def test_det_bwd_workspace_size_and_errors():
     fa = _fa()
     assert fa.bwd_workspace_size(2, 3, 100, 64, deterministic=True) == 2560
