@@ -135,15 +135,15 @@ int fwd_q1(long long pair_items, int sms) {
   return v >= 0 ? v : (pair_items < sms ? 1 : 0);
 }
 
-int fwd_causal_group() {
+int fwd_causal_group(bool persistent) {
   const int v = tune_raw(FA_TUNE_FWD_CAUSAL_GROUP);
-  return v >= 0 ? v : kDefaultFwdCausalGroup;
+  return v >= 0 ? v : persistent ? kDefaultFwdCausalGroupPersistent : kDefaultFwdCausalGroupOneCta;
 }
 
 // Heads per group of the causal item order (see FwdParams::group_heads):
 // K and V of the group's K/V heads within kCausalGroupBytes.
-int fwd_group_heads(int BH, int kv_group, int N, int d, int elem_bytes) {
-  if (!fwd_causal_group()) return BH;
+int fwd_group_heads(int BH, int kv_group, int N, int d, int elem_bytes, bool persistent) {
+  if (!fwd_causal_group(persistent)) return BH;
   const long long kv_bytes = 2ll * N * d * elem_bytes;   // K and V of one K/V head
   const long long g = kCausalGroupBytes / kv_bytes * kv_group;
   return static_cast<int>(g < 1 ? 1 : g > BH ? BH : g);
@@ -314,7 +314,7 @@ extern "C" fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void
   p.o = static_cast<uint16_t*>(o);
   p.sms = di->sms;
   p.persistent = d == 256 ? 1 : fwd_persistent(false, causal != 0, poly_pairs(d), alibi_slopes);
-  p.group_heads = fwd_group_heads(B * H, H / H_kv, N, d, 2);
+  p.group_heads = fwd_group_heads(B * H, H / H_kv, N, d, 2, p.persistent != 0);
   if (!p.persistent && !encode_3d(&p.tm_o, o, bf, 2, d, N, BH, 64, kBlockM)) return FA_ERR_INVALID_ARG;
   p.lse = lse;
   p.status = di->status;
@@ -572,7 +572,7 @@ extern "C" fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v
   p.o = static_cast<uint16_t*>(o);
   p.sms = di->sms;
   p.persistent = fwd_persistent(true, causal != 0, fp8_poly_pairs(), alibi_slopes);
-  p.group_heads = fwd_group_heads(B * H, H / H_kv, N, d, 1);
+  p.group_heads = fwd_group_heads(B * H, H / H_kv, N, d, 1, p.persistent != 0);
   if (!p.persistent &&
       !encode_3d(&p.tm_o, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, BH, 64, kBlockM))
     return FA_ERR_INVALID_ARG;
@@ -645,7 +645,7 @@ extern "C" int fa_get_tuning(int knob, int d) {
     case FA_TUNE_FP8_POLY_PAIRS: return fp8_poly_pairs();
     case FA_TUNE_BWD_PAIR: return d == 128 ? bwd_pair() : 0;
     case FA_TUNE_FWD_PERSISTENT: return d == 256 ? 1 : tune_raw(FA_TUNE_FWD_PERSISTENT);   // -1: chosen per call
-    case FA_TUNE_FWD_CAUSAL_GROUP: return fwd_causal_group();
+    case FA_TUNE_FWD_CAUSAL_GROUP: return tune_raw(FA_TUNE_FWD_CAUSAL_GROUP);   // -1: by the grid
     case FA_TUNE_FWD_Q1: return d == 256 ? 0 : tune_raw(FA_TUNE_FWD_Q1);   // -1: chosen per call
     case FA_TUNE_BWD_CAUSAL_GROUP: return bwd_causal_group();
     default: return -1;

@@ -804,9 +804,12 @@ const FwdSched* causal_schedule(const FwdParams& p, int G) {
       const int n1 = std::min(qt0 + 2, p.n_kv) - j_start;
       cost[o] = 2 * n1 + 1;
     }
+    // items in order of decreasing cost; with head groups (group_heads <
+    // BH) group by group, each group's items longest first (item_at's order)
     std::vector<int> order(items);
     std::iota(order.begin(), order.end(), 0);
-    std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return cost[a] > cost[b]; });
+    if (p.group_heads >= p.BH)
+      std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return cost[a] > cost[b]; });
     std::vector<long long> load(G, 0);
     std::vector<std::vector<int>> lists(G);
     for (const int o : order) {

@@ -83,12 +83,15 @@ constexpr int kDefaultFwdPersistentCausal = 1;
 constexpr int kDefaultFwdPersistentNonCausal = 1;
 constexpr int kDefaultFwdPersistentFp8Causal = 1;
 constexpr int kDefaultFwdPersistentFp8NonCausal = 0;
-// Causal CTA order of the one-CTA-per-item kernel, measured (same-process
-// A/B): grouping heads helped only once K and V of all heads far exceed L2
-// (B8 H16 N4096 d128: 948 vs 910 TFLOPS) and cost about 1% at B4 H16 N4096
-// (926 vs 932) and B1 H16 N16384, so the global longest-first order is the
-// default.
-constexpr int kDefaultFwdCausalGroup = 0;
+// Causal item order of the two-tile forward, measured (same-process A/B):
+// with one CTA per work item, grouping heads helped only once K and V of all
+// heads far exceed L2 (B8 H16 N4096 d128: 948 vs 910 TFLOPS) and cost about
+// 1% at B4 H16 N4096 (926 vs 932) and B1 H16 N16384, so that grid orders
+// globally by default; the persistent grid's host-made deal gains from the
+// groups (B4 H16 N4096 d128 962 vs 969, B1 H16 N16384 1143 vs 1160, d64 601
+// vs 606, FP8 857 vs 863), so it groups by default.
+constexpr int kDefaultFwdCausalGroupOneCta = 0;
+constexpr int kDefaultFwdCausalGroupPersistent = 1;
 // bf16 forward at d <= 128: the one-tile kernel with two score buffers runs
 // by default only where the two-tile kernel would have fewer work items
 // (pairs of query tiles) than SMs; measured on B200: B2 H8 N1024 d64 causal

@@ -264,9 +264,11 @@ fa_status fa_fwd_fp8_ex(const void* q8, const void* k8, const void* v8, const fl
  *                           non-causal forward), which fa_get_tuning reports as -1; calls
  *                           with ALiBi or a polynomial exp2 share use one CTA
  *                           per item
- *  FA_TUNE_FWD_CAUSAL_GROUP causal forward, one CTA per work item: longest
- *                           first within groups of heads whose K and V fit in
- *                           L2 together (1), or over all heads (0)
+ *  FA_TUNE_FWD_CAUSAL_GROUP causal two-tile forward: work items longest first
+ *                           within groups of heads whose K and V fit in L2
+ *                           together (1), or over all heads (0); by default
+ *                           grouped on the persistent grid and global with one
+ *                           CTA per work item, which fa_get_tuning reports as -1
  *  FA_TUNE_FWD_Q1           bf16 forward, d <= 128: one 128-row query tile per
  *                           work item with two score buffers (1), or two query
  *                           tiles per CTA (0; FA_TUNE_FWD_PERSISTENT picks which);

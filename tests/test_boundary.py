@@ -152,7 +152,7 @@ def test_tuning_controls(L):
     assert L.fa_get_tuning(TUNE_BWD_CAUSAL_GROUP, 128) == 1
     for knob in (TUNE_FWD_PERSISTENT, TUNE_FWD_CAUSAL_GROUP, TUNE_FWD_Q1, TUNE_BWD_CAUSAL_GROUP):
         default = L.fa_get_tuning(knob, 128)
-        assert default in ((-1,) if knob in (TUNE_FWD_Q1, TUNE_FWD_PERSISTENT) else (0, 1))
+        assert default in ((-1,) if knob in (TUNE_FWD_Q1, TUNE_FWD_PERSISTENT, TUNE_FWD_CAUSAL_GROUP) else (0, 1))
         for v in (0, 1):
             assert L.fa_set_tuning(knob, v) == 0 and L.fa_get_tuning(knob, 128) == v
         assert L.fa_set_tuning(knob, 2) == 1

@@ -169,7 +169,7 @@ def test_fwd_exp2_split_variants(d, pairs, deg, causal, restore_tuning):
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("persistent,group,q1", [(0, 1, 0), (0, 0, 0), (1, 0, 0), (0, 0, 1)])
+@pytest.mark.parametrize("persistent,group,q1", [(0, 1, 0), (0, 0, 0), (1, 0, 0), (1, 1, 0), (0, 0, 1)])
 def test_fwd_kernel_variants_every_head(d, persistent, group, q1, restore_tuning):
     """The forward kernels (two query tiles per item: one CTA per work item,
     with the grouped and the global causal order, or the persistent grid; one
