@@ -108,9 +108,6 @@ struct TileCfg {
   static constexpr uint32_t kColP = 384;
   // P outside S: S_t(j+1) may start as soon as S_t(j) has been read out
   static constexpr bool kEarlyS = kSepP;
-  // bf16: the first copies go out before the CTA-wide sync (the FP8 build
-  // measured slower that way)
-  static constexpr bool kEarlyLoads = !FP8;
 };
 static_assert(TileCfg<128, true>::kSmemBytes <= 232448, "fp8 forward shared memory");
 static_assert(TileCfg<128, false>::kSmemBytes <= 232448, "bf16 forward shared memory");
@@ -251,7 +248,7 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(
                   pn * C::kPanelElems, (it.qt0 + t) * kBlockM, it.bh);
   };
   // ring copies of the first item that need no free slot
-  const int n_first = (C::kEarlyLoads && it0.bh < p.BH) ? min(NS, 2 * it0.n1) : 0;
+  const int n_first = it0.bh < p.BH ? min(NS, 2 * it0.n1) : 0;
   if (warp == 8 && lane == 0) {
     mbar_init(bar(bar_q(0)), 1);
     mbar_init(bar(bar_q(1)), 1);
@@ -269,16 +266,14 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(
     mbar_init(bar(bar_drain<NS>()), 1);
     *abort_flag = 0;
     fence_mbar_init();
-    if constexpr (C::kEarlyLoads) {
-      tma_prefetch_desc(&p.tm_q);
-      tma_prefetch_desc(&p.tm_k);
-      tma_prefetch_desc(&p.tm_v);
-      if (n_first > 0) {
-        load_q(0, it0);
-        load_kv(0, it0, 0);
-        load_q(1, it0);
-        for (int sq = 1; sq < n_first; ++sq) load_kv(sq, it0, sq);
-      }
+    tma_prefetch_desc(&p.tm_q);
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
+    if (n_first > 0) {
+      load_q(0, it0);
+      load_kv(0, it0, 0);
+      load_q(1, it0);
+      for (int sq = 1; sq < n_first; ++sq) load_kv(sq, it0, sq);
     }
   }
   if (warp == 9) {
@@ -294,12 +289,7 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      if constexpr (!C::kEarlyLoads) {
-        tma_prefetch_desc(&p.tm_q);
-        tma_prefetch_desc(&p.tm_k);
-        tma_prefetch_desc(&p.tm_v);
-      }
-      int seq = n_first;   // bf16: the first ring round went out before the sync
+      int seq = n_first;   // the first ring round went out before the sync
       int nq[2] = {n_first > 0 ? 1 : 0, n_first > 0 ? 1 : 0};   // Q loads issued per tile
       bool ok = true;
       for (int k = 0; ok && (PERS || k == 0); ++k) {
@@ -620,6 +610,7 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(
           const float f8 = 256.f * sv_j / v_max;
           const uint64_t c2 = f2_pack(c, c);
           const uint64_t nm2 = f2_pack(neg_m, neg_m);
+          const uint64_t f82 = f2_pack(f8, f8);   // P is stored as E4M3 of p * f8 (packed products)
           float keep0 = 0.f, keep1 = 0.f;
 #pragma unroll
           for (int i = 0; i < 64; ++i) {
@@ -627,12 +618,12 @@ __global__ void __launch_bounds__(320, 1) fwd_tile_kernel(
             const uint64_t x2 = masked ? f2_add(s2, nm2) : f2_fma(s2, c2, nm2);
             const uint64_t p2 = ((i & 7) < NPOLY) ? exp2_poly_f2<DEG>(x2) : exp2_sfu_f2(x2);
             acc[i & 3] = f2_add(acc[i & 3], p2);
-            float p0, p1;
-            f2_unpack(p2, p0, p1);
+            float q0, q1;
+            f2_unpack(f2_mul(p2, f82), q0, q1);
             if (i & 1)
-              u[i / 2] = pack_e4m3x4(keep0 * f8, keep1 * f8, p0 * f8, p1 * f8);
-            keep0 = p0;
-            keep1 = p1;
+              u[i / 2] = pack_e4m3x4(keep0, keep1, q0, q1);
+            keep0 = q0;
+            keep1 = q1;
           }
           tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
         } else {
