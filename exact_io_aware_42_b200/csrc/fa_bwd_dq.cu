@@ -309,10 +309,14 @@ __global__ void __launch_bounds__(320, 1) bwd_dq_kernel(const __grid_constant__ 
       {
         uint32_t dp[64];
         tmem_ld64(tDP, dp);
+        // dS = P (dP - D), two columns per fp32x2 operation (dP + (-D) is dP - D exactly)
+        const uint64_t nd2 = f2_pack(-dlt, -dlt);
 #pragma unroll
         for (int c2 = 0; c2 < 32; ++c2) {
-          const float d0 = __uint_as_float(u[2 * c2]) * (__uint_as_float(dp[2 * c2]) - dlt);
-          const float d1 = __uint_as_float(u[2 * c2 + 1]) * (__uint_as_float(dp[2 * c2 + 1]) - dlt);
+          float d0, d1;
+          f2_unpack(f2_mul(f2_pack(__uint_as_float(u[2 * c2]), __uint_as_float(u[2 * c2 + 1])),
+                           f2_add(f2_pack(__uint_as_float(dp[2 * c2]), __uint_as_float(dp[2 * c2 + 1])), nd2)),
+                    d0, d1);
           ds[c2] = pack_bf16x2(d0, d1);
         }
       }
