@@ -456,17 +456,26 @@ __global__ void __launch_bounds__(320, 1) bwd_kv256_kernel(const __grid_constant
         tma_load_3d(vAddr + pn * kP128, &p.tm_v, bar(B_KV), pn * 64, j * 128, kvh);
       }
     }
-    // L (log2 units, +inf past N) or D (0 past N) of the 64 queries of block i
-    auto stage_rows = [&](float* dst, const float* src, int qh, int i, float mul, float pad) {
-      float v2[2];
+    // L (log2 units, +inf past N) and D (0 past N) of the 64 queries of
+    // block idx, two per lane.  The next block's values are loaded into
+    // registers right after this block's copies are issued, so their latency
+    // runs while the warp waits for the next free slots instead of delaying
+    // the next copies.
+    auto fetch_rows = [&](int idx, float2& l2, float2& d2) {
+      const int i = q_block(idx), qh = q_head(idx);
+      float lv[2], dv[2];
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         const int q = i * 64 + lane * 2 + t;
-        v2[t] = q < p.N ? src[static_cast<size_t>(qh) * p.N + q] * mul : pad;
+        const size_t g = static_cast<size_t>(qh) * p.N + q;
+        lv[t] = q < p.N ? p.lse[g] * 1.4426950408889634f : INFINITY;
+        dv[t] = q < p.N ? p.delta[g] : 0.f;
       }
-      reinterpret_cast<float2*>(dst)[lane] = make_float2(v2[0], v2[1]);
-      __syncwarp();
+      l2 = make_float2(lv[0], lv[1]);
+      d2 = make_float2(dv[0], dv[1]);
     };
+    float2 l_next = make_float2(0.f, 0.f), d_next = l_next;
+    if (n_it > 0) fetch_rows(0, l_next, d_next);
     for (int idx = 0; idx < n_it && ok; ++idx) {
       const int i = q_block(idx), qh = q_head(idx);
       const int sq = idx % NQ, sd = idx % ND;
@@ -475,8 +484,9 @@ __global__ void __launch_bounds__(320, 1) bwd_kv256_kernel(const __grid_constant
       if (!(ok = __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0)) break;
       // L and D of the block live with the Q stage: both are read before
       // the dS phase ends, and the stage is released after dK, which follows it
-      stage_rows(reinterpret_cast<float*>(smem + C::kOffL + sq * 256), p.lse, qh, i, 1.4426950408889634f, INFINITY);
-      stage_rows(reinterpret_cast<float*>(smem + C::kOffDl + sq * 256), p.delta, qh, i, 1.f, 0.f);
+      reinterpret_cast<float2*>(smem + C::kOffL + sq * 256)[lane] = l_next;
+      reinterpret_cast<float2*>(smem + C::kOffDl + sq * 256)[lane] = d_next;
+      __syncwarp();
       if (lane == 0) {
         mbar_arrive_expect_tx(bar(B_QF(sq)), C::kTileQ);
         for (int pn = 0; pn < 4; ++pn)
@@ -491,6 +501,7 @@ __global__ void __launch_bounds__(320, 1) bwd_kv256_kernel(const __grid_constant
           tma_load_3d(doAddr(sd) + pn * kP64, &p.tm_do64, bar(B_DF(sd)), pn * 64, i * 64, qh);
         ++issued_d;
       }
+      if (idx + 1 < n_it) fetch_rows(idx + 1, l_next, d_next);
     }
     if (lane == 0 && *abort_flag) {
       volatile int never = 0;
