@@ -150,18 +150,29 @@ __global__ void __launch_bounds__(320, 1) bwd_dq256_kernel(const __grid_constant
       }
       int nk = 0, nv = 0;
       bool ok = true;
-      for (int j = 0; j < n_j && ok; ++j) {
-        const int sk = j % NK, sv = j % NV;
-        if (!(ok = mbar_wait(bar(B_KE(sk)), ((j / NK) & 1) ^ 1, ab, kQ2Prod))) break;
+      auto load_k = [&](int j) {
+        const int sk = j % NK;
+        if (!mbar_wait(bar(B_KE(sk)), ((j / NK) & 1) ^ 1, ab, kQ2Prod)) return false;
         mbar_arrive_expect_tx(bar(B_KF(sk)), C::kTileK);
         for (int pn = 0; pn < 4; ++pn)
           tma_load_3d(kAddr(sk) + pn * kP64, &p.tm_k64, bar(B_KF(sk)), pn * 64, (j_start + j) * 64, kvh);
         ++nk;
-        if (!(ok = mbar_wait(bar(B_VE(sv)), ((j / NV) & 1) ^ 1, ab, kQ2Prod))) break;
+        return true;
+      };
+      auto load_v = [&](int j) {
+        const int sv = j % NV;
+        if (!mbar_wait(bar(B_VE(sv)), ((j / NV) & 1) ^ 1, ab, kQ2Prod)) return false;
         mbar_arrive_expect_tx(bar(B_VF(sv)), C::kTileK);
         for (int pn = 0; pn < 4; ++pn)
           tma_load_3d(vAddr(sv) + pn * kP64, &p.tm_v64, bar(B_VF(sv)), pn * 64, (j_start + j) * 64, kvh);
         ++nv;
+        return true;
+      };
+      // V_j's slot is freed by dP_{j-1}, K_j's by dQ_{j-2}, which the MMA
+      // issuer runs after it: past the first ring of K, V goes out first.
+      for (int j = 0; j < n_j && ok; ++j) {
+        if (j < NK) ok = load_k(j) && load_v(j);
+        else ok = load_v(j) && load_k(j);
       }
       if (*abort_flag) {   // let the copies in flight land before the CTA leaves
         volatile int never = 0;
