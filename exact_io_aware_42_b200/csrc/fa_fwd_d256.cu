@@ -15,15 +15,20 @@
 // panel each): S(j) = sum over the 4 panels p of Q_p K_{j,p}^T, and
 // O[:, 64 p .. 64 p + 63] += P(j) V_{j,p} (N = 64 per product).
 //
-// Roles (192 threads):
-//   warps 0-3  softmax (thread r owns query row r = TMEM lane r) and the
-//              epilogue (O / l written from registers to global memory)
-//   warp  4    TMA producer: Q (4 panels), then the key blocks' panels in
+// Roles (320 threads):
+//   warps 0-7  softmax and the epilogue: thread = query row = TMEM lane;
+//              warpgroup wg takes key columns [64 wg, 64 wg + 64) of every
+//              score tile and O columns [128 wg, 128 wg + 128).  The two
+//              warps of a row exchange partial row maxima through shared
+//              memory, so both take the same max and rescale decision, and
+//              keep partial row sums that are added at the epilogue.
+//   warp  8    TMA producer: Q (4 panels), then the key blocks' panels in
 //              the order the products consume them: K(0), K(1), V(0), K(2),
 //              V(1), ... into the panel ring (full/empty mbarriers)
-//   warp  5    allocates TMEM; one thread issues every tcgen05.mma
-// TMEM: [0,128) and [128,256) score buffers (P packed over the first 64
-// columns of its buffer as bf16 pairs), [256,512) O.
+//   warp  9    allocates TMEM; one thread issues every tcgen05.mma
+// TMEM: [0,128) and [128,256) score buffers (each warpgroup packs its 64
+// P values as bf16 pairs over the first 32 of its own 64 columns),
+// [256,512) O.
 //
 // The grid is persistent: one CTA per SM walks its share of the (b, h,
 // query tile) items, longest first when causal, in snake order.  Causal
@@ -45,13 +50,14 @@ struct F256 {
   static constexpr int kPanels = 4;                  // 64-element panels of a row
   static constexpr int kPanelBytes = 128 * 128;      // 128 rows x 128 bytes
   static constexpr int kStages = 10;                 // panel ring
-  static constexpr int kThreads = 192;
+  static constexpr int kThreads = 320;
   static constexpr int kOffQ = 0;                    // 4 panels
   static constexpr int kOffRing = kPanels * kPanelBytes;
   static constexpr int kOffBar = kOffRing + kStages * kPanelBytes;
   static constexpr int kNumBars = 10 + 2 * kStages;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // + base alignment slack
+  static constexpr int kOffRed = kOffMisc + 16;      // partial row maxima / sums: [2 slots][2 wg][128] fp32
+  static constexpr int kSmemBytes = kOffRed + 2 * 2 * 128 * 4;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS = 0;      // + 128 * buffer
   static constexpr uint32_t kColO = 256;
@@ -59,13 +65,13 @@ struct F256 {
 static_assert(F256::kSmemBytes <= 232448, "d = 256 forward shared memory");
 
 // barrier slots
-constexpr int kBarQ = 0, kBarQFree = 1, kBarP = 2, kBarPH = 3, kBarPV = 4, kBarOFree = 5, kBarDrain = 6;
+constexpr int kBarQ = 0, kBarQFree = 1, kBarP = 2, kBarPV = 4, kBarOFree = 5, kBarDrain = 6;   // slot 3 unused
 __device__ __forceinline__ int bar_s256(int b) { return 7 + b; }                 // S buffer b written
 __device__ __forceinline__ int bar_full256(int s) { return 10 + s; }
 __device__ __forceinline__ int bar_empty256(int s) { return 10 + F256::kStages + s; }
 
 enum : unsigned int { kS2ProdEmpty = 60, kS2ProdQ, kS2MmaQ, kS2MmaFull, kS2MmaP, kS2MmaO, kS2SmS, kS2SmPv,
-                      kS2EpiPv, kS2Drain };
+                      kS2EpiPv, kS2Drain, kS2Align };
 
 __device__ __forceinline__ void st_global_v4_256(void* dst, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "r"(a), "r"(b), "r"(c), "r"(d)
@@ -97,14 +103,16 @@ __device__ __forceinline__ int my_item256(int k) {
 }
 
 template <bool CAUSAL, int NPOLY, int DEG>
-__global__ void __launch_bounds__(192, 1) fwd256_kernel(const __grid_constant__ FwdParams p) {
+__global__ void __launch_bounds__(F256::kThreads, 1) fwd256_kernel(const __grid_constant__ FwdParams p) {
   using C = F256;
   constexpr int NS = C::kStages;
   constexpr int D = C::D;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {   // the swizzled layouts need a 1024-byte aligned base
+    if (threadIdx.x == 0) atomicCAS(p.status, 0u, FA_ERR_LAUNCH | (kS2Align << 8));
+    return;
+  }
   auto bar = [&](int i) -> uint32_t { return sbase + C::kOffBar + 8 * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
@@ -116,10 +124,9 @@ __global__ void __launch_bounds__(192, 1) fwd256_kernel(const __grid_constant__ 
   if (threadIdx.x == 0) {
     mbar_init(bar(kBarQ), 1);
     mbar_init(bar(kBarQFree), 1);
-    mbar_init(bar(kBarP), 128);
-    mbar_init(bar(kBarPH), 128);
+    mbar_init(bar(kBarP), 256);
     mbar_init(bar(kBarPV), 1);
-    mbar_init(bar(kBarOFree), 128);
+    mbar_init(bar(kBarOFree), 256);
     mbar_init(bar(kBarDrain), 1);
     for (int b = 0; b < 2; ++b) mbar_init(bar(bar_s256(b)), 1);
     for (int s = 0; s < NS; ++s) {
@@ -129,7 +136,7 @@ __global__ void __launch_bounds__(192, 1) fwd256_kernel(const __grid_constant__ 
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
     tmem_relinquish();
   }
@@ -139,7 +146,7 @@ __global__ void __launch_bounds__(192, 1) fwd256_kernel(const __grid_constant__ 
   const uint32_t tmem = *tmem_slot;
   const Abort ab{abort_flag, p.status};
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_q);
@@ -183,7 +190,7 @@ __global__ void __launch_bounds__(192, 1) fwd256_kernel(const __grid_constant__ 
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);
@@ -219,8 +226,9 @@ __global__ void __launch_bounds__(192, 1) fwd256_kernel(const __grid_constant__ 
         ++gS;
         return true;
       };
-      // O += P(gP) V_j in two halves of 64 keys (after bar_p, then bar_ph),
-      // each over the 4 V panels (64 O columns each).
+      // O += P(gP) V_j once both warpgroups have stored their P and
+      // rescaled their O columns: keys [64 h, 64 h + 64) from warpgroup h's
+      // packed P, each half over the 4 V panels (64 O columns each).
       auto issue_pv = [&](bool acc) -> bool {
         const int b = gP & 1;
         int slot[C::kPanels];
@@ -229,16 +237,16 @@ __global__ void __launch_bounds__(192, 1) fwd256_kernel(const __grid_constant__ 
           if (!mbar_wait(bar(bar_full256(slot[pn])), (seq / NS) & 1, ab, kS2MmaFull)) return false;
           ++seq;
         }
+        if (!mbar_wait(bar(kBarP), gP & 1, ab, kS2MmaP)) return false;
+        tc_fence_after();
         for (int h = 0; h < 2; ++h) {
-          if (!mbar_wait(bar(h ? kBarPH : kBarP), gP & 1, ab, kS2MmaP)) return false;
-          tc_fence_after();
 #pragma unroll
           for (int pn = 0; pn < C::kPanels; ++pn) {
             const uint32_t va = sbase + C::kOffRing + slot[pn] * C::kPanelBytes;
 #pragma unroll
             for (int kq = 0; kq < 4; ++kq) {
               const int kk = 4 * h + kq;     // 16 keys per product
-              mma_f16_ts(tmem + C::kColO + 64 * pn, tmem + C::kColS + 128 * b + kk * 8,
+              mma_f16_ts(tmem + C::kColO + 64 * pn, tmem + C::kColS + 128 * b + 64 * h + 8 * kq,
                          smem_desc_sw128(va + kk * 16 * 128, C::kPanelBytes, 1024), kIdescO,
                          (acc || kk > 0) ? 1u : 0u);
             }
@@ -273,10 +281,14 @@ __global__ void __launch_bounds__(192, 1) fwd256_kernel(const __grid_constant__ 
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax (warps 0-3)
-    const int r = threadIdx.x;                 // query row within the tile == TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tO = tmem + C::kColO + lane_off;
+    // ------------------------------------------------------------ softmax (warps 0-7)
+    const int wg = warp >> 2;
+    const int r = threadIdx.x & 127;            // query row within the tile == TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tO = tmem + C::kColO + lane_off + 128u * wg;   // this warpgroup's O columns
+    const uint32_t pair_bar = 2 + (warp & 3);   // warps w and w + 4 share rows
+    float* red = reinterpret_cast<float*>(smem + C::kOffRed);
+    auto red_at = [&](int slot, int w) -> float& { return red[(slot * 2 + w) * 128 + r]; };
     int g = 0;         // score tiles over all items: buffer g % 2, barrier phases
     bool ok = true;
     for (int k = 0; ok; ++k) {
@@ -288,54 +300,57 @@ __global__ void __launch_bounds__(192, 1) fwd256_kernel(const __grid_constant__ 
       const int row = qi * kBlockM + r;
       const float c = p.scale_log2;
       float m_use = -INFINITY;
-      float l = 0.f;
+      float l = 0.f;    // this warpgroup's share of the row sum
       for (int j = 0; j < it.n; ++j) {
         const int jb = it.j_start + j;
         const int gj = g + j;
         const int b = gj & 1;
-        const uint32_t tS = tmem + C::kColS + 128 * b + lane_off;
-        if (!(ok = mbar_wait_warp(bar(bar_s256(b)), (gj >> 1) & 1, ab, kS2SmS))) break;
-        tc_fence_after();
-        uint32_t u[128];
-        tmem_ld128(tS, u);
+        const uint32_t tS = tmem + C::kColS + 128 * b + 64u * wg + lane_off;
         const bool masked = (CAUSAL && (jb == qi || jb * kBlockN < qi * kBlockM + kBlockM - 1 - p.window)) ||
                             ((jb + 1) * kBlockN > p.N) || p.alibi != nullptr;
-        if (masked) {
-          const int key0 = jb * kBlockN;
-          const int hi = (CAUSAL ? min(row + 1, p.N) : p.N) - key0;
-          const int lo = CAUSAL ? row - p.window - key0 : 0;
-          if (p.alibi != nullptr) {
-            const float sl2 = p.alibi[bh % p.H] * 1.4426950408889634f;
-            const float dk = static_cast<float>(key0 - row);
+        uint32_t u[64];
+        float mt = -INFINITY;
+        const bool ws = mbar_wait_warp(bar(bar_s256(b)), (gj >> 1) & 1, ab, kS2SmS);
+        if (ws) {
+          tc_fence_after();
+          tmem_ld64(tS, u);
+          if (masked) {
+            const int key0 = jb * kBlockN + 64 * wg;
+            const int hi = (CAUSAL ? min(row + 1, p.N) : p.N) - key0;
+            const int lo = CAUSAL ? row - p.window - key0 : 0;
+            if (p.alibi != nullptr) {
+              const float sl2 = p.alibi[bh % p.H] * 1.4426950408889634f;
+              const float dk = static_cast<float>(key0 - row);
 #pragma unroll
-            for (int i = 0; i < 128; ++i) {
-              const bool vis = i >= lo && i < hi;
-              const float bias = -sl2 * fabsf(dk + static_cast<float>(i));
-              u[i] = __float_as_uint(vis ? fmaf(__uint_as_float(u[i]), c, bias) : -INFINITY);
-            }
-          } else {
+              for (int i = 0; i < 64; ++i) {
+                const bool vis = i >= lo && i < hi;
+                const float bias = -sl2 * fabsf(dk + static_cast<float>(i));
+                u[i] = __float_as_uint(vis ? fmaf(__uint_as_float(u[i]), c, bias) : -INFINITY);
+              }
+            } else {
 #pragma unroll
-            for (int i = 0; i < 128; ++i) {
-              const bool vis = i >= lo && i < hi;
-              u[i] = __float_as_uint(vis ? __uint_as_float(u[i]) * c : -INFINITY);
+              for (int i = 0; i < 64; ++i) {
+                const bool vis = i >= lo && i < hi;
+                u[i] = __float_as_uint(vis ? __uint_as_float(u[i]) * c : -INFINITY);
+              }
             }
           }
-        }
-        float mt;
-        {
-          float a[8];
+          float a8[8];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) a[q] = fmaxf(__uint_as_float(u[q]), __uint_as_float(u[8 + q]));
+          for (int q = 0; q < 8; ++q) a8[q] = fmaxf(__uint_as_float(u[q]), __uint_as_float(u[8 + q]));
 #pragma unroll
-          for (int i = 16; i < 128; i += 16) {
+          for (int i = 16; i < 64; i += 16) {
 #pragma unroll
             for (int q = 0; q < 8; ++q)
-              a[q] = max3f(a[q], __uint_as_float(u[i + q]), __uint_as_float(u[i + 8 + q]));
+              a8[q] = max3f(a8[q], __uint_as_float(u[i + q]), __uint_as_float(u[i + 8 + q]));
           }
-          mt = max3f(max3f(a[0], a[1], a[2]), max3f(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+          mt = max3f(max3f(a8[0], a8[1], a8[2]), max3f(a8[3], a8[4], a8[5]), fmaxf(a8[6], a8[7]));
           if (!masked) mt *= c;
+          red_at(b, wg) = mt;
         }
-        const float m_new = fmaxf(m_use, mt);
+        // both warps of the row pair leave together if either wait failed
+        if (!(ok = named_bar_and(pair_bar, 64, ws))) break;
+        const float m_new = fmaxf(m_use, fmaxf(mt, red_at(b, wg ^ 1)));
         const bool need = m_new > m_use + kRescaleTau;
         float alpha = 1.f;
         if (need) {
@@ -346,54 +361,47 @@ __global__ void __launch_bounds__(192, 1) fwd256_kernel(const __grid_constant__ 
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
         const uint64_t c2 = f2_pack(c, c);
         const uint64_t nm2 = f2_pack(neg_m, neg_m);
-        auto exp_half = [&](auto hc) {
-          constexpr int h = decltype(hc)::value;
-          if (masked) {
+        if (masked) {
 #pragma unroll
-            for (int i = 32 * h; i < 32 * h + 32; ++i) {
-              const float p0 = ex2_sfu(__uint_as_float(u[2 * i]) + neg_m);
-              const float p1 = ex2_sfu(__uint_as_float(u[2 * i + 1]) + neg_m);
-              acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
-              u[i] = pack_bf16x2(p0, p1);
-            }
-          } else {
-#pragma unroll
-            for (int i = 32 * h; i < 32 * h + 32; ++i) {
-              const uint64_t x2 =
-                  f2_fma(f2_pack(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1])), c2, nm2);
-              const uint64_t p2 = ((i & 7) < NPOLY) ? exp2_poly_f2<DEG>(x2) : exp2_sfu_f2(x2);
-              acc[i & 3] = f2_add(acc[i & 3], p2);
-              float p0, p1;
-              f2_unpack(p2, p0, p1);
-              u[i] = pack_bf16x2(p0, p1);
-            }
+          for (int i = 0; i < 32; ++i) {
+            const float p0 = ex2_sfu(__uint_as_float(u[2 * i]) + neg_m);
+            const float p1 = ex2_sfu(__uint_as_float(u[2 * i + 1]) + neg_m);
+            acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
+            u[i] = pack_bf16x2(p0, p1);
           }
-        };
-        exp_half(std::integral_constant<int, 0>{});
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1])), c2, nm2);
+            const uint64_t p2 = ((i & 7) < NPOLY) ? exp2_poly_f2<DEG>(x2) : exp2_sfu_f2(x2);
+            acc[i & 3] = f2_add(acc[i & 3], p2);
+            float p0, p1;
+            f2_unpack(p2, p0, p1);
+            u[i] = pack_bf16x2(p0, p1);
+          }
+        }
         tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+        bool wpv = true;
         if (j > 0) {
           // P(j-1) V must be done before O is rescaled or P(j) is released
-          if (!(ok = mbar_wait_warp(bar(kBarPV), (gj - 1) & 1, ab, kS2SmPv))) break;
-          tc_fence_after();
-          if (__any_sync(0xffffffffu, need)) {
+          wpv = mbar_wait_warp(bar(kBarPV), (gj - 1) & 1, ab, kS2SmPv);
+          if (wpv) {
+            tc_fence_after();
+            if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
-            for (int ch = 0; ch < D / 32; ++ch) {
-              uint32_t w[32];
-              tmem_ld32(tO + ch * 32, w);
+              for (int ch = 0; ch < 4; ++ch) {
+                uint32_t w[32];
+                tmem_ld32(tO + ch * 32, w);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
-              tmem_st32(tO + ch * 32, w);
+                for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
+                tmem_st32(tO + ch * 32, w);
+              }
             }
           }
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar(kBarP));
-        exp_half(std::integral_constant<int, 1>{});
-        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(bar(kBarPH));
+        if (wpv) mbar_arrive(bar(kBarP));
         float sum4[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -402,17 +410,25 @@ __global__ void __launch_bounds__(192, 1) fwd256_kernel(const __grid_constant__ 
           sum4[q] = lo + hi;
         }
         l = l * alpha + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
+        // a failed wait ends the loop at the next pair barrier or the epilogue's
+        ok = wpv;
       }
       g += it.n;
       if (ok) ok = mbar_wait_warp(bar(kBarPV), (g - 1) & 1, ab, kS2EpiPv);
-      ok = named_bar_and(1, 128, ok);
+      ok = named_bar_and(1, 256, ok);
       if (!ok) break;
       tc_fence_after();
-      // epilogue: O / l from TMEM straight to global memory (row r's 512 bytes)
-      const float inv_l = 1.f / l;
-      uint16_t* orow = p.o + (static_cast<size_t>(bh) * p.N + (row < p.N ? row : 0)) * D;
+      // row sum over both halves; the slot of the item's last tile is free
+      // (both warps read its maxima before the barrier above)
+      const int ls = (g - 1) & 1;
+      red_at(ls, wg) = l;
+      named_bar_sync(pair_bar, 64);
+      const float l_all = red_at(ls, 0) + red_at(ls, 1);
+      // epilogue: this warpgroup's 128 O columns / l from TMEM to global memory
+      const float inv_l = 1.f / l_all;
+      uint16_t* orow = p.o + (static_cast<size_t>(bh) * p.N + (row < p.N ? row : 0)) * D + 128 * wg;
 #pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
+      for (int ch = 0; ch < 4; ++ch) {
         uint32_t w[32];
         tmem_ld32(tO + ch * 32, w);
         uint32_t pk[16];
@@ -427,13 +443,13 @@ __global__ void __launch_bounds__(192, 1) fwd256_kernel(const __grid_constant__ 
       }
       tc_fence_before();
       mbar_arrive(bar(kBarOFree));
-      if (row < p.N) p.lse[static_cast<size_t>(bh) * p.N + row] = (m_use + log2f(l)) * 0.69314718055994531f;
+      if (wg == 0 && row < p.N)
+        p.lse[static_cast<size_t>(bh) * p.N + row] = (m_use + log2f(l_all)) * 0.69314718055994531f;
     }
   }
-
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
