@@ -100,11 +100,14 @@ def test_fwd_one_hot_values_recover_p(causal):
     assert_fwd_close(o, lse, o_ref, l_ref, "one-hot V")
 
 
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("causal", [False, True])
-def test_fwd_large_magnitude_exercises_rescale(causal):
+def test_fwd_large_magnitude_exercises_rescale(causal, d):
     """Q x 8 with a growing ramp: the running max moves by more than the
-    rescale threshold across tiles, so the O correction path runs."""
-    N, d = 1024, 64
+    rescale threshold across tiles, so the O correction path runs (at
+    d = 256 each of the two softmax warpgroups rescales its own O columns
+    after the pair has agreed on the row maximum)."""
+    N = 1024
     q, k, v = inputs.make_qkv(1, 2, N, d, seed=9)
     ramp = torch.linspace(0.2, 3.0, N)[None, None, :, None]
     q = (q.float() * 8.0).to(torch.bfloat16)
