@@ -10,13 +10,15 @@
 // Q, dO, K, V tiles are 64 KB each.  So the work is split three ways; every
 // kernel sums in a fixed order, and the result is reproducible:
 //
-//   kv kernel   one CTA per (K/V head, key block of 128, head-dim half h):
-//               K_j, V_j resident (64 KB each); query blocks of 64 rows
-//               stream past; per block S^T and dP^T over the full d
-//               (M = 128 keys, N = 64 queries), then dV_h += P^T dO[:, h]
-//               and dK_h += dS^T Q[:, h] (N = 128).  TMEM: S^T 64, dP^T 64,
-//               dV_h 128, dK_h 128 columns.  The two halves h recompute the
-//               same S^T and dP^T: 1.5x the minimal tensor work.
+//   kv kernel   two CTAs per (K/V head, key block of 128): role r = 0
+//               computes dV, role r = 1 dK, each over the full d (N = 256
+//               products, one 256-column TMEM accumulator).  Query blocks of
+//               64 rows stream past; per block both roles compute S^T
+//               (M = 128 keys, N = 64 queries, K_j resident); the dV role
+//               then dV += P^T dO, the dK role dP^T = V dO^T (V_j resident
+//               in that role only), dS and dK += dS^T Q.  TMEM: S^T 64,
+//               dP^T 64 (dK role), accumulator 256 columns.  S^T is computed
+//               twice: 1.25x the minimal tensor work of dK, dV.
 //   dq kernel   one CTA per (query head, query block of 128): Q_i, dO_i
 //               resident (64 KB each); key blocks of 64 stream past; per
 //               block S and dP (N = 64 keys), dQ += dS K_j (N = 256).
@@ -368,8 +370,7 @@ struct Kv256 {
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColA = 0;      // S^T / P^T (64 query columns)
   static constexpr uint32_t kColB = 64;     // dP^T / dS^T
-  static constexpr uint32_t kColDV = 128;   // dV_h: 128 columns
-  static constexpr uint32_t kColDK = 256;   // dK_h
+  static constexpr uint32_t kColAcc = 128;  // dV (role 0) or dK (role 1): 256 columns
 };
 static_assert(Kv256::kSmemBytes <= 232448, "d = 256 dK/dV kernel shared memory");
 
@@ -400,9 +401,9 @@ __global__ void __launch_bounds__(320, 1) bwd_kv256_kernel(const __grid_constant
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // CTA -> (K/V head, split, key block j, head-dim half h); head-major
+  // CTA -> (K/V head, split, key block j, role h: 0 dV, 1 dK); head-major
   // non-causal; causal: longest first within groups of K/V heads
-  // (causal_kv_order), the two halves of a key block adjacent
+  // (causal_kv_order), the two roles of a key block adjacent
   const int h = blockIdx.x & 1;
   const int rest = blockIdx.x >> 1;
   int kvh, split, j;
@@ -461,10 +462,11 @@ __global__ void __launch_bounds__(320, 1) bwd_kv256_kernel(const __grid_constant
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_q64);
       tma_prefetch_desc(&p.tm_do64);
-      mbar_arrive_expect_tx(bar(B_KV), 2 * C::kTileKV);
+      // V_j only in the dK role (dP^T = V dO^T)
+      mbar_arrive_expect_tx(bar(B_KV), (h ? 2 : 1) * C::kTileKV);
       for (int pn = 0; pn < 4; ++pn) {
         tma_load_3d(kAddr + pn * kP128, &p.tm_k, bar(B_KV), pn * 64, j * 128, kvh);
-        tma_load_3d(vAddr + pn * kP128, &p.tm_v, bar(B_KV), pn * 64, j * 128, kvh);
+        if (h) tma_load_3d(vAddr + pn * kP128, &p.tm_v, bar(B_KV), pn * 64, j * 128, kvh);
       }
     }
     // L (log2 units, +inf past N) and D (0 past N) of the 64 queries of
@@ -528,7 +530,7 @@ __global__ void __launch_bounds__(320, 1) bwd_kv256_kernel(const __grid_constant
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdescKK = idesc_bf16_f32(128, 64, false, false);    // S^T, dP^T: 64 queries
-      constexpr uint32_t kIdescTS = idesc_bf16_f32(128, 128, false, true);    // dV_h, dK_h: N = 128
+      constexpr uint32_t kIdescTS = idesc_bf16_f32(128, kD2, false, true);    // dV, dK: N = 256
       // A = 128 key rows (16 KB panels), B = 64 query rows (8 KB panels), K = 256
       auto gemm_kk = [&](uint32_t dcol, uint32_t a_addr, uint32_t b_addr) {
 #pragma unroll
@@ -538,12 +540,12 @@ __global__ void __launch_bounds__(320, 1) bwd_kv256_kernel(const __grid_constant
                      kk > 0 ? 1u : 0u);
       };
       // A = packed P^T / dS^T (queries 0..31 at a_col, 32..63 at a_col + 32),
-      // B = head-dim panels 2h, 2h + 1 of the 64 query rows (MN-major)
+      // B = all four head-dim panels of the 64 query rows (MN-major)
       auto gemm_ts = [&](uint32_t dcol, uint32_t a_col, uint32_t b_addr, bool acc) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_f16_ts(tmem + dcol, tmem + a_col + (kk < 2 ? kk * 8 : 32 + (kk - 2) * 8),
-                     smem_desc_sw128(b_addr + 2 * h * kP64 + kk * 2048, kP64, 1024), kIdescTS,
+                     smem_desc_sw128(b_addr + kk * 2048, kP64, 1024), kIdescTS,
                      (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(bar(B_KV), 0, ab, kK2MmaKV);
@@ -556,23 +558,32 @@ __global__ void __launch_bounds__(320, 1) bwd_kv256_kernel(const __grid_constant
         const int sq = idx % NQ, sd = idx % ND;
         if (!(ok = mbar_wait(bar(B_DF(sd)), (idx / ND) & 1, ab, kK2MmaQ))) break;
         tc_fence_after();
-        gemm_kk(C::kColB, vAddr, doAddr(sd));                    // dP^T = V dO^T
-        tc_commit(bar(B_DP));
+        if (h) {
+          gemm_kk(C::kColB, vAddr, doAddr(sd));                  // dP^T = V dO^T
+          tc_commit(bar(B_DP));
+          tc_commit(bar(B_DE(sd)));                              // dO_i is read for the last time
+        }
+        // dV role: P^T is in region A; dK role: the P phase has read S^T
         if (!(ok = mbar_wait(bar(B_P), idx & 1, ab, kK2MmaP))) break;
         tc_fence_after();
-        gemm_ts(C::kColDV, C::kColA, doAddr(sd), idx > 0);       // dV_h += P^T dO[:, h]
-        tc_commit(bar(B_DE(sd)));                                // dO_i is read for the last time
-        if (idx + 1 < n_it) {                                    // next S^T right behind dV
+        if (!h) {
+          gemm_ts(C::kColAcc, C::kColA, doAddr(sd), idx > 0);    // dV += P^T dO
+          tc_commit(bar(B_DE(sd)));                              // dO_i is read for the last time
+          tc_commit(bar(B_QE(sq)));                              // Q_i (S^T) and its L rows (P phase) too
+        }
+        if (idx + 1 < n_it) {                                    // next S^T into region A
           const int s1 = (idx + 1) % NQ;
           if (!(ok = mbar_wait(bar(B_QF(s1)), ((idx + 1) / NQ) & 1, ab, kK2MmaQ))) break;
           tc_fence_after();
           gemm_kk(C::kColA, kAddr, qAddr(s1));
           tc_commit(bar(B_S));
         }
-        if (!(ok = mbar_wait(bar(B_DS), idx & 1, ab, kK2MmaDS))) break;
-        tc_fence_after();
-        gemm_ts(C::kColDK, C::kColB, qAddr(sq), idx > 0);        // dK_h += dS^T Q[:, h]
-        tc_commit(bar(B_QE(sq)));
+        if (h) {
+          if (!(ok = mbar_wait(bar(B_DS), idx & 1, ab, kK2MmaDS))) break;
+          tc_fence_after();
+          gemm_ts(C::kColAcc, C::kColB, qAddr(sq), idx > 0);     // dK += dS^T Q
+          tc_commit(bar(B_QE(sq)));
+        }
       }
       tc_commit(bar(B_FINAL));
       tc_commit(bar(B_DRAIN));
@@ -632,11 +643,12 @@ __global__ void __launch_bounds__(320, 1) bwd_kv256_kernel(const __grid_constant
           p_rows(std::true_type{});
         else
           p_rows(std::false_type{});
-        tmem_st16(tS, pp);
+        if (!h) tmem_st16(tS, pp);   // P^T for dV; the dK role keeps P in registers only
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(B_P));
+      if (!h) continue;
       if (!(ok = mbar_wait_warp(bar(B_DP), idx & 1, ab, kK2SmDP))) break;
       tc_fence_after();
       uint32_t ds[16];
@@ -658,19 +670,20 @@ __global__ void __launch_bounds__(320, 1) bwd_kv256_kernel(const __grid_constant
     if (ok) ok = mbar_wait_warp(bar(B_FINAL), 0, ab, kK2Epi);
     ok = named_bar_and(1, 256, ok);
     if (ok) {
-      // dV_h, dK_h of this CTA's keys: wg 0 columns [0, 64) of the half, wg 1 [64, 128)
+      // dV (role 0) or dK (role 1, times scale) of this CTA's keys: wg 0
+      // columns [0, 128), wg 1 [128, 256)
       tc_fence_after();
-      const size_t g = (static_cast<size_t>(kvh) * p.N + (key_ok ? key : 0)) * kD2 + 128 * h;
+      const size_t g = (static_cast<size_t>(kvh) * p.N + (key_ok ? key : 0)) * kD2;
       const size_t kv_elems = static_cast<size_t>(p.BH / p.kv_group) * p.N * kD2;
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {      // 0: dV, 1: dK (times scale)
-        const uint32_t src = tmem + (which ? C::kColDK : C::kColDV) + lane_off;
+      {
+        const int which = h;
+        const uint32_t src = tmem + C::kColAcc + lane_off;
         uint16_t* dst = (which ? p.dk : p.dv) + g;
         const float mul = which ? p.scale : 1.f;
         float* part = p.kv_part + (static_cast<size_t>(split) * 2 + which) * kv_elems + g;
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int ch = wg * 2 + cc;
+        for (int cc = 0; cc < 4; ++cc) {
+          const int ch = wg * 4 + cc;
           uint32_t u[32];
           tmem_ld32(src + 32 * ch, u);
           if (p.kv_split > 1) {
