@@ -364,7 +364,10 @@ struct Kv256 {
   static constexpr int kOffL = kOffDO + kStagesD * kTileQ;       // + s * 256: L log2 e of 64 queries
   static constexpr int kOffDl = kOffL + kStagesQ * 256;          // + s * 256: D (with the Q stage)
   static constexpr int kOffBar = kOffDl + kStagesQ * 256;
-  static constexpr int kNumBars = 1 + 2 * kStagesQ + 2 * kStagesD + 6;
+  // The dV role has no V tile: its 64 KB hold two more dO stages (three in
+  // all); the dK role keeps one.
+  static constexpr int kStagesDV = 3;
+  static constexpr int kNumBars = 1 + 2 * kStagesQ + 2 * kStagesDV + 6;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
   static constexpr uint32_t kTmemCols = 512;
@@ -381,7 +384,7 @@ template <bool CAUSAL>
 __global__ void __launch_bounds__(320, 1) bwd_kv256_kernel(const __grid_constant__ BwdParams p) {
   using C = Kv256;
   constexpr int NQ = C::kStagesQ;
-  constexpr int ND = C::kStagesD;
+  constexpr int NDB = C::kStagesDV;   // dO barrier pairs (the deepest ring)
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   if (sbase & 1023u) {
@@ -393,8 +396,8 @@ __global__ void __launch_bounds__(320, 1) bwd_kv256_kernel(const __grid_constant
   auto B_QF = [](int s) { return 1 + s; };
   auto B_QE = [](int s) { return 1 + NQ + s; };
   auto B_DF = [](int s) { return 1 + 2 * NQ + s; };
-  auto B_DE = [](int s) { return 1 + 2 * NQ + ND + s; };
-  const int B_S = 1 + 2 * NQ + 2 * ND, B_DP = B_S + 1, B_P = B_S + 2, B_DS = B_S + 3, B_FINAL = B_S + 4,
+  auto B_DE = [](int s) { return 1 + 2 * NQ + NDB + s; };
+  const int B_S = 1 + 2 * NQ + 2 * NDB, B_DP = B_S + 1, B_P = B_S + 2, B_DS = B_S + 3, B_FINAL = B_S + 4,
             B_DRAIN = B_S + 5;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
@@ -429,7 +432,7 @@ __global__ void __launch_bounds__(320, 1) bwd_kv256_kernel(const __grid_constant
       mbar_init(bar(B_QF(s)), 1);
       mbar_init(bar(B_QE(s)), 1);
     }
-    for (int s = 0; s < ND; ++s) {
+    for (int s = 0; s < NDB; ++s) {
       mbar_init(bar(B_DF(s)), 1);
       mbar_init(bar(B_DE(s)), 1);
     }
@@ -453,7 +456,12 @@ __global__ void __launch_bounds__(320, 1) bwd_kv256_kernel(const __grid_constant
   const Abort ab{abort_flag, p.status};
   const uint32_t kAddr = sbase + C::kOffK, vAddr = sbase + C::kOffV;
   auto qAddr = [&](int s) -> uint32_t { return sbase + C::kOffQ + s * C::kTileQ; };
-  auto doAddr = [&](int s) -> uint32_t { return sbase + C::kOffDO + s * C::kTileQ; };
+  // dO stages: 1 in the dK role; 3 in the dV role, stages 1 and 2 in the V region
+  const int ND = h ? C::kStagesD : C::kStagesDV;
+  auto doAddr = [&](int s) -> uint32_t {
+    return sbase + (s == 0 ? C::kOffDO : C::kOffV + (s - 1) * C::kTileQ);
+  };
+  static_assert(2 * Kv256::kTileQ <= Kv256::kTileKV, "two dO stages fit in the V tile");
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
