@@ -608,15 +608,24 @@ def run_ours(args):
     burst_note = (f"{peak_src} bf16_tflops (burst: the timed region is short and the SM clock "
                   f"sampled during it is {clocks.get('sm_mhz')} of {clocks.get('sm_max_mhz')} MHz)")
     cz = "causal" if causal else "non-causal"
-    if BWD_MODE == "atomic":
+    if d == 256:
+        # one path at d = 256 (both modes): the dK/dV and dQ kernels; traffic
+        # is theirs summed while both captures match the current source
+        bwd_kernel = f"bwd_kv256_kernel<{cz}> + bwd_dq256_kernel<{cz}> (+ preprocess) in the timed call"
+        t_kv = profiled_traffic("bwd_kv256_kernel", w["name"], "bwd256")
+        t_dq = profiled_traffic("bwd_dq256_kernel", w["name"], "bwd256")
+        bwd_traffic = t_kv + t_dq if t_kv is not None and t_dq is not None else None
+    elif BWD_MODE == "atomic":
         bwd_kernel = f"bwd_main_kernel<{d}, {cz}> (+ preprocess and dQ postprocess launches in the timed call)"
+        bwd_traffic = profiled_traffic("bwd_main_kernel", w["name"], "bwd")
     else:
         main = "bwd_pair_kernel (CTA pairs)" if TUNING.get("bwd_pair") == 1 else f"bwd_main_kernel<{d}, {cz}, no dQ>"
         bwd_kernel = f"{main} + bwd_dq_kernel (+ preprocess) in the timed call"
+        bwd_traffic = None
     roof_bwd = None
     if not w["fwd_only"]:
         roof_bwd = roof(stages, per_stage, "bwd_bf16", bwd_kernel, bwd_bytes(B, H, N, d, H_kv), burst, burst_note,
-                        profiled_traffic("bwd_main_kernel", w["name"], "bwd") if BWD_MODE == "atomic" else None)
+                        bwd_traffic)
         roof_bwd["frac_sustained"] = roof_bwd["achieved"] / sustained
         roof_bwd["frac_nominal_2250"] = roof_bwd["achieved"] / 2250.0
     # the two-tile forward's grid: set explicitly, or (-1) the library's
